@@ -1,0 +1,6 @@
+"""fp64 CPU oracle for exact attention -- test infrastructure, never part of the product path."""
+from .attention import (attention_forward, attention_forward_online, attention_backward,
+                        attention_probs, attention_head_subset)
+
+__all__ = ["attention_forward", "attention_forward_online", "attention_backward",
+           "attention_probs", "attention_head_subset"]
