@@ -1,0 +1,167 @@
+"""exact_io_aware_43_b200 -- exact, IO-aware attention on B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libfattn.so`` (include/fattn.h).  The functions
+``fa_fwd``, ``fa_bwd``, ``fa_bwd_workspace_size``, ``fa_last_error``, ``fa_device_status`` have
+the same names and arguments as the C entry points (pointers as Python ints, streams as raw
+``cudaStream_t`` handles).  ``forward``/``backward``/``attention`` are conveniences that take
+torch tensors, allocate the outputs with torch (device memory and streams are the only things
+torch provides here) and call the same entry points.  There is no other code path: if the
+library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "lib", "libfattn.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "fattn.h")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_MISALIGNED, FA_ERR_CUDA, \
+    FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(7)
+
+_lib = None
+
+
+class FattnError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libfattn error {code}: {msg}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfattn.so (built in-tree by ``python -m exact_io_aware_43_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise FattnError(-1, f"{LIB_PATH} is missing; build it with "
+                             "`python -m exact_io_aware_43_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+    L.fa_fwd.restype = i
+    L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    L.fa_bwd_workspace_size.restype = sz
+    L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
+    L.fa_bwd.restype = i
+    L.fa_last_error.argtypes = []
+    L.fa_last_error.restype = ctypes.c_char_p
+    L.fa_device_status.argtypes = [vp]
+    L.fa_device_status.restype = i
+    L.fa_version.argtypes = []
+    L.fa_version.restype = i
+    _lib = L
+    return L
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/fattn.h declares."""
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fa_\w+)\s*\(", txt, flags=re.M)
+
+
+# ------------------------------------------------------------------ C entry points, same names
+def fa_last_error() -> str:
+    return lib().fa_last_error().decode()
+
+
+def _check(rc: int) -> int:
+    if rc != FA_OK:
+        raise FattnError(rc, fa_last_error())
+    return rc
+
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, stream) -> int:
+    return lib().fa_fwd(q, k, v, o, lse, B, H, N, d, int(causal), float(scale), stream)
+
+
+def fa_bwd_workspace_size(B, H, N, d) -> int:
+    return lib().fa_bwd_workspace_size(B, H, N, d)
+
+
+def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, workspace,
+           workspace_bytes, stream) -> int:
+    return lib().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, int(causal), float(scale),
+                        workspace, workspace_bytes, stream)
+
+
+def fa_device_status(stream=None) -> int:
+    return lib().fa_device_status(stream)
+
+
+def fa_version() -> int:
+    return lib().fa_version()
+
+
+# ------------------------------------------------------------------ torch conveniences
+def _stream_handle(t):
+    import torch
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    return tuple(q.shape)
+
+
+def _default_scale(d):
+    import numpy as np
+    return float(np.float32(1.0 / np.sqrt(np.float64(d))))
+
+
+def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
+    """O, L = attention(q, k, v) for contiguous bf16 CUDA tensors [B, H, N, d]."""
+    import torch
+    B, H, N, d = _shape(q)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or \
+                tuple(t.shape) != (B, H, N, d):
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors of one shape")
+    scale = _default_scale(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    L = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
+                  B, H, N, d, causal, scale, _stream_handle(q)))
+    return o, L
+
+
+def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
+             workspace=None, grads=None):
+    """dQ, dK, dV for contiguous bf16 CUDA tensors; ``workspace`` (uint8 CUDA tensor) optional."""
+    import torch
+    B, H, N, d = _shape(q)
+    scale = _default_scale(d) if scale is None else float(scale)
+    need = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    dq, dk, dv = grads
+    _check(fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                  do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                  B, H, N, d, causal, scale, workspace.data_ptr(), workspace.numel(),
+                  _stream_handle(q)))
+    return dq, dk, dv
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None):
+    """Differentiable attention (torch.autograd.Function over fa_fwd / fa_bwd)."""
+    import torch
+
+    class _Fn(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, q, k, v):
+            o, L = forward(q, k, v, causal, scale)
+            ctx.save_for_backward(q, k, v, o, L)
+            return o
+
+        @staticmethod
+        def backward(ctx, do):
+            q, k, v, o, L = ctx.saved_tensors
+            return backward(q, k, v, o, L, do.contiguous(), causal, scale)
+
+    return _Fn.apply(q, k, v)

@@ -1,0 +1,219 @@
+// fattn.cu -- host side of libfattn: argument checks, TMA descriptors, launches (C ABI in
+// include/fattn.h).  Every step of the attention computation runs in the kernels of fwd.cuh and
+// bwd.cuh; this file only validates, encodes descriptors and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fattn.h"
+#include "bwd.cuh"
+#include "fwd.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---- driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime)
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tiled map over a contiguous bf16 [BH, N, d] tensor: box = 64 columns (128 bytes, one swizzle
+// row) x `box_rows` rows x 1 head, 128-byte swizzle, zero fill past N.
+int make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(N) * cuuint64_t(d) * 2};
+  cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return FA_OK;
+}
+
+uint64_t wait_limit_ns() {
+  static uint64_t v = [] {
+    const char* e = getenv("FA_WAIT_LIMIT_NS");
+    uint64_t x = e ? strtoull(e, nullptr, 10) : 0;
+    return x ? x : uint64_t(2000000000ull);  // 2 s: far above any legitimate wait
+  }();
+  return v;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int H, int N, int d, float scale) {
+  if (B < 1 || H < 1 || N < 1)
+    return fail(FA_ERR_INVALID_ARG, "B, H and N must be >= 1 (got %d, %d, %d)", B, H, N);
+  if (d != 64 && d != 128 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dim d=%d is not supported (64, 128 or 256)", d);
+  if (!std::isfinite(scale) || !(scale > 0.f))
+    return fail(FA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  const long long bh = (long long)B * H;
+  if (bh > (1ll << 30) || (long long)N > (1ll << 30))
+    return fail(FA_ERR_INVALID_ARG, "B*H or N too large");
+  const long long blocks = bh * ((N + 127) / 128);
+  if (blocks > 0x7fffffffll) return fail(FA_ERR_INVALID_ARG, "problem too large for one grid");
+  return FA_OK;
+}
+
+int check_device() {
+  static thread_local int cached_dev = -1, cached_ok = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != cached_dev) {
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    cached_ok = (prop.major == 10 && prop.minor == 0);
+    cached_dev = dev;
+  }
+  if (!cached_ok) return fail(FA_ERR_UNSUPPORTED, "libfattn needs an sm_100 (B200) device");
+  return FA_OK;
+}
+
+template <typename K>
+int set_smem(K kernel, int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  return FA_OK;
+}
+
+template <int D, bool CAUSAL, int NQT>
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               fattn::FwdParams p, int BH, cudaStream_t st) {
+  using C = fattn::FwdCfg<D, NQT>;
+  auto kern = fattn::fa_fwd_kernel<D, CAUSAL, NQT>;
+  int rc = set_smem(kern, C::SMEM_BYTES);
+  if (rc) return rc;
+  p.nqb = (p.N + NQT * C::BM - 1) / (NQT * C::BM);
+  dim3 grid(unsigned(BH) * unsigned(p.nqb));
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fa_fwd launch");
+  return FA_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_last_error(void) { return g_msg; }
+
+int fa_version(void) { return 100; }
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+           int d, int causal, float scale, void* stream) {
+  g_msg[0] = 0;
+  if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID_ARG, "null tensor pointer");
+  int rc = check_common(B, H, N, d, scale);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return fail(FA_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+  if ((rc = check_device())) return rc;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if ((rc = make_map(&mq, q, BH, N, d, 128))) return rc;
+  if ((rc = make_map(&mk, k, BH, N, d, 128))) return rc;
+  if ((rc = make_map(&mv, v, BH, N, d, 128))) return rc;
+  fattn::FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.N = N;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.limit_ns = wait_limit_ns();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return causal ? launch_fwd<64, true, 2>(mq, mk, mv, p, BH, st)
+                  : launch_fwd<64, false, 2>(mq, mk, mv, p, BH, st);
+  if (d == 128)
+    return causal ? launch_fwd<128, true, 2>(mq, mk, mv, p, BH, st)
+                  : launch_fwd<128, false, 2>(mq, mk, mv, p, BH, st);
+  return causal ? launch_fwd<256, true, 1>(mq, mk, mv, p, BH, st)
+                : launch_fwd<256, false, 1>(mq, mk, mv, p, BH, st);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128 && d != 256)) return 0;
+  const size_t bh = size_t(B) * size_t(H);
+  const size_t npad = round_up(size_t(N), 128);
+  const size_t dq = round_up(bh * size_t(N) * size_t(d) * 4, 256);
+  const size_t rows = round_up(bh * npad * 4, 256);
+  return dq + 2 * rows;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal,
+           float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  g_msg[0] = 0;
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv)
+    return fail(FA_ERR_INVALID_ARG, "null tensor pointer");
+  int rc = check_common(B, H, N, d, scale);
+  if (rc) return rc;
+  for (const void* ptr : {q, k, v, o, static_cast<const void*>(lse), dO,
+                          static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv)})
+    if (!aligned16(ptr)) return fail(FA_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need)
+    return fail(FA_ERR_WORKSPACE, "workspace must be 16-byte aligned and >= %zu bytes", need);
+  if ((rc = check_device())) return rc;
+  return fattn_bwd_launch(q, k, v, o, lse, dO, dq, dk, dv, B * H, N, d, causal != 0, scale,
+                          workspace, wait_limit_ns(), static_cast<cudaStream_t>(stream));
+}
+
+int fa_device_status(void* stream) {
+  g_msg[0] = 0;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int h[2] = {0, 0};
+  e = cudaMemcpyFromSymbol(h, fattn::g_status, sizeof(h));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol");
+  if (h[0] != 0) {
+    int z[2] = {0, 0};
+    cudaMemcpyToSymbol(fattn::g_status, z, sizeof(z));
+    return fail(h[0], "a kernel abandoned a bounded wait (site %d)", h[1]);
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

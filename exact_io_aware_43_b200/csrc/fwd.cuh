@@ -1,0 +1,344 @@
+// fwd.cuh -- fused attention forward for sm_100a.
+//
+// One CTA owns NQT query tiles of 128 rows of one (batch, head) and streams every K_j, V_j tile
+// of 128 keys through a shared-memory ring (chipfoundryservices.com glossary "Flash Attention",
+// "Tiling Algorithm" steps 1-2; robocikowo.com "Flash Attention": a Q block is loaded once, then
+// the loop runs over the K, V blocks).  Per KV tile and query tile:
+//   S   = Q_t K_j^T                  tcgen05.mma, bf16 x bf16 -> fp32 in tensor memory (step 3)
+//   m   = max(m, rowmax(S*s))        one softmax thread owns one row (one TMEM lane)   (step 4)
+//   P~  = exp2(S*s*log2e - m)        rounded to bf16 and written back into tensor memory
+//   O  *= exp2(m_old - m_new)        rescale of the running output (robocikowo.com update rule)
+//   O  += P~ V_j                     tcgen05.mma with A = P~ from tensor memory         (step 5)
+// and after the last tile O /= l, L = (m + log2 l) ln 2 (step 6; L is kept for the backward).
+// The score tile lives only in tensor memory: the N x N matrix never reaches HBM
+// (systems-analysis.info "FlashAttention (PL)", "Scalanie operacji w jedno jadro CUDA").
+//
+// Warp roles: warps [0, 4*NQT) are the softmax warpgroups (warpgroup t owns query tile t),
+// warp 4*NQT issues TMA loads, warp 4*NQT+1 allocates tensor memory and issues the MMAs.
+// With NQT = 2 the two query tiles ping-pong: the tensor core works on one tile while the
+// softmax warpgroup of the other computes its exponentials.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fattn {
+
+struct FwdParams {
+  __nv_bfloat16* o;
+  float* lse;
+  int N;            // sequence length (queries = keys)
+  int nqb;          // query blocks (of NQT*128 rows) per head
+  float scale_log2; // scale * log2(e)
+  uint64_t limit_ns;
+};
+
+template <int D, int NQT>
+struct FwdCfg {
+  static constexpr int BM = 128;                 // query rows per tile (MMA M)
+  static constexpr int BN = 128;                 // keys per KV tile
+  static constexpr int KB = D / 64;              // 128-byte swizzle blocks across d
+  static constexpr int QTILE_BYTES = BM * D * 2;
+  static constexpr int KVTILE_BYTES = BN * D * 2;
+  static constexpr int STAGES = (D == 64) ? 4 : (D == 128 ? 2 : 1);
+  static constexpr int SOFTMAX_WARPS = 4 * NQT;
+  static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;
+  static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
+  static constexpr int THREADS = (SOFTMAX_WARPS + 2) * 32;
+  static constexpr int TMEM_S = 0;               // S_t at column t*BN (P_t aliases its first BN/2)
+  static constexpr int TMEM_O = NQT * BN;        // O_t at TMEM_O + t*D
+  static constexpr int TMEM_COLS = 512;
+  static_assert(NQT * (BN + D) <= TMEM_COLS, "tensor memory budget");
+  // shared memory map (offsets from a 1024-aligned base)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + NQT * QTILE_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * KVTILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + STAGES * KVTILE_BYTES;
+  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT], p_full[NQT],
+  //           o_done[NQT], drain
+  static constexpr int NBAR = 1 + 4 * STAGES + 3 * NQT + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem address + abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);   // Q, K both K-major
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);   // P (tmem), V MN-major
+};
+
+template <int D, bool CAUSAL, int NQT>
+__global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D, NQT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: (head, query block), heaviest query blocks first when causal
+  const int head = blockIdx.x / p.nqb;
+  const int qb_lin = blockIdx.x % p.nqb;
+  const int qb = CAUSAL ? (p.nqb - 1 - qb_lin) : qb_lin;
+  const int q0 = qb * NQT * C::BM;
+  const int n_kv_total = (p.N + C::BN - 1) / C::BN;
+  int nkv[NQT];
+  int J = 0;
+#pragma unroll
+  for (int t = 0; t < NQT; ++t) {
+    const int r0 = q0 + t * C::BM;
+    int n = 0;
+    if (r0 < p.N) n = CAUSAL ? min(n_kv_total, (r0 + C::BM - 1) / C::BN + 1) : n_kv_total;
+    nkv[t] = n;
+    J = max(J, n);
+  }
+
+  auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
+  const uint32_t BAR_Q = bar(0);
+  auto BAR_KF = [&](int s) { return bar(1 + s); };
+  auto BAR_KE = [&](int s) { return bar(1 + C::STAGES + s); };
+  auto BAR_VF = [&](int s) { return bar(1 + 2 * C::STAGES + s); };
+  auto BAR_VE = [&](int s) { return bar(1 + 3 * C::STAGES + s); };
+  auto BAR_SF = [&](int t) { return bar(1 + 4 * C::STAGES + t); };
+  auto BAR_PF = [&](int t) { return bar(1 + 4 * C::STAGES + NQT + t); };
+  auto BAR_OD = [&](int t) { return bar(1 + 4 * C::STAGES + 2 * NQT + t); };
+  const uint32_t BAR_DRAIN = bar(C::NBAR - 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  const Waiter W{abort_flag, p.limit_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR_Q, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(BAR_KF(s), 1);
+      mbar_init(BAR_KE(s), 1);
+      mbar_init(BAR_VF(s), 1);
+      mbar_init(BAR_VE(s), 1);
+    }
+    for (int t = 0; t < NQT; ++t) {
+      mbar_init(BAR_SF(t), 1);
+      mbar_init(BAR_PF(t), 4);
+      mbar_init(BAR_OD(t), 1);
+    }
+    mbar_init(BAR_DRAIN, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::PRODUCER_WARP) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int q_tiles = 0;
+      for (int t = 0; t < NQT; ++t) q_tiles += (nkv[t] > 0);
+      mbar_arrive_expect_tx(BAR_Q, q_tiles * C::QTILE_BYTES);
+      for (int t = 0; t < NQT; ++t) {
+        if (nkv[t] == 0) continue;
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_3d(sbase + C::OFF_Q + t * C::QTILE_BYTES + kb * (C::BM * 128), &tmQ, BAR_Q,
+                      kb * 64, q0 + t * C::BM, head);
+      }
+      int j = 0;
+      for (; j < J; ++j) {
+        const int s = j % C::STAGES;
+        const uint32_t ph = (j / C::STAGES) & 1;
+        if (!W.wait(BAR_KE(s), ph ^ 1, 1)) break;
+        mbar_arrive_expect_tx(BAR_KF(s), C::KVTILE_BYTES);
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_3d(sbase + C::OFF_K + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmK,
+                      BAR_KF(s), kb * 64, j * C::BN, head);
+        if (!W.wait(BAR_VE(s), ph ^ 1, 2)) {
+          ++j;  // the K load of tile j is in flight
+          break;
+        }
+        mbar_arrive_expect_tx(BAR_VF(s), C::KVTILE_BYTES);
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_3d(sbase + C::OFF_V + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmV,
+                      BAR_VF(s), kb * 64, j * C::BN, head);
+      }
+      if (W.aborted()) {
+        // drain: wait (bounded) for every load already issued before the CTA exits
+        W.drain(BAR_Q, 0);
+        for (int jj = max(0, j - C::STAGES); jj < j; ++jj) {
+          W.drain(BAR_KF(jj % C::STAGES), (jj / C::STAGES) & 1);
+          W.drain(BAR_VF(jj % C::STAGES), (jj / C::STAGES) & 1);
+        }
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = W.wait(BAR_Q, 0, 10);
+      for (int j = 0; ok && j < J; ++j) {
+        const int s = j % C::STAGES;
+        const uint32_t ph = (j / C::STAGES) & 1;
+        const uint32_t k_addr = sbase + C::OFF_K + s * C::KVTILE_BYTES;
+        const uint32_t v_addr = sbase + C::OFF_V + s * C::KVTILE_BYTES;
+        if (!(ok = W.wait(BAR_KF(s), ph, 11))) break;
+        for (int t = 0; t < NQT && ok; ++t) {
+          if (j >= nkv[t]) continue;
+          // S_t's columns hold P_t(j-1) until PV_t(j-1) has read it
+          if (j > 0 && !(ok = W.wait(BAR_OD(t), (j - 1) & 1, 12))) break;
+          tc_fence_after();
+          const uint32_t q_addr = sbase + C::OFF_Q + t * C::QTILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_ss(tmem + C::TMEM_S + t * C::BN, sdesc_sw128(q_addr + koff, 16, 1024),
+                   sdesc_sw128(k_addr + koff, 16, 1024), C::IDESC_S, kk > 0);
+          }
+          tc_commit(BAR_SF(t));
+        }
+        if (!ok) break;
+        tc_commit(BAR_KE(s));
+        if (!(ok = W.wait(BAR_VF(s), ph, 13))) break;
+        for (int t = 0; t < NQT && ok; ++t) {
+          if (j >= nkv[t]) continue;
+          if (!(ok = W.wait(BAR_PF(t), j & 1, 14))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk) {
+            // P~ is packed bf16: 16 keys = 8 columns; V rows (keys) are 128 B apart, so a
+            // 16-key slice is 2048 B further on; 64-wide d blocks are BN*128 B apart.
+            mma_ts(tmem + C::TMEM_O + t * D, tmem + C::TMEM_S + t * C::BN + kk * 8,
+                   sdesc_sw128(v_addr + kk * 2048, C::BN * 128, 1024), C::IDESC_PV,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(BAR_OD(t));
+        }
+        if (!ok) break;
+        tc_commit(BAR_VE(s));
+      }
+      // every MMA issued above has completed before the tensor memory is released
+      tc_commit(BAR_DRAIN);
+      W.drain(BAR_DRAIN, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warpgroups
+    const int t = warp >> 2;                  // query tile of this warpgroup
+    const int r = threadIdx.x & 127;          // row within the tile == TMEM lane
+    const int row = q0 + t * C::BM + r;       // query index
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + C::TMEM_S + t * C::BN;
+    const uint32_t tO = tmem + lane_base + C::TMEM_O + t * D;
+    const int n = nkv[t];
+    float m = -INFINITY;  // running max of s*log2e*scale
+    float l = 0.f;        // running sum of exponentials (relative to m)
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      if (!(ok = W.wait(BAR_SF(t), j & 1, 20))) break;
+      tc_fence_after();
+      uint32_t s[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_wait_ld(s[c]);
+      // mask keys past N and, on diagonal tiles, keys after the query (causal)
+      const int key0 = j * C::BN;
+      const int lim = CAUSAL ? min(row, p.N - 1) - key0 : (p.N - 1) - key0;  // last valid col
+      if (lim < C::BN - 1) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (32 * c + e > lim) s[c][e] = __float_as_uint(-INFINITY);
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
+      const float m_new = fmaxf(m, mx * p.scale_log2);
+      const float alpha = (m_new == m) ? 1.f : ex2(m - m_new);
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[c][2 * e]), p.scale_log2, -m_new));
+          const float p1 = ex2(fmaf(__uint_as_float(s[c][2 * e + 1]), p.scale_log2, -m_new));
+          sum += p0 + p1;
+          pk[e] = pack_bf16(p0, p1);
+        }
+        // 32 keys -> 16 packed columns; two chunks share one 32-column store
+        if (c & 1) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) s[c - 1][16 + e] = pk[e];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) s[c][e] = pk[e];
+        }
+      }
+      // P~ (bf16) over the first 64 columns of S_t
+      tmem_st32(tS + 0, s[0]);
+      tmem_st32(tS + 32, s[2]);
+      l = l * alpha + sum;
+      m = m_new;
+      if (j > 0) {
+        // O_t must hold PV_t(j-1) before it is rescaled
+        if (!(ok = W.wait(BAR_OD(t), (j - 1) & 1, 21))) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_wait_ld(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + 32 * c, o);
+          }
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR_PF(t));
+    }
+    if (ok && n > 0) {
+      // ---- epilogue: O / l -> bf16 -> global; L = (m + log2 l) * ln 2
+      ok = W.wait(BAR_OD(t), (n - 1) & 1, 22);
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        __nv_bfloat16* orow = p.o + (size_t(head) * p.N + row) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld(o);
+          uint4 pk[4];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pw[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l,
+                              __uint_as_float(o[2 * e + 1]) * inv_l);
+          if (row < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = pk[e];
+          }
+        }
+        if (row < p.N) p.lse[size_t(head) * p.N + row] = (m + lg2(l)) * 0.69314718055994531f;
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fattn

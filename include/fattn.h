@@ -1,0 +1,108 @@
+/*
+ * fattn.h -- C ABI of libfattn: exact, IO-aware scaled-dot-product attention on B200 (sm_100a).
+ *
+ * The operation (systems-analysis.info "FlashAttention (PL)", section "Problematyka standardowego
+ * mechanizmu uwagi"; chipfoundryservices.com glossary "Flash Attention", first paragraph):
+ *
+ *     O = softmax(scale * Q K^T [+ causal mask]) V,      L_i = ln sum_j exp(scale * q_i . k_j)
+ *
+ * computed tile by tile with the online-softmax recurrence (chipfoundryservices.com glossary,
+ * "Tiling Algorithm" steps 1-6; robocikowo.com "Flash Attention", the running max m and sum l and
+ * the update O <- rescale(O_prev, m_old, m_new) + exp(S_new - m_new) V_j), so the N x N score
+ * matrix is never written to device memory.  The backward recomputes P from the saved L instead
+ * of storing it (robocikowo.com "Flash Attention": backward by recomputation from O and L).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are DEVICE pointers, contiguous, row-major:
+ *      q, k, v, o, dO, dq, dk, dv : bfloat16 [B, H, N, d]   (element (b,h,n,c) at ((b*H+h)*N+n)*d+c)
+ *      lse                        : float32  [B, H, N]      natural-log logsumexp of the scaled
+ *                                                            scores of each query row
+ *  - Every pointer must be 16-byte aligned (the kernels read and write through the Tensor Memory
+ *    Accelerator); a misaligned pointer returns FA_ERR_MISALIGNED before any launch.
+ *  - d must be 64, 128 or 256; any N >= 1 is accepted (rows past N are masked, stores clipped).
+ *  - causal != 0 hides key j from query i when j > i (N_q = N_k, so both alignments agree).
+ *  - scale is the factor applied to q.k (1/sqrt(d) in the usual use); it must be finite and > 0.
+ *  - The caller owns and allocates every buffer, including the backward workspace; the library
+ *    allocates no device memory on these paths.  It keeps only host-side caches (device
+ *    attributes, resolved driver entry points).
+ *  - stream is a cudaStream_t (NULL = legacy default stream).  All work is enqueued
+ *    asynchronously on it; no call synchronises the host.
+ *  - Return value: FA_OK (0) or an fa_status code.  Argument errors are detected on the host
+ *    before anything is launched; a failed launch returns FA_ERR_CUDA.  fa_last_error() gives a
+ *    message for the last non-OK status returned on the calling thread.
+ *  - Every wait inside the kernels is bounded in time.  If one ever expires (it does not in
+ *    correct operation), the kernel records FA_ERR_TIMEOUT in a device status word and returns
+ *    instead of hanging; fa_device_status() reads and clears that word.
+ */
+#ifndef FATTN_H_
+#define FATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null pointer, B/H/N < 1, non-finite or non-positive scale, size overflow */
+  FA_ERR_UNSUPPORTED = 2, /* d not in {64, 128, 256}, or no sm_100 device current */
+  FA_ERR_MISALIGNED = 3,  /* a tensor pointer is not 16-byte aligned */
+  FA_ERR_CUDA = 4,        /* a CUDA runtime or driver call failed (message in fa_last_error) */
+  FA_ERR_TIMEOUT = 5,     /* a kernel gave up on a bounded wait (reported by fa_device_status) */
+  FA_ERR_WORKSPACE = 6    /* workspace pointer null/misaligned or smaller than fa_bwd_workspace_size */
+} fa_status;
+
+/*
+ * fa_fwd -- forward pass.  Writes o = softmax(scale*q k^T [masked]) v (bf16, rounded once from
+ * the fp32 accumulator after the final division by the row sum, "Tiling Algorithm" step 6) and
+ * lse = m + ln l per query row (fp32; robocikowo.com: L is kept for the backward).
+ * Inputs q, k, v are read only.  o and lse are fully overwritten.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for this shape:
+ * an fp32 dQ accumulator [B,H,N,d] plus two fp32 row vectors [B,H,roundup(N,128)]
+ * (the logsumexp in base 2 and D_i = sum_c dO_ic O_ic).  Returns 0 for invalid sizes.
+ * The workspace is O(N) per head: no N x N buffer exists on any path.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * fa_bwd -- backward pass.  Given the forward's inputs, its outputs o and lse, and the upstream
+ * gradient dO, writes dq, dk, dv (bf16, overwritten, never accumulated into).  P is recomputed
+ * from lse (robocikowo.com "Flash Attention": backward by recomputation); then
+ *   dV = P^T dO, dP = dO V^T, D = rowsum(dO * o), dS = P * (dP - D), dQ = scale dS K,
+ *   dK = scale dS^T Q.
+ * o and lse must come from fa_fwd on the same q, k, v, causal and scale.
+ * workspace: device pointer, 16-byte aligned, at least fa_bwd_workspace_size(B,H,N,d) bytes,
+ * owned by the caller; its contents on entry are ignored and on exit are unspecified.
+ * Calls that share a workspace must not overlap on the GPU.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv,
+           int B, int H, int N, int d, int causal, float scale,
+           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Message for the last non-OK status returned on this host thread ("" if none). */
+const char* fa_last_error(void);
+
+/*
+ * fa_device_status -- synchronises `stream`, then reads and clears the device status word of
+ * the current device.  Returns FA_OK, FA_ERR_TIMEOUT if a kernel abandoned a bounded wait since
+ * the last call, or FA_ERR_CUDA if the synchronisation itself failed.
+ */
+int fa_device_status(void* stream);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FATTN_H_ */
