@@ -1,5 +1,486 @@
+// bwd.cuh -- attention backward for sm_100a, by recomputation (robocikowo.com "Flash Attention":
+// the backward recomputes the attention matrix from the saved O and L instead of storing it).
+//
+// Three kernels on the caller's stream:
+//   fa_bwd_pre_kernel   D_i = sum_c dO_ic O_ic, L2_i = L_i log2(e) (padded rows: +inf, 0),
+//                       and zeroes the fp32 dQ accumulator.                         (HBM bound)
+//   fa_bwd_kernel       one CTA per (head, block of 128 keys [, 128-wide slice of d]): K_j, V_j
+//                       stay in shared memory while the CTA loops over 64-query blocks i:
+//                         S^T  = K_j Q_i^T               tcgen05.mma -> TMEM (keys on lanes)
+//                         P^T  = exp2(S^T s log2e - L2_i)   recomputed from L
+//                         dV  += P^T dO_i                A = P^T (bf16, TMEM)
+//                         dP^T = V_j dO_i^T
+//                         dS^T = P^T * (dP^T - D_i)
+//                         dK  += dS^T Q_i                A = dS^T (bf16, TMEM)
+//                         dQ_i^T += K_j^T dS^T           -> fp32 reduction into the accumulator
+//                       dK is scaled by s in the epilogue, dQ when it is reduced.
+//   fa_bwd_post_kernel  dq = bf16(dQ accumulator).
+// No N x N buffer exists: the score and probability tiles live in tensor memory.
+//
+// Warp roles of fa_bwd_kernel: warps 0-3 compute P and dS (thread = key row = TMEM lane),
+// warps 4-7 drain dQ^T from tensor memory into the accumulator, warp 8 issues TMA loads,
+// warp 9 allocates tensor memory and issues the MMAs.
 #pragma once
+
 #include "sm100.cuh"
-static int fattn_bwd_launch(const void*, const void*, const void*, const void*, const float*,
-                            const void*, void*, void*, void*, int, int, int, bool, float, void*,
-                            uint64_t, cudaStream_t) { return 2; }
+
+namespace fattn {
+
+struct BwdParams {
+  const __nv_bfloat16* o;
+  const __nv_bfloat16* dO;
+  const float* lse;
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  float* dq_acc;   // [BH, N, D] fp32
+  float* L2;       // [BH, Npad] fp32: lse * log2(e), +inf on padded rows
+  float* Drow;     // [BH, Npad] fp32: rowsum(dO * O), 0 on padded rows
+  int BH;
+  int N;
+  int Npad;        // N rounded up to 128
+  int nkb;         // key blocks of 128 per head
+  float scale;
+  float scale_log2;
+  uint64_t limit_ns;
+};
+
+// ------------------------------------------------------------------------------------------
+// preprocess: D, L2, zero dQ accumulator
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
+  constexpr int G = D / 8;  // lanes per row, 8 bf16 (16 bytes) each
+  const long long total_rows = (long long)p.BH * p.Npad;
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long nthreads = (long long)gridDim.x * blockDim.x;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane % G;
+  constexpr int ROWS_PER_WARP = 32 / G;
+  // rows: D and L2.  The loop bound is warp-uniform so the shuffles see the whole warp.
+  const long long warp_id = tid >> 5;
+  const long long nwarps = nthreads >> 5;
+  for (long long rb = warp_id * ROWS_PER_WARP; rb < total_rows; rb += nwarps * ROWS_PER_WARP) {
+    const long long r = rb + lane / G;
+    const bool in = r < total_rows;
+    const int head = in ? int(r / p.Npad) : 0;
+    const int q = in ? int(r % p.Npad) : p.N;
+    float acc = 0.f;
+    if (q < p.N) {
+      const size_t off = (size_t(head) * p.N + q) * D + sub * 8;
+      const uint4 a = *reinterpret_cast<const uint4*>(p.o + off);
+      const uint4 b = *reinterpret_cast<const uint4*>(p.dO + off);
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x = __bfloat1622float2(a2[e]);
+        const float2 y = __bfloat1622float2(b2[e]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+    }
+#pragma unroll
+    for (int w = G / 2; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
+    if (in && sub == 0) {
+      p.Drow[r] = acc;
+      p.L2[r] = (q < p.N) ? p.lse[size_t(head) * p.N + q] * 1.4426950408889634f : INFINITY;
+    }
+  }
+  // zero the dQ accumulator (its size is a multiple of 4 floats: D >= 64)
+  const long long n4 = (long long)p.BH * p.N * D / 4;
+  float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
+  for (long long i = tid; i < n4; i += nthreads) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ------------------------------------------------------------------------------------------
+// postprocess: dq = bf16(accumulator)
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restrict__ acc,
+                                                          __nv_bfloat16* __restrict__ dq,
+                                                          long long n8) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long nthreads = (long long)gridDim.x * blockDim.x;
+  for (long long i = tid; i < n8; i += nthreads) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    uint4 o;
+    o.x = pack_bf16(a.x, a.y);
+    o.y = pack_bf16(a.z, a.w);
+    o.z = pack_bf16(b.x, b.y);
+    o.w = pack_bf16(b.z, b.w);
+    reinterpret_cast<uint4*>(dq)[i] = o;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// main backward kernel
+// ------------------------------------------------------------------------------------------
+template <int D>
+struct BwdCfg {
+  static constexpr int BC = 128;                  // keys per CTA (MMA M for S^T, dV, dK)
+  static constexpr int BR = 64;                   // queries per inner step
+  static constexpr int DO = D > 128 ? 128 : D;    // width of the dK/dV/dQ slice of this CTA
+  static constexpr int NSL = D / DO;              // slices of d (CTAs per key block)
+  static constexpr int KB = D / 64;               // 128-byte swizzle blocks across d
+  static constexpr int KV_BLK = BC * 128;         // bytes of one 64-column block of K_j / V_j
+  static constexpr int Q_BLK = BR * 128;          // bytes of one 64-column block of Q_i / dO_i
+  static constexpr int KV_BYTES = KB * KV_BLK;
+  static constexpr int Q_BYTES = KB * Q_BLK;
+  static constexpr int STAGES = D == 64 ? 3 : (D == 128 ? 2 : 1);
+  static constexpr int THREADS = 320;
+  static constexpr int DQ_WARP0 = 4;
+  static constexpr int PRODUCER_WARP = 8;
+  static constexpr int MMA_WARP = 9;
+  // tensor memory columns
+  static constexpr int T_S = 0, T_DP = 64, T_P = 128, T_DS = 160, T_DQ = 192, T_DV = 256,
+                       T_DK = 256 + DO;
+  static constexpr int TMEM_COLS = (T_DK + DO) <= 256 ? 256 : 512;
+  // shared memory map
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_BYTES;
+  static constexpr int OFF_Q = OFF_V + KV_BYTES;                 // STAGES x Q_i
+  static constexpr int OFF_DO = OFF_Q + STAGES * Q_BYTES;        // STAGES x dO_i
+  static constexpr int OFF_DS = OFF_DO + STAGES * Q_BYTES;       // dS^T [128 keys][64 q] bf16
+  static constexpr int OFF_ROWS = OFF_DS + BC * BR * 2;          // STAGES x (L2[64], D[64])
+  static constexpr int OFF_BAR = OFF_ROWS + STAGES * 2 * BR * 4;
+  // barriers: kv_full, q_full[S], q_empty[S], s_full, s_free, dp_full, dp_free, p_full,
+  //           ds_full, dv_done, dq_full, dq_empty, drain
+  static constexpr int NBAR = 1 + 2 * STAGES + 11;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t IDESC_ST = idesc_bf16_f32(BC, BR, 0, 0);  // S^T, dP^T
+  static constexpr uint32_t IDESC_KV = idesc_bf16_f32(BC, DO, 0, 1);  // dV, dK (A in TMEM)
+  static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(DO, BR, 1, 1);  // dQ^T = K^T dS^T
+};
+
+__device__ __forceinline__ void red_add_f32(float* addr, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                  const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: (head, key block j, d slice); key blocks with more queries first
+  const int per_head = p.nkb * C::NSL;
+  const int head = blockIdx.x / per_head;
+  const int rem = blockIdx.x % per_head;
+  const int j = rem / C::NSL;
+  const int slice = rem % C::NSL;
+  const int k0 = j * C::BC;
+  const int nqblk = (p.N + C::BR - 1) / C::BR;
+  const int i_start = CAUSAL ? (k0 / C::BR) : 0;
+  const int nit = nqblk - i_start;  // >= 1
+
+  auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
+  const uint32_t BAR_KV = bar(0);
+  auto BAR_QF = [&](int s) { return bar(1 + s); };
+  auto BAR_QE = [&](int s) { return bar(1 + C::STAGES + s); };
+  const int b0 = 1 + 2 * C::STAGES;
+  const uint32_t BAR_SF = bar(b0 + 0), BAR_SFREE = bar(b0 + 1), BAR_DPF = bar(b0 + 2),
+                 BAR_DPFREE = bar(b0 + 3), BAR_PF = bar(b0 + 4), BAR_DSF = bar(b0 + 5),
+                 BAR_DVD = bar(b0 + 6), BAR_DQF = bar(b0 + 7), BAR_DQE = bar(b0 + 8),
+                 BAR_DRAIN = bar(b0 + 9);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  const Waiter W{abort_flag, p.limit_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR_KV, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(BAR_QF(s), 1);
+      mbar_init(BAR_QE(s), 1);
+    }
+    mbar_init(BAR_SF, 1);
+    mbar_init(BAR_SFREE, 4);
+    mbar_init(BAR_DPF, 1);
+    mbar_init(BAR_DPFREE, 4);
+    mbar_init(BAR_PF, 4);
+    mbar_init(BAR_DSF, 4);
+    mbar_init(BAR_DVD, 1);
+    mbar_init(BAR_DQF, 1);
+    mbar_init(BAR_DQE, 4);
+    mbar_init(BAR_DRAIN, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const float* rows_smem = reinterpret_cast<const float*>(smem + C::OFF_ROWS);
+
+  if (warp == C::PRODUCER_WARP) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      mbar_arrive_expect_tx(BAR_KV, 2 * C::KV_BYTES);
+      for (int kb = 0; kb < C::KB; ++kb) {
+        tma_load_3d(sbase + C::OFF_K + kb * C::KV_BLK, &tmK, BAR_KV, kb * 64, k0, head);
+        tma_load_3d(sbase + C::OFF_V + kb * C::KV_BLK, &tmV, BAR_KV, kb * 64, k0, head);
+      }
+      int it = 0;
+      for (; it < nit; ++it) {
+        const int i = i_start + it;
+        const int s = it % C::STAGES;
+        if (!W.wait(BAR_QE(s), ((it / C::STAGES) & 1) ^ 1, 31)) break;
+        mbar_arrive_expect_tx(BAR_QF(s), 2 * C::Q_BYTES + 2 * C::BR * 4);
+        for (int kb = 0; kb < C::KB; ++kb) {
+          tma_load_3d(sbase + C::OFF_Q + s * C::Q_BYTES + kb * C::Q_BLK, &tmQ, BAR_QF(s), kb * 64,
+                      i * C::BR, head);
+          tma_load_3d(sbase + C::OFF_DO + s * C::Q_BYTES + kb * C::Q_BLK, &tmdO, BAR_QF(s),
+                      kb * 64, i * C::BR, head);
+        }
+        const size_t roff = size_t(head) * p.Npad + size_t(i) * C::BR;
+        bulk_load(sbase + C::OFF_ROWS + s * 2 * C::BR * 4, p.L2 + roff, C::BR * 4, BAR_QF(s));
+        bulk_load(sbase + C::OFF_ROWS + s * 2 * C::BR * 4 + C::BR * 4, p.Drow + roff, C::BR * 4,
+                  BAR_QF(s));
+      }
+      if (W.aborted()) {
+        W.drain(BAR_KV, 0);
+        for (int jj = max(0, it - C::STAGES); jj < it; ++jj)
+          W.drain(BAR_QF(jj % C::STAGES), (jj / C::STAGES) & 1);
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t k_addr = sbase + C::OFF_K, v_addr = sbase + C::OFF_V;
+      const uint32_t ds_addr = sbase + C::OFF_DS;
+      auto issue_st = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
+        // [S^T | dP^T] (128 x 64) = A (128 keys x D) * B (64 queries x D)^T, both K-major
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (kk >> 2) * C::KV_BLK + (kk & 3) * 32;
+          const uint32_t kb = (kk >> 2) * C::Q_BLK + (kk & 3) * 32;
+          mma_ss(tmem + d_col, sdesc_sw128(a_base + ka, 16, 1024),
+                 sdesc_sw128(b_base + kb, 16, 1024), C::IDESC_ST, kk > 0);
+        }
+      };
+      auto issue_kv = [&](uint32_t d_col, uint32_t a_col, uint32_t b_base, bool acc) {
+        // [dV | dK] (128 x DO) += A (tmem, 128 keys x 64 queries) * B (DO x 64 queries, MN-major)
+#pragma unroll
+        for (int kk = 0; kk < C::BR / 16; ++kk)
+          mma_ts(tmem + d_col, tmem + a_col + kk * 8,
+                 sdesc_sw128(b_base + slice * 2 * C::Q_BLK + kk * 2048, C::Q_BLK, 1024),
+                 C::IDESC_KV, (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = W.wait(BAR_KV, 0, 40);
+      if (ok) ok = W.wait(BAR_QF(0), 0, 41);
+      if (ok) {
+        tc_fence_after();
+        issue_st(C::T_S, k_addr, sbase + C::OFF_Q);
+        tc_commit(BAR_SF);
+        issue_st(C::T_DP, v_addr, sbase + C::OFF_DO);
+        tc_commit(BAR_DPF);
+      }
+      for (int it = 0; ok && it < nit; ++it) {
+        const int s = it % C::STAGES;
+        const int sn = (it + 1) % C::STAGES;
+        const uint32_t q_addr = sbase + C::OFF_Q + s * C::Q_BYTES;
+        const uint32_t do_addr = sbase + C::OFF_DO + s * C::Q_BYTES;
+        // dV += P^T dO_i
+        if (!(ok = W.wait(BAR_PF, it & 1, 42))) break;
+        tc_fence_after();
+        issue_kv(C::T_DV, C::T_P, do_addr, it > 0);
+        tc_commit(BAR_DVD);
+        // S^T for the next query block as soon as its tile and the S^T columns are free.  With a
+        // single stage the next tile can only arrive after this one is released, further down.
+        const bool more = it + 1 < nit;
+        auto issue_next_st = [&]() -> bool {
+          if (!W.wait(BAR_QF(sn), ((it + 1) / C::STAGES) & 1, 43)) return false;
+          if (!W.wait(BAR_SFREE, it & 1, 44)) return false;
+          tc_fence_after();
+          issue_st(C::T_S, k_addr, sbase + C::OFF_Q + sn * C::Q_BYTES);
+          tc_commit(BAR_SF);
+          return true;
+        };
+        if (more && C::STAGES > 1 && !(ok = issue_next_st())) break;
+        // dK += dS^T Q_i ; dQ_i^T = K_j^T dS^T
+        if (!(ok = W.wait(BAR_DSF, it & 1, 45))) break;
+        if (it > 0 && !(ok = W.wait(BAR_DQE, (it - 1) & 1, 46))) break;
+        tc_fence_after();
+        issue_kv(C::T_DK, C::T_DS, q_addr, it > 0);
+#pragma unroll
+        for (int kk = 0; kk < C::BC / 16; ++kk)
+          mma_ss(tmem + C::T_DQ,
+                 sdesc_sw128(k_addr + slice * 2 * C::KV_BLK + kk * 2048, C::KV_BLK, 1024),
+                 sdesc_sw128(ds_addr + kk * 2048, C::Q_BLK, 1024), C::IDESC_DQ, kk > 0);
+        tc_commit(BAR_DQF);
+        tc_commit(BAR_QE(s));
+        if (more) {
+          if (C::STAGES == 1 && !(ok = issue_next_st())) break;
+          if (!(ok = W.wait(BAR_DPFREE, it & 1, 47))) break;
+          tc_fence_after();
+          issue_st(C::T_DP, v_addr, sbase + C::OFF_DO + sn * C::Q_BYTES);
+          tc_commit(BAR_DPF);
+        }
+      }
+      tc_commit(BAR_DRAIN);
+      W.drain(BAR_DRAIN, 0);
+    }
+  } else if (warp < 4) {
+    // ---------------------------------------------------------------- P / dS warpgroup
+    const int r = threadIdx.x;               // key row within the block == TMEM lane
+    const int key = k0 + r;
+    const bool key_ok = key < p.N;
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    uint8_t* ds_row = smem + C::OFF_DS + r * 128;
+    bool ok = true;
+    for (int it = 0; it < nit; ++it) {
+      const int i = i_start + it;
+      const int s = it % C::STAGES;
+      const float* L2s = rows_smem + s * 2 * C::BR;
+      const float* Ds = L2s + C::BR;
+      if (!(ok = W.wait(BAR_SF, it & 1, 50))) break;
+      if (!(ok = W.wait(BAR_QF(s), (it / C::STAGES) & 1, 51))) break;
+      tc_fence_after();
+      uint32_t st[2][32];
+      tmem_ld32(tmem + lane_base + C::T_S, st[0]);
+      tmem_ld32(tmem + lane_base + C::T_S + 32, st[1]);
+      tmem_wait_ld(st[0]);
+      tmem_wait_ld(st[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR_SFREE);
+      // P^T = exp2(S^T s log2e - L2); zero for masked (causal key > query) and padded keys
+      float pr[64];
+      const int qbase = i * C::BR;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float x = fmaf(__uint_as_float(st[c >> 5][c & 31]), p.scale_log2, -L2s[c]);
+        bool valid = key_ok;
+        if (CAUSAL) valid = valid && (key <= qbase + c);
+        pr[c] = valid ? ex2(x) : 0.f;
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
+      // P^T columns are free once dV(it-1) has read them
+      if (it > 0 && !(ok = W.wait(BAR_DVD, (it - 1) & 1, 52))) break;
+      tc_fence_after();
+      tmem_st32(tmem + lane_base + C::T_P, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR_PF);
+      // dS^T = P^T * (dP^T - D)
+      if (!(ok = W.wait(BAR_DPF, it & 1, 53))) break;
+      tc_fence_after();
+      tmem_ld32(tmem + lane_base + C::T_DP, st[0]);
+      tmem_ld32(tmem + lane_base + C::T_DP + 32, st[1]);
+      tmem_wait_ld(st[0]);
+      tmem_wait_ld(st[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR_DPFREE);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float d0 = pr[2 * c] * (__uint_as_float(st[(2 * c) >> 5][(2 * c) & 31]) - Ds[2 * c]);
+        const float d1 =
+            pr[2 * c + 1] * (__uint_as_float(st[(2 * c + 1) >> 5][(2 * c + 1) & 31]) - Ds[2 * c + 1]);
+        pk[c] = pack_bf16(d0, d1);
+      }
+      // dS^T columns and the dS smem tile are free once dK(it-1) and dQ(it-1) have read them
+      if (it > 0 && !(ok = W.wait(BAR_DQF, (it - 1) & 1, 54))) break;
+      tc_fence_after();
+      tmem_st32(tmem + lane_base + C::T_DS, pk);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(ds_row + ((c ^ (r & 7)) << 4)) = v;
+      }
+      fence_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR_DSF);
+    }
+    if (ok) {
+      // ---- epilogue: dV, dK (x scale) -> bf16 -> global
+      ok = W.wait(BAR_DQF, (nit - 1) & 1, 55);
+      if (ok) {
+        tc_fence_after();
+        const size_t base = (size_t(head) * p.N + key) * D + slice * C::DO;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t col = which == 0 ? C::T_DV : C::T_DK;
+          const float mul = which == 0 ? 1.f : p.scale;
+          __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + base;
+#pragma unroll
+          for (int c = 0; c < C::DO / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_base + col + 32 * c, v);
+            tmem_wait_ld(v);
+            uint4 pkd[4];
+            uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              pw[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+            if (key_ok) {
+              uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) d4[e] = pkd[e];
+            }
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  } else if (warp < 8) {
+    // ---------------------------------------------------------------- dQ drain warpgroup
+    const int wq = warp - C::DQ_WARP0;
+    const uint32_t lane_base = uint32_t(wq * 32) << 16;
+    // dQ^T rows are d indices.  M = 128: lane i of warp w holds row 32w+i.  M = 64: rows
+    // 16w..16w+15 sit in lanes 0..15 of warp w's lane quarter; lanes 16..31 hold nothing.
+    const int drow = (C::DO == 128) ? (wq * 32 + lane) : (wq * 16 + lane);
+    const bool row_ok = (C::DO == 128) || (lane < 16);
+    for (int it = 0; it < nit; ++it) {
+      const int i = i_start + it;
+      if (!W.wait(BAR_DQF, it & 1, 60)) break;
+      tc_fence_after();
+      uint32_t v[2][32];
+      tmem_ld32(tmem + lane_base + C::T_DQ, v[0]);
+      tmem_ld32(tmem + lane_base + C::T_DQ + 32, v[1]);
+      tmem_wait_ld(v[0]);
+      tmem_wait_ld(v[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR_DQE);
+      if (row_ok) {
+        const int qbase = i * C::BR;
+        const int nq = min(C::BR, p.N - qbase);
+        float* dst = p.dq_acc + (size_t(head) * p.N + qbase) * D + slice * C::DO + drow;
+#pragma unroll
+        for (int c = 0; c < C::BR; ++c)
+          if (c < nq) red_add_f32(dst + size_t(c) * D, __uint_as_float(v[c >> 5][c & 31]) * p.scale);
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fattn

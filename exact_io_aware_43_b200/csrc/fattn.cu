@@ -133,6 +133,72 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+int sm_count() {
+  static thread_local int dev_cached = -1, n = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev != dev_cached) {
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    dev_cached = dev;
+  }
+  return n;
+}
+
+template <int D, bool CAUSAL>
+int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, cudaStream_t st) {
+  using C = fattn::BwdCfg<D>;
+  int rc;
+  CUtensorMap mq, mk, mv, mdo;
+  if ((rc = make_map(&mq, q, p.BH, p.N, D, C::BR))) return rc;
+  if ((rc = make_map(&mk, k, p.BH, p.N, D, C::BC))) return rc;
+  if ((rc = make_map(&mv, v, p.BH, p.N, D, C::BC))) return rc;
+  if ((rc = make_map(&mdo, p.dO, p.BH, p.N, D, C::BR))) return rc;
+  const int grid_ew = sm_count() * 8;
+  fattn::fa_bwd_pre_kernel<D><<<grid_ew, 256, 0, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fa_bwd preprocess launch");
+  auto kern = fattn::fa_bwd_kernel<D, CAUSAL>;
+  if ((rc = set_smem(kern, C::SMEM_BYTES))) return rc;
+  dim3 grid(unsigned(p.BH) * unsigned(p.nkb) * unsigned(C::NSL));
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fa_bwd launch");
+  const long long n8 = (long long)p.BH * p.N * D / 8;
+  fattn::fa_bwd_post_kernel<<<grid_ew, 256, 0, st>>>(p.dq_acc, p.dq, n8);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fa_bwd postprocess launch");
+  return FA_OK;
+}
+
+int bwd_dispatch(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv, int BH, int N, int d, bool causal,
+                 float scale, void* workspace, cudaStream_t st) {
+  fattn::BwdParams p{};
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.dO = static_cast<const __nv_bfloat16*>(dO);
+  p.lse = lse;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  const size_t npad = round_up(size_t(N), 128);
+  const size_t dq_bytes = round_up(size_t(BH) * size_t(N) * size_t(d) * 4, 256);
+  const size_t row_bytes = round_up(size_t(BH) * npad * 4, 256);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.dq_acc = reinterpret_cast<float*>(ws);
+  p.L2 = reinterpret_cast<float*>(ws + dq_bytes);
+  p.Drow = reinterpret_cast<float*>(ws + dq_bytes + row_bytes);
+  p.BH = BH;
+  p.N = N;
+  p.Npad = int(npad);
+  p.nkb = (N + 127) / 128;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.limit_ns = wait_limit_ns();
+  if (d == 64) return causal ? launch_bwd<64, true>(q, k, v, p, st) : launch_bwd<64, false>(q, k, v, p, st);
+  if (d == 128)
+    return causal ? launch_bwd<128, true>(q, k, v, p, st) : launch_bwd<128, false>(q, k, v, p, st);
+  return causal ? launch_bwd<256, true>(q, k, v, p, st) : launch_bwd<256, false>(q, k, v, p, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -197,8 +263,8 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if (!workspace || !aligned16(workspace) || workspace_bytes < need)
     return fail(FA_ERR_WORKSPACE, "workspace must be 16-byte aligned and >= %zu bytes", need);
   if ((rc = check_device())) return rc;
-  return fattn_bwd_launch(q, k, v, o, lse, dO, dq, dk, dv, B * H, N, d, causal != 0, scale,
-                          workspace, wait_limit_ns(), static_cast<cudaStream_t>(stream));
+  return bwd_dispatch(q, k, v, o, lse, dO, dq, dk, dv, B * H, N, d, causal != 0, scale,
+                      workspace, static_cast<cudaStream_t>(stream));
 }
 
 int fa_device_status(void* stream) {

@@ -1,0 +1,91 @@
+"""Backward parity: fa_bwd (CUDA, through the C ABI) against the fp64 oracle.
+
+The forward outputs fed to fa_bwd are the GPU's own (bf16 O, fp32 L), as a user would pass them;
+the oracle uses its own fp64 O and L (the tolerance covers the difference)."""
+import numpy as np
+import pytest
+
+import attn_inputs as ai
+from oracle import attention_backward, attention_forward
+from parity import assert_bwd, to_np
+from gpu_util import cuda_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_fwd_bwd(B, H, N, d, causal, seed=0, sigma_qk=1.0):
+    import torch
+    import exact_io_aware_43_b200 as fa
+    dev, f64 = cuda_inputs(B, H, N, d, seed, sigma_qk)
+    s = ai.default_scale(d)
+    o, lse = fa.forward(dev["q"], dev["k"], dev["v"], causal, s)
+    dq, dk, dv = fa.backward(dev["q"], dev["k"], dev["v"], o, lse, dev["do"], causal, s)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == 0
+    return (to_np(dq), to_np(dk), to_np(dv)), f64, s
+
+
+def oracle_grads(f64, causal, s, heads=None):
+    if heads is None:
+        O, L = attention_forward(f64["q"], f64["k"], f64["v"], causal, s)
+        return attention_backward(f64["q"], f64["k"], f64["v"], O, L, f64["do"], causal, s)
+    out = []
+    for (b, h) in heads:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        O, L = attention_forward(f64["q"][sl], f64["k"][sl], f64["v"][sl], causal, s)
+        g = attention_backward(f64["q"][sl], f64["k"][sl], f64["v"][sl], O, L, f64["do"][sl],
+                               causal, s)
+        out.append(tuple(x[0, 0] for x in g))
+    return out
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 3, 64, 100, 128, 129, 200, 256, 300, 513])
+def test_ragged_lengths(N, d, causal):
+    g, f64, s = gpu_fwd_bwd(1, 2, N, d, causal, seed=N + 7)
+    assert_bwd(g, oracle_grads(f64, causal, s), f"N={N} d={d} causal={causal}")
+
+
+def test_gpt2_small_causal():
+    g, f64, s = gpu_fwd_bwd(8, 12, 1024, 64, True)
+    assert_bwd(g, oracle_grads(f64, True, s), "GPT-2-small causal")
+
+
+@pytest.mark.parametrize("sigma", [1.0, 3.0])
+def test_bert_large(sigma):
+    g, f64, s = gpu_fwd_bwd(16, 16, 512, 64, False, sigma_qk=sigma)
+    assert_bwd(g, oracle_grads(f64, False, s), f"BERT-large sigma_qk={sigma}")
+
+
+def test_long_context_sampled_heads():
+    """B=2 H=16 N=8192 d=128 causal: complete gradients of the first and last heads."""
+    g, f64, s = gpu_fwd_bwd(2, 16, 8192, 128, True)
+    heads = [(0, 0), (1, 15)]
+    for (b, h), ref in zip(heads, oracle_grads(f64, True, s, heads)):
+        assert_bwd(tuple(x[b, h] for x in g), ref, f"long context head {(b, h)}")
+
+
+def test_gradient_invariants_on_gpu():
+    """sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i per head (rows of P sum to 1), within the
+    backward tolerance scaled to the size of the sums."""
+    import torch
+    g, f64, s = gpu_fwd_bwd(2, 3, 777, 128, True, seed=11)
+    dq, dk, dv = g
+    sum_dk = dk.sum(axis=2)
+    assert np.abs(sum_dk).max() <= 2e-2 * np.abs(dk).max() * np.sqrt(777)
+    err = np.abs(dv.sum(axis=2) - f64["do"].sum(axis=2)).max()
+    assert err <= 2e-2 * np.abs(dv).max() * np.sqrt(777)
+
+
+def test_dk_dv_deterministic():
+    import torch
+    import exact_io_aware_43_b200 as fa
+    dev, _ = cuda_inputs(2, 4, 1000, 128, seed=3)
+    o, lse = fa.forward(dev["q"], dev["k"], dev["v"], True)
+    a = fa.backward(dev["q"], dev["k"], dev["v"], o, lse, dev["do"], True)
+    b = fa.backward(dev["q"], dev["k"], dev["v"], o, lse, dev["do"], True)
+    torch.cuda.synchronize()
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    # dQ is reduced with fp32 atomics: order varies, only the tolerance applies
+    assert (a[0].float() - b[0].float()).abs().max().item() <= 1e-2
