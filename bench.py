@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200: one step = forward + backward of the
+long-context causal workload (B=2, H=16, N=8192, d=128, bf16), all four library kernels.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints ONE JSON line (rank 0).  The metric is attention fwd+bwd TFLOP/s with the FLOP count
+4*B*H*N^2*d (halved for causal) for the forward and 2.5x that for the backward, and its fraction
+of the measured dense-bf16 tensor peak.  Multi-GPU runs (torchrun) give every rank its own batch
+of heads (heads are independent: no collective on the data path) and report the whole-job
+throughput over the slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle on the same metric (a bounded sample of the same
+workload per step) -- the only other place this file runs the oracle is the ``cpu_baseline`` leg.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import attn_inputs as ai  # noqa: E402
+
+METRIC = "attention fwd/bwd TFLOP/s bf16 at N=8K d=128 causal; % of B200 BF16 peak"
+WORKLOAD = dict(B=2, H=16, N=8192, d=128, causal=True)
+WORKLOAD_NAME = "long-context causal fwd+bwd, B=2 H=16 N=8192 d=128 bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def flops(B, H, N, d, causal):
+    fwd = 4.0 * B * H * N * N * d * (0.5 if causal else 1.0)
+    return fwd, 2.5 * fwd
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="fattn", choices=["fattn", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--shape", default=None,
+                    help="B,H,N,d,causal override (profiling runs on a smaller case)")
+    args = ap.parse_args(argv)
+    if args.shape:
+        B, H, N, d, c = (int(x) for x in args.shape.split(","))
+        WORKLOAD.update(B=B, H=H, N=N, d=d, causal=bool(c))
+        global WORKLOAD_NAME
+        WORKLOAD_NAME = f"shape override B={B} H={H} N={N} d={d} causal={bool(c)} (profiling)"
+    return args
+
+
+# ---------------------------------------------------------------------------------- ranks
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def dist_init(backend):
+    import datetime
+
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def rank_seed(rank: int) -> int:
+    """Every rank draws its own batch (weak scaling: per-GPU work fixed as N grows)."""
+    return 1000 + rank
+
+
+def reduce_max(x: float, device=None) -> float:
+    """Max over ranks (timing is the slowest rank's device time)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------------------------- oracle leg
+def oracle_sample(rows: int, seed: int = 0):
+    """fp64 oracle fwd+bwd on one head of the workload restricted to its first `rows` positions
+    (a causal prefix: a shorter instance of the same computation).  Returns (seconds, flops)."""
+    from oracle import attention_backward, attention_forward
+    d = WORKLOAD["d"]
+    x = ai.make_inputs(1, 1, rows, d, seed=seed)
+    f = {k: ai.bf16_bits_to_f64(v) for k, v in x.items()}
+    s = ai.default_scale(d)
+    t0 = time.perf_counter()
+    O, L = attention_forward(f["q"], f["k"], f["v"], True, s)
+    attention_backward(f["q"], f["k"], f["v"], O, L, f["do"], True, s)
+    dt = time.perf_counter() - t0
+    ff, fb = flops(1, 1, rows, d, True)
+    return dt, ff + fb
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return int(max(i.get("num_threads", 1) for i in info))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline():
+    dt, fl = oracle_sample(WORKLOAD["N"])
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, forward+backward of 1 of the {WORKLOAD['B'] * WORKLOAD['H']}"
+                      f" heads (N=8192, d=128, causal) in {dt:.1f} s; algorithmic FLOPs"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    # size one step so the whole --warmup + --steps run stays within about three minutes
+    t_cal, _ = oracle_sample(1024)
+    rows = 1024
+    for r in (8192, 4096, 2048):
+        est = t_cal * (r / 1024) ** 2
+        if est * (args.steps + args.warmup) <= 180:
+            rows = r
+            break
+    for _ in range(args.warmup):
+        oracle_sample(rows)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample(rows)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAME, **WORKLOAD,
+                   "reference_sample": f"1 head, first {rows} positions per step"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(),
+                         "kind": "oracle",
+                         "sample": f"fp64 numpy oracle fwd+bwd, 1 head x {rows} positions "
+                                   "(causal prefix of the workload) per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------- GPU arm
+def kernel_traffic(kernel_name: str):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel_name)
+    except (OSError, ValueError):
+        return None
+    if not rec:
+        return None
+    src = hashlib.sha256()
+    for fn in sorted(os.listdir(os.path.join(ROOT, "exact_io_aware_43_b200", "csrc"))):
+        with open(os.path.join(ROOT, "exact_io_aware_43_b200", "csrc", fn), "rb") as f:
+            src.update(f.read())
+    if rec.get("csrc_sha256") != src.hexdigest():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def run_gpu(args):
+    import torch
+    import exact_io_aware_43_b200 as fa
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    rank, world = dist_init("nccl")
+    W = WORKLOAD
+    B, H, N, d, causal = W["B"], W["H"], W["N"], W["d"], W["causal"]
+    s = ai.default_scale(d)
+    x = ai.make_inputs(B, H, N, d, seed=rank_seed(rank))
+    host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) for k, v in x.items()}
+    q, k, v, do = (host[t].to(dev) for t in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        fa.forward(q, k, v, causal, s, out=o, lse=lse)
+        fa.backward(q, k, v, o, lse, do, causal, s, workspace=ws, grads=(dq, dk, dv))
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == 0, "a kernel reported a timeout during warm-up"
+    for kk in range(4):
+        fa.fa_timer_read(kk)  # discard anything recorded before the timed region
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(dev)
+    torch.cuda.synchronize()
+    fa.fa_timer_enable(True)
+    for i in range(args.steps):
+        flush.zero_()  # L2 flushed before every step, outside the timed events
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    fa.fa_timer_enable(False)
+    barrier(dev)
+    clocks = sampler.stop()
+    status = fa.fa_device_status()
+    ms_local = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    ktimes = {kk: fa.fa_timer_read(kk) for kk in range(4)}
+    ms = reduce_max(ms_local, dev)
+
+    ff, fb = flops(B, H, N, d, causal)
+    value = world * (ff + fb) / (ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    fwd_ms = ktimes[fa.FA_KERNEL_FWD][1] / max(1, ktimes[fa.FA_KERNEL_FWD][0])
+    bwd_ms = sum(ktimes[kk][1] for kk in (1, 2, 3)) / max(1, ktimes[fa.FA_KERNEL_BWD_MAIN][0])
+
+    # roofline of the dominant kernel (largest share of device time)
+    dom = max(range(4), key=lambda kk: ktimes[kk][1])
+    n_l, tot = ktimes[dom]
+    avg_ms = tot / max(1, n_l)
+    if dom in (fa.FA_KERNEL_FWD, fa.FA_KERNEL_BWD_MAIN):
+        work = ff if dom == fa.FA_KERNEL_FWD else fb
+        achieved = work / (avg_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak)}
+    else:
+        nbytes = (B * H * N * d * 2 * 2 + B * H * N * 4 + B * H * N * d * 4 + 2 * B * H * N * 4
+                  if dom == fa.FA_KERNEL_BWD_PRE else B * H * N * d * (4 + 2))
+        achieved = nbytes / (avg_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs"}
+    roof["kernel"] = fa.KERNEL_NAMES[dom]
+    roof["launches"] = n_l
+    roof["avg_ms"] = avg_ms
+    roof["traffic"] = kernel_traffic(fa.KERNEL_NAMES[dom])
+    shares = {fa.KERNEL_NAMES[kk]: ktimes[kk][1] / max(1e-9, sum(t for _, t in ktimes.values()))
+              for kk in range(4)}
+
+    # end to end through the public API: pinned host inputs -> device -> fwd+bwd -> host grads
+    e2e = None
+    if args.e2e_steps > 0:
+        hin = {t: host[t].pin_memory() for t in ("q", "k", "v", "do")}
+        hout = [torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+        e_ev = []
+        torch.cuda.synchronize()
+        barrier(dev)
+        for i in range(args.e2e_steps + 2):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            q.copy_(hin["q"], non_blocking=True)
+            k.copy_(hin["k"], non_blocking=True)
+            v.copy_(hin["v"], non_blocking=True)
+            do.copy_(hin["do"], non_blocking=True)
+            step()
+            for hsrc, dsrc in zip(hout, (dq, dk, dv)):
+                hsrc.copy_(dsrc, non_blocking=True)
+            b.record()
+            if i >= 2:
+                e_ev.append((a, b))
+        torch.cuda.synchronize()
+        e_ms = reduce_max(sum(a.elapsed_time(b) for a, b in e_ev) / len(e_ev), dev)
+        h2d = sum(t.numel() * t.element_size() for t in hin.values())
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+        e2e = {"value": world * (ff + fb) / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAME, **WORKLOAD, "scale": s,
+                       "flops_per_step_per_gpu": ff + fb,
+                       "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                       "parallelism": f"heads: {world} independent replicas, no collective"},
+            "pct_of_peak": value / world / peaks["bf16_tflops"] * 100.0,
+            "fwd_tflops": ff / (fwd_ms * 1e-3) / 1e12, "bwd_tflops": fb / (bwd_ms * 1e-3) / 1e12,
+            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "kernel_time_share": shares,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": sum(ktimes[kk][0] for kk in range(4)),
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -52,6 +52,10 @@ def lib() -> ctypes.CDLL:
     L.fa_device_status.restype = i
     L.fa_version.argtypes = []
     L.fa_version.restype = i
+    L.fa_timer_enable.argtypes = [i]
+    L.fa_timer_enable.restype = i
+    L.fa_timer_read.argtypes = [i, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
+    L.fa_timer_read.restype = i
     _lib = L
     return L
 
@@ -94,6 +98,23 @@ def fa_device_status(stream=None) -> int:
 
 def fa_version() -> int:
     return lib().fa_version()
+
+
+FA_KERNEL_FWD, FA_KERNEL_BWD_PRE, FA_KERNEL_BWD_MAIN, FA_KERNEL_BWD_POST = range(4)
+KERNEL_NAMES = {FA_KERNEL_FWD: "fa_fwd_kernel", FA_KERNEL_BWD_PRE: "fa_bwd_pre_kernel",
+                FA_KERNEL_BWD_MAIN: "fa_bwd_kernel", FA_KERNEL_BWD_POST: "fa_bwd_post_kernel"}
+
+
+def fa_timer_enable(on: bool) -> int:
+    return lib().fa_timer_enable(int(bool(on)))
+
+
+def fa_timer_read(kernel: int):
+    """(launches, total_ms) recorded for one kernel kind since the last read."""
+    n = ctypes.c_int(0)
+    ms = ctypes.c_double(0.0)
+    _check(lib().fa_timer_read(kernel, ctypes.byref(n), ctypes.byref(ms)))
+    return n.value, ms.value
 
 
 # ------------------------------------------------------------------ torch conveniences

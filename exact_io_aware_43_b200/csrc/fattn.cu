@@ -10,6 +10,8 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "../../include/fattn.h"
 #include "bwd.cuh"
@@ -66,6 +68,34 @@ int make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_row
   if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
   return FA_OK;
 }
+
+// ---- optional per-kernel event timing (benchmark support)
+struct KernelTimer {
+  std::mutex mu;
+  bool on = false;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev[4];
+};
+KernelTimer g_timer;
+
+struct TimedLaunch {
+  int kind;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr, b = nullptr;
+  TimedLaunch(int k, cudaStream_t s) : kind(k), st(s) {
+    if (!g_timer.on) return;
+    if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) {
+      a = b = nullptr;
+      return;
+    }
+    cudaEventRecord(a, st);
+  }
+  ~TimedLaunch() {
+    if (!a) return;
+    cudaEventRecord(b, st);
+    std::lock_guard<std::mutex> g(g_timer.mu);
+    g_timer.ev[kind].emplace_back(a, b);
+  }
+};
 
 uint64_t wait_limit_ns() {
   static uint64_t v = [] {
@@ -125,6 +155,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   if (rc) return rc;
   p.nqb = (p.N + NQT * C::BM - 1) / (NQT * C::BM);
   dim3 grid(unsigned(BH) * unsigned(p.nqb));
+  TimedLaunch tl(FA_KERNEL_FWD, st);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fa_fwd launch");
@@ -153,17 +184,26 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
   if ((rc = make_map(&mv, v, p.BH, p.N, D, C::BC))) return rc;
   if ((rc = make_map(&mdo, p.dO, p.BH, p.N, D, C::BR))) return rc;
   const int grid_ew = sm_count() * 8;
-  fattn::fa_bwd_pre_kernel<D><<<grid_ew, 256, 0, st>>>(p);
+  {
+    TimedLaunch tl(FA_KERNEL_BWD_PRE, st);
+    fattn::fa_bwd_pre_kernel<D><<<grid_ew, 256, 0, st>>>(p);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fa_bwd preprocess launch");
   auto kern = fattn::fa_bwd_kernel<D, CAUSAL>;
   if ((rc = set_smem(kern, C::SMEM_BYTES))) return rc;
   dim3 grid(unsigned(p.BH) * unsigned(p.nkb) * unsigned(C::NSL));
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
+  {
+    TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fa_bwd launch");
   const long long n8 = (long long)p.BH * p.N * D / 8;
-  fattn::fa_bwd_post_kernel<<<grid_ew, 256, 0, st>>>(p.dq_acc, p.dq, n8);
+  {
+    TimedLaunch tl(FA_KERNEL_BWD_POST, st);
+    fattn::fa_bwd_post_kernel<<<grid_ew, 256, 0, st>>>(p.dq_acc, p.dq, n8);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fa_bwd postprocess launch");
   return FA_OK;
@@ -265,6 +305,36 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if ((rc = check_device())) return rc;
   return bwd_dispatch(q, k, v, o, lse, dO, dq, dk, dv, B * H, N, d, causal != 0, scale,
                       workspace, static_cast<cudaStream_t>(stream));
+}
+
+int fa_timer_enable(int on) {
+  std::lock_guard<std::mutex> g(g_timer.mu);
+  g_timer.on = on != 0;
+  return FA_OK;
+}
+
+int fa_timer_read(int kernel, int* launches, double* total_ms) {
+  if (kernel < 0 || kernel > 3 || !launches || !total_ms)
+    return fail(FA_ERR_INVALID_ARG, "fa_timer_read: bad kernel kind or null output");
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> evs;
+  {
+    std::lock_guard<std::mutex> g(g_timer.mu);
+    evs.swap(g_timer.ev[kernel]);
+  }
+  double sum = 0.0;
+  int rc = FA_OK;
+  for (auto& pr : evs) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(pr.second);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, pr.first, pr.second);
+    if (e != cudaSuccess && rc == FA_OK) rc = cuda_fail(e, "fa_timer_read");
+    sum += ms;
+    cudaEventDestroy(pr.first);
+    cudaEventDestroy(pr.second);
+  }
+  *launches = int(evs.size());
+  *total_ms = sum;
+  return rc;
 }
 
 int fa_device_status(void* stream) {

@@ -101,6 +101,18 @@ int fa_device_status(void* stream);
 /* Library version as major*10000 + minor*100 + patch. */
 int fa_version(void);
 
+/*
+ * Benchmark support: per-kernel device time.  Not part of the attention computation.
+ * fa_timer_enable(on != 0) makes every later kernel launch of the library record a pair of CUDA
+ * events around itself on its launching stream (host-side objects only; no device memory).
+ * fa_timer_read(kernel, &launches, &total_ms) waits for the recorded events of one kernel kind,
+ * returns the number of launches and their summed device time, and forgets them.
+ * Kernel kinds: FA_KERNEL_FWD, FA_KERNEL_BWD_PRE, FA_KERNEL_BWD_MAIN, FA_KERNEL_BWD_POST.
+ */
+enum { FA_KERNEL_FWD = 0, FA_KERNEL_BWD_PRE = 1, FA_KERNEL_BWD_MAIN = 2, FA_KERNEL_BWD_POST = 3 };
+int fa_timer_enable(int on);
+int fa_timer_read(int kernel, int* launches, double* total_ms);
+
 #ifdef __cplusplus
 }
 #endif

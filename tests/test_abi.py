@@ -1,0 +1,105 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry point, and rejects
+bad arguments on the host before any launch."""
+import json
+import os
+
+import pytest
+
+import exact_io_aware_43_b200 as fa
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+A = 1 << 20  # a 16-byte aligned fake device address (never dereferenced: checks run first)
+
+
+def test_exports_every_declared_symbol():
+    names = fa.header_functions()
+    assert {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_last_error"} <= set(names)
+    L = fa.lib()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version():
+    assert fa.fa_version() >= 100
+
+
+def test_workspace_size_formula():
+    B, H, N, d = 2, 16, 8192, 128
+    npad = (N + 127) // 128 * 128
+    want = B * H * N * d * 4 + 2 * B * H * npad * 4
+    assert fa.fa_bwd_workspace_size(B, H, N, d) == want
+    # ragged N: the row vectors are padded to 128
+    got = fa.fa_bwd_workspace_size(1, 1, 129, 64)
+    assert got >= 129 * 64 * 4 + 2 * 256 * 4
+    for bad in ((0, 1, 1, 64), (1, 0, 1, 64), (1, 1, 0, 64), (1, 1, 8, 96)):
+        assert fa.fa_bwd_workspace_size(*bad) == 0
+
+
+def test_workspace_is_linear_not_quadratic():
+    """The naive score matrix at B*H = 32, N = 8192 would take about 4 GB (the pages' example);
+    the backward's whole workspace is O(N) per head and a small fraction of it."""
+    g = json.load(open(os.path.join(GOLDEN, "naive_score_matrix_bytes.json")))
+    ws = fa.fa_bwd_workspace_size(2, 16, 8192, 128)
+    assert ws * 20 < g["bytes"]
+    # doubling N doubles (not quadruples) the workspace
+    assert fa.fa_bwd_workspace_size(2, 16, 16384, 128) == 2 * ws
+
+
+def fwd(**kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, N=128, d=64, causal=0, scale=0.125, stream=None)
+    a.update(kw)
+    return fa.fa_fwd(**a)
+
+
+def bwd(**kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, dO=A, dq=A, dk=A, dv=A, B=1, H=1, N=128, d=64, causal=0,
+             scale=0.125, workspace=A, workspace_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return fa.fa_bwd(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), fa.FA_ERR_INVALID_ARG),
+    (dict(lse=None), fa.FA_ERR_INVALID_ARG),
+    (dict(B=0), fa.FA_ERR_INVALID_ARG),
+    (dict(N=0), fa.FA_ERR_INVALID_ARG),
+    (dict(N=-5), fa.FA_ERR_INVALID_ARG),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=32), fa.FA_ERR_UNSUPPORTED),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), fa.FA_ERR_INVALID_ARG),
+    (dict(q=A + 8), fa.FA_ERR_MISALIGNED),
+    (dict(o=A + 2), fa.FA_ERR_MISALIGNED),
+])
+def test_fwd_rejects(kw, code):
+    assert fwd(**kw) == code
+    assert fa.fa_last_error() != ""
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dO=None), fa.FA_ERR_INVALID_ARG),
+    (dict(dq=None), fa.FA_ERR_INVALID_ARG),
+    (dict(d=100), fa.FA_ERR_UNSUPPORTED),
+    (dict(dk=A + 4), fa.FA_ERR_MISALIGNED),
+    (dict(workspace=None), fa.FA_ERR_WORKSPACE),
+    (dict(workspace=A + 8), fa.FA_ERR_WORKSPACE),
+    (dict(workspace_bytes=100), fa.FA_ERR_WORKSPACE),
+])
+def test_bwd_rejects(kw, code):
+    assert bwd(**kw) == code
+    assert fa.fa_last_error() != ""
+
+
+def test_timer_read_rejects_bad_kind():
+    import ctypes
+    n, ms = ctypes.c_int(0), ctypes.c_double(0)
+    assert fa.lib().fa_timer_read(7, ctypes.byref(n), ctypes.byref(ms)) == fa.FA_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(fa, "_lib", None)
+    monkeypatch.setattr(fa, "LIB_PATH", "/nonexistent/libfattn.so")
+    with pytest.raises(fa.FattnError):
+        fa.lib()
