@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
     L.fa_device_status.restype = i
     L.fa_version.argtypes = []
     L.fa_version.restype = i
+    L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+    L.fa_bwd_noalloc.restype = i
     L.fa_timer_enable.argtypes = [i]
     L.fa_timer_enable.restype = i
     L.fa_timer_read.argtypes = [i, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
@@ -90,6 +92,16 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, workspace
            workspace_bytes, stream) -> int:
     return lib().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, int(causal), float(scale),
                         workspace, workspace_bytes, stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, stream) -> int:
+    """fa_bwd with the library's static scratch instead of a caller workspace (for callers that
+    cannot allocate device memory; shapes up to FA_NOALLOC_SCRATCH_BYTES of workspace)."""
+    return lib().fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, int(causal),
+                                float(scale), stream)
+
+
+FA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 def fa_device_status(stream=None) -> int:

@@ -353,3 +353,57 @@ int fa_device_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// fa_bwd_noalloc: fa_bwd with its workspace in a static device array (callers that cannot
+// allocate).  Host code never uses the array's name as an address: the device address comes
+// from cudaGetSymbolAddress, looked up once per device with that device current.
+// ------------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* ptrs[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 128) return fail(FA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> g(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                              const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                              int B, int H, int N, int d, int causal, float scale, void* stream) {
+  g_msg[0] = 0;
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv)
+    return fail(FA_ERR_INVALID_ARG, "null tensor pointer");
+  int rc = check_common(B, H, N, d, scale);
+  if (rc) return rc;
+  for (const void* ptr : {q, k, v, o, static_cast<const void*>(lse), dO,
+                          static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv)})
+    if (!aligned16(ptr)) return fail(FA_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (need > FA_NOALLOC_SCRATCH_BYTES)
+    return fail(FA_ERR_WORKSPACE,
+                "fa_bwd_noalloc: this shape needs %zu bytes of scratch but the library's static "
+                "scratch holds %u bytes; use fa_bwd with a caller-provided workspace",
+                need, unsigned(FA_NOALLOC_SCRATCH_BYTES));
+  if ((rc = check_device())) return rc;
+  void* ws = nullptr;
+  if ((rc = noalloc_scratch(&ws))) return rc;
+  return bwd_dispatch(q, k, v, o, lse, dO, dq, dk, dv, B * H, N, d, causal != 0, scale, ws,
+                      static_cast<cudaStream_t>(stream));
+}

@@ -88,6 +88,35 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            int B, int H, int N, int d, int causal, float scale,
            void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * fa_bwd_noalloc -- the backward pass for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it is an interface addition of this library.
+ *
+ * Who needs it: a program whose own pooled allocator already holds nearly all of the GPU's
+ * memory (a direct cudaMalloc would fail or fragment that pool), or a host application that
+ * forbids allocation while it runs a step, for latency or memory-accounting reasons, cannot
+ * provide the workspace fa_bwd asks for.  This variant takes the same tensors as fa_bwd, minus
+ * the workspace, and uses a scratch array compiled into the library instead.
+ *
+ * The scratch is a file-scope static device array of FA_NOALLOC_SCRATCH_BYTES (32 MiB).  Every
+ * GPU on which the library's kernels are loaded holds that array until the process exits.
+ * Shapes whose fa_bwd_workspace_size exceeds it return FA_ERR_WORKSPACE before any launch
+ * (for example B=8, H=12, N=1024, d=64 needs about 26 MB and fits; B=2, H=16, N=8192, d=128
+ * needs 130 MB and does not).  The entry point calls no cudaMalloc, cudaFree or other allocating
+ * routine.
+ *
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current) and caches it; make that first call before any stream capture.
+ * All calls on a device share the one array, which keeps whatever the last call left in it
+ * (the kernels clear what must start at zero).  Calls that overlap on the GPU -- on different
+ * streams, or from different host threads -- race on the array and corrupt each other's
+ * results: serialise them.  Arguments, layouts and results are otherwise those of fa_bwd.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv,
+                   int B, int H, int N, int d, int causal, float scale, void* stream);
+
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 const char* fa_last_error(void);
 
