@@ -143,7 +143,12 @@ struct BwdCfg {
   static constexpr int OFF_DO = OFF_Q + STAGES * Q_BYTES;        // STAGES x dO_i
   static constexpr int OFF_DS = OFF_DO + STAGES * Q_BYTES;       // dS^T [128 keys][64 q] bf16
   static constexpr int OFF_ROWS = OFF_DS + BC * BR * 2;          // STAGES x (L2[64], D[64])
-  static constexpr int OFF_BAR = OFF_ROWS + STAGES * 2 * BR * 4;
+  // dQ staging: slots of [64 queries][64 d] fp32 reduced into the accumulator by TMA
+  static constexpr int DQ_CH = DO / 64;                          // 64-wide chunks per tile
+  static constexpr int DQ_SLOT = BR * 64 * 4;
+  static constexpr int DQ_SLOTS = D == 64 ? 2 : (D == 128 ? 4 : 1);
+  static constexpr int OFF_DQS = OFF_ROWS + STAGES * 2 * BR * 4;
+  static constexpr int OFF_BAR = OFF_DQS + DQ_SLOTS * DQ_SLOT;
   // barriers: kv_full, q_full[S], q_empty[S], s_full, s_free, dp_full, dp_free, p_full,
   //           ds_full, dv_done, dq_full, dq_empty, drain
   static constexpr int NBAR = 1 + 2 * STAGES + 11;
@@ -154,15 +159,11 @@ struct BwdCfg {
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(DO, BR, 1, 1);  // dQ^T = K^T dS^T
 };
 
-__device__ __forceinline__ void red_add_f32(float* addr, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
-}
-
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -349,8 +350,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const int s = it % C::STAGES;
       const float* L2s = rows_smem + s * 2 * C::BR;
       const float* Ds = L2s + C::BR;
-      if (!(ok = W.wait(BAR_SF, it & 1, 50))) break;
-      if (!(ok = W.wait(BAR_QF(s), (it / C::STAGES) & 1, 51))) break;
+      if (!(ok = W.wait_warp(BAR_SF, it & 1, 50))) break;
+      if (!(ok = W.wait_warp(BAR_QF(s), (it / C::STAGES) & 1, 51))) break;
       tc_fence_after();
       uint32_t st[2][32];
       tmem_ld32(tmem + lane_base + C::T_S, st[0]);
@@ -364,17 +365,23 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       float pr[64];
       const int qbase = i * C::BR;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float x = fmaf(__uint_as_float(st[c >> 5][c & 31]), p.scale_log2, -L2s[c]);
-        bool valid = key_ok;
-        if (CAUSAL) valid = valid && (key <= qbase + c);
-        pr[c] = valid ? ex2(x) : 0.f;
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 l4 = reinterpret_cast<const float4*>(L2s)[c4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * c4 + e;
+          const float x = fmaf(__uint_as_float(st[c >> 5][c & 31]), p.scale_log2, -lv[e]);
+          bool valid = key_ok;
+          if (CAUSAL) valid = valid && (key <= qbase + c);
+          pr[c] = valid ? ex2(x) : 0.f;
+        }
       }
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
       // P^T columns are free once dV(it-1) has read them
-      if (it > 0 && !(ok = W.wait(BAR_DVD, (it - 1) & 1, 52))) break;
+      if (it > 0 && !(ok = W.wait_warp(BAR_DVD, (it - 1) & 1, 52))) break;
       tc_fence_after();
       tmem_st32(tmem + lane_base + C::T_P, pk);
       tmem_wait_st();
@@ -382,7 +389,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_PF);
       // dS^T = P^T * (dP^T - D)
-      if (!(ok = W.wait(BAR_DPF, it & 1, 53))) break;
+      if (!(ok = W.wait_warp(BAR_DPF, it & 1, 53))) break;
       tc_fence_after();
       tmem_ld32(tmem + lane_base + C::T_DP, st[0]);
       tmem_ld32(tmem + lane_base + C::T_DP + 32, st[1]);
@@ -392,14 +399,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_DPFREE);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float d0 = pr[2 * c] * (__uint_as_float(st[(2 * c) >> 5][(2 * c) & 31]) - Ds[2 * c]);
-        const float d1 =
-            pr[2 * c + 1] * (__uint_as_float(st[(2 * c + 1) >> 5][(2 * c + 1) & 31]) - Ds[2 * c + 1]);
-        pk[c] = pack_bf16(d0, d1);
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 d4 = reinterpret_cast<const float4*>(Ds)[c4];
+        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = 4 * c4 + 2 * e;
+          const float d0 = pr[c] * (__uint_as_float(st[c >> 5][c & 31]) - dv4[2 * e]);
+          const float d1 = pr[c + 1] * (__uint_as_float(st[(c + 1) >> 5][(c + 1) & 31]) - dv4[2 * e + 1]);
+          pk[c >> 1] = pack_bf16(d0, d1);
+        }
       }
       // dS^T columns and the dS smem tile are free once dK(it-1) and dQ(it-1) have read them
-      if (it > 0 && !(ok = W.wait(BAR_DQF, (it - 1) & 1, 54))) break;
+      if (it > 0 && !(ok = W.wait_warp(BAR_DQF, (it - 1) & 1, 54))) break;
       tc_fence_after();
       tmem_st32(tmem + lane_base + C::T_DS, pk);
 #pragma unroll
@@ -415,7 +427,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
     if (ok) {
       // ---- epilogue: dV, dK (x scale) -> bf16 -> global
-      ok = W.wait(BAR_DQF, (nit - 1) & 1, 55);
+      ok = W.wait_warp(BAR_DQF, (nit - 1) & 1, 55);
       if (ok) {
         tc_fence_after();
         const size_t base = (size_t(head) * p.N + key) * D + slice * C::DO;
@@ -446,15 +458,25 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     tc_fence_before();
   } else if (warp < 8) {
     // ---------------------------------------------------------------- dQ drain warpgroup
+    // dQ^T (d on TMEM lanes, 64 queries on columns) -> x scale -> shared staging slots laid out
+    // [64 queries][64 d] fp32 -> TMA bulk reduce-add into the fp32 accumulator (rows past N are
+    // clipped by the tensor map).
     const int wq = warp - C::DQ_WARP0;
+    const int tq = threadIdx.x - C::DQ_WARP0 * 32;  // 0..127
+    const bool issuer = tq == 0;
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     // dQ^T rows are d indices.  M = 128: lane i of warp w holds row 32w+i.  M = 64: rows
     // 16w..16w+15 sit in lanes 0..15 of warp w's lane quarter; lanes 16..31 hold nothing.
     const int drow = (C::DO == 128) ? (wq * 32 + lane) : (wq * 16 + lane);
     const bool row_ok = (C::DO == 128) || (lane < 16);
+    const int my_chunk = drow >> 6;
+    float* slots = reinterpret_cast<float*>(smem + C::OFF_DQS);
+    if (issuer) tma_prefetch_desc(&tmdQ);
+    int group = 0;
     for (int it = 0; it < nit; ++it) {
       const int i = i_start + it;
-      if (!W.wait(BAR_DQF, it & 1, 60)) break;
+      // the four drain warps leave the loop together (they share named barriers below)
+      if (!named_bar_and(1, 128, W.wait_warp(BAR_DQF, it & 1, 60))) break;
       tc_fence_after();
       uint32_t v[2][32];
       tmem_ld32(tmem + lane_base + C::T_DQ, v[0]);
@@ -464,15 +486,26 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_DQE);
-      if (row_ok) {
-        const int qbase = i * C::BR;
-        const int nq = min(C::BR, p.N - qbase);
-        float* dst = p.dq_acc + (size_t(head) * p.N + qbase) * D + slice * C::DO + drow;
 #pragma unroll
-        for (int c = 0; c < C::BR; ++c)
-          if (c < nq) red_add_f32(dst + size_t(c) * D, __uint_as_float(v[c >> 5][c & 31]) * p.scale);
+      for (int ch = 0; ch < C::DQ_CH; ++ch, ++group) {
+        const int slot = group % C::DQ_SLOTS;
+        if (issuer) bulk_wait_group_read<C::DQ_SLOTS - 1>();  // slot's previous reduce has read it
+        named_bar_sync(1, 128);
+        if (row_ok && my_chunk == ch) {
+          float* dst = slots + slot * (C::BR * 64) + (drow & 63);
+#pragma unroll
+          for (int c = 0; c < C::BR; ++c) dst[c * 64] = __uint_as_float(v[c >> 5][c & 31]) * p.scale;
+        }
+        fence_async_smem();
+        named_bar_sync(1, 128);
+        if (issuer) {
+          tma_reduce_add_3d(&tmdQ, smem_u32(slots + slot * (C::BR * 64)), slice * C::DO + ch * 64,
+                            i * C::BR, head);
+          bulk_commit_group();
+        }
       }
     }
+    if (issuer) bulk_wait_group_all();
     tc_fence_before();
   }
 

@@ -97,6 +97,22 @@ struct TimedLaunch {
   }
 };
 
+// fp32 [BH, N, d] map for the dQ accumulator: box 64 columns x 64 rows x 1 head, no swizzle
+// (the reduce-add source in shared memory is a dense [64][64] fp32 tile).
+int make_map_f32(CUtensorMap* m, void* base, int BH, int N, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(N) * cuuint64_t(d) * 4};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled (f32) failed (%d)", int(r));
+  return FA_OK;
+}
+
 uint64_t wait_limit_ns() {
   static uint64_t v = [] {
     const char* e = getenv("FA_WAIT_LIMIT_NS");
@@ -153,6 +169,20 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   auto kern = fattn::fa_fwd_kernel<D, CAUSAL, NQT>;
   int rc = set_smem(kern, C::SMEM_BYTES);
   if (rc) return rc;
+  if (C::REALLOC) {
+    // setmaxnreg.inc can only draw on the registers the CTA was launched with; refuse to launch
+    // a build whose per-thread launch allocation is below the split the kernel asks for.
+    static int checked = 0;  // 0 unknown, 1 ok, 2 bad
+    if (checked == 0) {
+      cudaFuncAttributes fa_attr;
+      cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+      checked = (fa_attr.numRegs * C::THREADS >= C::CTRL_REGS * 128 + C::SOFTMAX_REGS * 256) ? 1 : 2;
+    }
+    if (checked == 2)
+      return fail(FA_ERR_UNSUPPORTED, "fa_fwd kernel built with too few launch registers for its "
+                                      "register split");
+  }
   p.nqb = (p.N + NQT * C::BM - 1) / (NQT * C::BM);
   dim3 grid(unsigned(BH) * unsigned(p.nqb));
   TimedLaunch tl(FA_KERNEL_FWD, st);
@@ -183,6 +213,8 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
   if ((rc = make_map(&mk, k, p.BH, p.N, D, C::BC))) return rc;
   if ((rc = make_map(&mv, v, p.BH, p.N, D, C::BC))) return rc;
   if ((rc = make_map(&mdo, p.dO, p.BH, p.N, D, C::BR))) return rc;
+  CUtensorMap mdq;
+  if ((rc = make_map_f32(&mdq, p.dq_acc, p.BH, p.N, D))) return rc;
   const int grid_ew = sm_count() * 8;
   {
     TimedLaunch tl(FA_KERNEL_BWD_PRE, st);
@@ -195,7 +227,7 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
   dim3 grid(unsigned(p.BH) * unsigned(p.nkb) * unsigned(C::NSL));
   {
     TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fa_bwd launch");

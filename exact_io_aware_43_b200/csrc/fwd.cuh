@@ -41,9 +41,17 @@ struct FwdCfg {
   static constexpr int KVTILE_BYTES = BN * D * 2;
   static constexpr int STAGES = (D == 64) ? 4 : (D == 128 ? 2 : 1);
   static constexpr int SOFTMAX_WARPS = 4 * NQT;
-  static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;
+  static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;  // control warpgroup: producer, MMA, 2 idle
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
-  static constexpr int THREADS = (SOFTMAX_WARPS + 2) * 32;
+  static constexpr int THREADS = (SOFTMAX_WARPS + 4) * 32;
+  // Register split with two softmax warpgroups (384 threads launched at 168 registers each):
+  // control warpgroup 40, softmax warpgroups 232; 40*128 + 232*256 = 384*168.
+  static constexpr bool REALLOC = NQT == 2;
+  static constexpr int LAUNCH_REGS = 168;
+  static constexpr int CTRL_REGS = 40;
+  static constexpr int SOFTMAX_REGS = 232;
+  static_assert(!REALLOC || CTRL_REGS * 128 + SOFTMAX_REGS * 256 <= LAUNCH_REGS * THREADS,
+                "register split exceeds the launch allocation");
   static constexpr int TMEM_S = 0;               // S_t at column t*BN (P_t aliases its first BN/2)
   static constexpr int TMEM_O = NQT * BN;        // O_t at TMEM_O + t*D
   static constexpr int TMEM_COLS = 512;
@@ -130,8 +138,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == C::PRODUCER_WARP) {
+  if (warp >= C::SOFTMAX_WARPS) {
+   // ================================================================ control warpgroup
+   if constexpr (C::REALLOC) regs_dec<C::CTRL_REGS>();
+   if (warp == C::PRODUCER_WARP) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -175,31 +185,34 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     }
   } else if (warp == C::MMA_WARP) {
     // ---------------------------------------------------------------- MMA issuer
+    // Order per KV tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  S_t(j+1) overwrites the tensor
+    // memory that holds P_t(j), so it waits for PV_t(j) to complete; issuing it right behind
+    // PV_t(j) lets softmax t start on tile j+1 while the other query tile's PV runs.
     if (lane == 0) {
-      bool ok = W.wait(BAR_Q, 0, 10);
+      auto issue_s = [&](int t, uint32_t k_addr) {
+        const uint32_t q_addr = sbase + C::OFF_Q + t * C::QTILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ss(tmem + C::TMEM_S + t * C::BN, sdesc_sw128(q_addr + koff, 16, 1024),
+                 sdesc_sw128(k_addr + koff, 16, 1024), C::IDESC_S, kk > 0);
+        }
+        tc_commit(BAR_SF(t));
+      };
+      bool ok = W.wait(BAR_Q, 0, 10) && W.wait(BAR_KF(0), 0, 11);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < NQT; ++t)
+          if (nkv[t] > 0) issue_s(t, sbase + C::OFF_K);
+        tc_commit(BAR_KE(0));
+      }
       for (int j = 0; ok && j < J; ++j) {
         const int s = j % C::STAGES;
-        const uint32_t ph = (j / C::STAGES) & 1;
-        const uint32_t k_addr = sbase + C::OFF_K + s * C::KVTILE_BYTES;
+        const int s1 = (j + 1) % C::STAGES;
         const uint32_t v_addr = sbase + C::OFF_V + s * C::KVTILE_BYTES;
-        if (!(ok = W.wait(BAR_KF(s), ph, 11))) break;
-        for (int t = 0; t < NQT && ok; ++t) {
-          if (j >= nkv[t]) continue;
-          // S_t's columns hold P_t(j-1) until PV_t(j-1) has read it
-          if (j > 0 && !(ok = W.wait(BAR_OD(t), (j - 1) & 1, 12))) break;
-          tc_fence_after();
-          const uint32_t q_addr = sbase + C::OFF_Q + t * C::QTILE_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            mma_ss(tmem + C::TMEM_S + t * C::BN, sdesc_sw128(q_addr + koff, 16, 1024),
-                   sdesc_sw128(k_addr + koff, 16, 1024), C::IDESC_S, kk > 0);
-          }
-          tc_commit(BAR_SF(t));
-        }
-        if (!ok) break;
-        tc_commit(BAR_KE(s));
-        if (!(ok = W.wait(BAR_VF(s), ph, 13))) break;
+        const uint32_t k1_addr = sbase + C::OFF_K + s1 * C::KVTILE_BYTES;
+        if (!(ok = W.wait(BAR_VF(s), (j / C::STAGES) & 1, 13))) break;
+        bool k_ready = false;
         for (int t = 0; t < NQT && ok; ++t) {
           if (j >= nkv[t]) continue;
           if (!(ok = W.wait(BAR_PF(t), j & 1, 14))) break;
@@ -213,16 +226,26 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
                    (j > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(BAR_OD(t));
+          if (j + 1 < nkv[t]) {
+            if (!k_ready && !(ok = W.wait(BAR_KF(s1), ((j + 1) / C::STAGES) & 1, 11))) break;
+            k_ready = true;
+            if (!(ok = W.wait(BAR_OD(t), j & 1, 12))) break;  // P_t(j) consumed
+            tc_fence_after();
+            issue_s(t, k1_addr);
+          }
         }
         if (!ok) break;
         tc_commit(BAR_VE(s));
+        if (k_ready) tc_commit(BAR_KE(s1));
       }
       // every MMA issued above has completed before the tensor memory is released
       tc_commit(BAR_DRAIN);
       W.drain(BAR_DRAIN, 0);
     }
+   }
   } else {
     // ---------------------------------------------------------------- softmax warpgroups
+    if constexpr (C::REALLOC) regs_inc<C::SOFTMAX_REGS>();
     const int t = warp >> 2;                  // query tile of this warpgroup
     const int r = threadIdx.x & 127;          // row within the tile == TMEM lane
     const int row = q0 + t * C::BM + r;       // query index
@@ -230,11 +253,16 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     const uint32_t tS = tmem + lane_base + C::TMEM_S + t * C::BN;
     const uint32_t tO = tmem + lane_base + C::TMEM_O + t * D;
     const int n = nkv[t];
-    float m = -INFINITY;  // running max of s*log2e*scale
-    float l = 0.f;        // running sum of exponentials (relative to m)
+    // m: reference max (log2 units of the scaled scores) that the exponentials and l are taken
+    // against.  It only moves when a row's max grows by more than kRescale (2^8 in value): the
+    // result is the same exact softmax, P~ stays <= 256, and O is rescaled far less often.
+    constexpr float kRescale = 8.0f;
+    float m = -INFINITY;
+    float l = 0.f;   // sum of the fp32 exponentials (for L)
+    float lr = 0.f;  // sum of the bf16-rounded exponentials (divides O)
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      if (!(ok = W.wait(BAR_SF(t), j & 1, 20))) break;
+      if (!(ok = W.wait_warp(BAR_SF(t), j & 1, 20))) break;
       tc_fence_after();
       uint32_t s[4][32];
 #pragma unroll
@@ -251,23 +279,44 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           for (int e = 0; e < 32; ++e)
             if (32 * c + e > lim) s[c][e] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      float mx8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
-      const float m_new = fmaxf(m, mx * p.scale_log2);
-      const float alpha = (m_new == m) ? 1.f : ex2(m - m_new);
-      float sum = 0.f;
+        for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(s[c][e]));
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float m_tile = mx * p.scale_log2;
+      const float m_use = (j == 0 || m_tile > m + kRescale) ? fmaxf(m, m_tile) : m;
+      const float alpha = (j == 0 || m_use == m) ? 1.f : ex2(m - m_use);
+      // exact fp32 sum (for L) and the sum of the bf16-rounded weights the PV MMA uses (for O's
+      // normalisation: numerator and denominator then agree, so a row dominated by one key
+      // reproduces that key's V), both accumulated in paired fp32
+      uint64_t sum_x[2] = {0ull, 0ull}, sum_r[2] = {0ull, 0ull};
+      const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
+      const uint64_t nm2 = f2pack(-m_use, -m_use);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[32];
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(fmaf(__uint_as_float(s[c][2 * e]), p.scale_log2, -m_new));
-          const float p1 = ex2(fmaf(__uint_as_float(s[c][2 * e + 1]), p.scale_log2, -m_new));
-          sum += p0 + p1;
+          float x0, x1, p0, p1;
+          f2unpack(ffma2(f2pack(__uint_as_float(s[c][2 * e]), __uint_as_float(s[c][2 * e + 1])),
+                         sc2, nm2),
+                   x0, x1);
+          // one pair in four goes through the FMA-pipe polynomial, the rest through MUFU
+          if ((e & 3) == 3) {
+            ex2_poly2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
           pk[e] = pack_bf16(p0, p1);
+          sum_x[e & 1] = fadd2(sum_x[e & 1], f2pack(p0, p1));
+          sum_r[e & 1] = fadd2(sum_r[e & 1], f2pack(__uint_as_float(pk[e] << 16),
+                                                   __uint_as_float(pk[e] & 0xffff0000u)));
         }
         // 32 keys -> 16 packed columns; two chunks share one 32-column store
         if (c & 1) {
@@ -281,22 +330,26 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       // P~ (bf16) over the first 64 columns of S_t
       tmem_st32(tS + 0, s[0]);
       tmem_st32(tS + 32, s[2]);
-      l = l * alpha + sum;
-      m = m_new;
-      if (j > 0) {
-        // O_t must hold PV_t(j-1) before it is rescaled
-        if (!(ok = W.wait(BAR_OD(t), (j - 1) & 1, 21))) break;
+      {
+        float a0, a1, b0, b1;
+        f2unpack(fadd2(sum_x[0], sum_x[1]), a0, a1);
+        f2unpack(fadd2(sum_r[0], sum_r[1]), b0, b1);
+        l = l * alpha + (a0 + a1);
+        lr = lr * alpha + (b0 + b1);
+      }
+      m = m_use;
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // O_t holds PV_t(j-1) (S_t(j) was issued only after it completed); rescale it
+        if (!(ok = W.wait_warp(BAR_OD(t), (j - 1) & 1, 21))) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * c, o);
-            tmem_wait_ld(o);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld(o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + 32 * c, o);
-          }
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + 32 * c, o);
         }
       }
       tmem_wait_st();
@@ -306,10 +359,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     }
     if (ok && n > 0) {
       // ---- epilogue: O / l -> bf16 -> global; L = (m + log2 l) * ln 2
-      ok = W.wait(BAR_OD(t), (n - 1) & 1, 22);
+      ok = W.wait_warp(BAR_OD(t), (n - 1) & 1, 22);
       if (ok) {
         tc_fence_after();
-        const float inv_l = 1.f / l;
+        const float inv_l = 1.f / lr;
         __nv_bfloat16* orow = p.o + (size_t(head) * p.N + row) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {

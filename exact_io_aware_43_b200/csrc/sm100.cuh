@@ -90,6 +90,12 @@ struct Waiter {
     return true;
   }
   __device__ __forceinline__ bool aborted() const { return *abort_flag != 0; }
+  // Warp-collective form: every lane gets the same answer, so warp-wide instructions that follow
+  // (tcgen05.ld/st are .sync.aligned) are never reached by part of a warp.
+  __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, int site) const {
+    const bool ok = wait(bar, parity, site);
+    return __all_sync(0xffffffffu, ok);
+  }
 };
 
 // ------------------------------------------------------------------------------------------
@@ -117,6 +123,53 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
           "r"(dst),
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
+}
+
+// 3-D tiled reduce-add of a shared-memory box into global memory (fp32 add), bulk-group tracked.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, uint32_t src, int x, int y,
+                                                  int z) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most N bulk groups of this thread still have to read their shared source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until every bulk group of this thread has completed (writes performed).
+__device__ __forceinline__ void bulk_wait_group_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Barrier among `count` threads on hardware barrier `id` (id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Same barrier, returning the AND of `pred` over the participating threads.
+__device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(uint32_t(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+// Per-warpgroup register reallocation (all four warps of a warpgroup execute it together).
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // Make generic-proxy shared-memory writes visible to the async proxy (tcgen05.mma operands).
@@ -256,6 +309,69 @@ __device__ __forceinline__ float lg2(float x) {
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x on the FMA/ALU pipes, for the share of exponentials taken off the MUFU unit.
+// Range reduction x = n + f with n = round(x) obtained by the 1.5*2^23 shifter trick (exact for
+// |x| < 2^22), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients are our own
+// minimax fit of the relative error on [-1/2, 1/2] (linear-programming fit on 4001 points;
+// max relative error 7.5e-5, far below the bf16 rounding applied to P afterwards); 2^n is
+// applied by adding n to the exponent field.  Inputs below -126 return 0 (masked scores are
+// -inf).  Valid for x <= 127.
+__device__ __forceinline__ float ex2_poly(float x) {
+  const float kShift = 12582912.0f;  // 1.5 * 2^23
+  const float xc = fmaxf(x, -126.0f);
+  const float t = xc + kShift;
+  const float n = t - kShift;
+  const float f = xc - n;
+  float p = fmaf(f, 0.0551716685295105f, 0.2426111251115799f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999280571937561f);
+  const uint32_t bits = __float_as_uint(p) + (__float_as_uint(t) << 23);
+  return x < -126.0f ? 0.f : __uint_as_float(bits);
+}
+
+// Paired fp32 arithmetic (sm_100 f32x2 instructions: two lanes of fp32 per instruction).
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// ex2_poly on a pair, with the range reduction and polynomial in paired fp32 instructions.
+__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& p0, float& p1) {
+  const float kShift = 12582912.0f;  // 1.5 * 2^23
+  const float a0 = fmaxf(x0, -126.0f), a1 = fmaxf(x1, -126.0f);
+  const uint64_t xc = f2pack(a0, a1);
+  const uint64_t t = fadd2(xc, f2pack(kShift, kShift));
+  const uint64_t nn = fadd2(t, f2pack(-kShift, -kShift));
+  float n0, n1;
+  f2unpack(nn, n0, n1);
+  const uint64_t f = fadd2(xc, f2pack(-n0, -n1));
+  uint64_t q = ffma2(f, f2pack(0.0551716685295105f, 0.0551716685295105f),
+                     f2pack(0.2426111251115799f, 0.2426111251115799f));
+  q = ffma2(q, f, f2pack(0.6932609677314758f, 0.6932609677314758f));
+  q = ffma2(q, f, f2pack(0.9999280571937561f, 0.9999280571937561f));
+  float q0, q1, t0, t1;
+  f2unpack(q, q0, q1);
+  f2unpack(t, t0, t1);
+  const float r0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+  p0 = x0 < -126.0f ? 0.f : r0;
+  p1 = x1 < -126.0f ? 0.f : r1;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
