@@ -24,6 +24,19 @@
 
 #include "sm100.cuh"
 
+// Tuning knobs (compile time).  FA_BWD_POLY_EVERY: one pair of exponentials in N goes through
+// the FMA-pipe polynomial (0: all MUFU).  FA_BWD_STAGES128: depth of the Q_i/dO_i ring for d=128.
+// FA_BWD_PAIRED: paired fp32 instructions and a block-level mask test in the P/dS arithmetic.
+#ifndef FA_BWD_POLY_EVERY
+#define FA_BWD_POLY_EVERY 0
+#endif
+#ifndef FA_BWD_STAGES128
+#define FA_BWD_STAGES128 3
+#endif
+#ifndef FA_BWD_PAIRED
+#define FA_BWD_PAIRED 0
+#endif
+
 namespace fattn {
 
 struct BwdParams {
@@ -127,7 +140,7 @@ struct BwdCfg {
   static constexpr int Q_BLK = BR * 128;          // bytes of one 64-column block of Q_i / dO_i
   static constexpr int KV_BYTES = KB * KV_BLK;
   static constexpr int Q_BYTES = KB * Q_BLK;
-  static constexpr int STAGES = D == 64 ? 3 : (D == 128 ? 2 : 1);
+  static constexpr int STAGES = D == 64 ? 3 : (D == 128 ? FA_BWD_STAGES128 : 1);
   static constexpr int THREADS = 320;
   static constexpr int DQ_WARP0 = 4;
   static constexpr int PRODUCER_WARP = 8;
@@ -146,7 +159,7 @@ struct BwdCfg {
   // dQ staging: slots of [64 queries][64 d] fp32 reduced into the accumulator by TMA
   static constexpr int DQ_CH = DO / 64;                          // 64-wide chunks per tile
   static constexpr int DQ_SLOT = BR * 64 * 4;
-  static constexpr int DQ_SLOTS = D == 64 ? 2 : (D == 128 ? 4 : 1);
+  static constexpr int DQ_SLOTS = D == 64 ? 2 : (D == 128 ? (FA_BWD_STAGES128 > 2 ? 2 : 4) : 1);
   static constexpr int OFF_DQS = OFF_ROWS + STAGES * 2 * BR * 4;
   static constexpr int OFF_BAR = OFF_DQS + DQ_SLOTS * DQ_SLOT;
   // barriers: kv_full, q_full[S], q_empty[S], s_full, s_free, dp_full, dp_free, p_full,
@@ -171,6 +184,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  FA_TRACE_DECL;
 
   // ---- work unit: (head, key block j, d slice); key blocks with more queries first
   const int per_head = p.nkb * C::NSL;
@@ -364,6 +378,33 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       // P^T = exp2(S^T s log2e - L2); zero for masked (causal key > query) and padded keys
       float pr[64];
       const int qbase = i * C::BR;
+#if FA_BWD_PAIRED
+      {
+        // only blocks that reach the diagonal (or padded keys) need the per-element mask
+        const bool need_mask = !key_ok || (CAUSAL && qbase < k0 + C::BC);
+        const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) {
+          const int c = 2 * c2;
+          float x0, x1;
+          f2unpack(ffma2(f2pack(__uint_as_float(st[c >> 5][c & 31]),
+                                __uint_as_float(st[c >> 5][(c & 31) + 1])),
+                         sc2, f2pack(-L2s[c], -L2s[c + 1])),
+                   x0, x1);
+          if (need_mask) {
+            if (!key_ok || (CAUSAL && key > qbase + c)) x0 = -INFINITY;
+            if (!key_ok || (CAUSAL && key > qbase + c + 1)) x1 = -INFINITY;
+          }
+          if (FA_BWD_POLY_EVERY > 0 &&
+              (c2 % (FA_BWD_POLY_EVERY > 0 ? FA_BWD_POLY_EVERY : 1)) == FA_BWD_POLY_EVERY - 1) {
+            ex2_poly2(x0, x1, pr[c], pr[c + 1]);
+          } else {
+            pr[c] = ex2(x0);
+            pr[c + 1] = ex2(x1);
+          }
+        }
+      }
+#else
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
         const float4 l4 = reinterpret_cast<const float4*>(L2s)[c4];
@@ -377,6 +418,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           pr[c] = valid ? ex2(x) : 0.f;
         }
       }
+#endif
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);

@@ -439,3 +439,16 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
   return bwd_dispatch(q, k, v, o, lse, dO, dq, dk, dv, B * H, N, d, causal != 0, scale, ws,
                       static_cast<cudaStream_t>(stream));
 }
+
+#ifdef FA_TRACE
+// Trace build only: copy out (all per-warp slots) and clear the pipeline trace.
+extern "C" int fa_trace_read(unsigned long long* host, int max_records) {
+  cudaDeviceSynchronize();
+  int n = (int)fattn::kTraceMax;
+  if (n > max_records) n = max_records;
+  cudaMemcpyFromSymbol(host, fattn::g_trace, sizeof(unsigned long long) * 2 * n);
+  static unsigned long long zeros[2 * fattn::kTraceMax];
+  cudaMemcpyToSymbol(fattn::g_trace, zeros, sizeof(zeros));
+  return n;
+}
+#endif

@@ -21,6 +21,30 @@
 
 #include "sm100.cuh"
 
+// Tuning knobs (compile time).  One pair of exponentials in FA_FWD_POLY_EVERY goes through the
+// FMA-pipe polynomial instead of MUFU (0: none); FA_FWD_POLY_CLAMPED picks the cheaper form
+// (masked scores are clamped to -126 first, giving ~2^-126 instead of 0 -- far below the bf16
+// resolution of P); FA_FWD_MAX3 uses the three-input max for the row maximum.
+#ifndef FA_FWD_POLY_EVERY
+#define FA_FWD_POLY_EVERY 0
+#endif
+// FA_FWD_RSUM: how O's normaliser is formed.  0: the fp32 sum (also used for L); 1: sum of the
+// bf16-rounded weights via integer unpack; 2: the same sum with mixed bf16+fp32 adds.
+#ifndef FA_FWD_RSUM
+#define FA_FWD_RSUM 2
+#endif
+// FA_FWD_RESCALE: the reference max moves (and O is rescaled) only when a row's max grows by more
+// than this many log2 units; 0 rescales on every increase.
+#ifndef FA_FWD_RESCALE
+#define FA_FWD_RESCALE 8.0f
+#endif
+#ifndef FA_FWD_POLY_CLAMPED
+#define FA_FWD_POLY_CLAMPED 0
+#endif
+#ifndef FA_FWD_MAX3
+#define FA_FWD_MAX3 0
+#endif
+
 namespace fattn {
 
 struct FwdParams {
@@ -81,6 +105,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  FA_TRACE_DECL;
 
   // ---- work unit: (head, query block), heaviest query blocks first when causal
   const int head = blockIdx.x / p.nqb;
@@ -256,7 +281,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     // m: reference max (log2 units of the scaled scores) that the exponentials and l are taken
     // against.  It only moves when a row's max grows by more than kRescale (2^8 in value): the
     // result is the same exact softmax, P~ stays <= 256, and O is rescaled far less often.
-    constexpr float kRescale = 8.0f;
+    constexpr float kRescale = FA_FWD_RESCALE;
     float m = -INFINITY;
     float l = 0.f;   // sum of the fp32 exponentials (for L)
     float lr = 0.f;  // sum of the bf16-rounded exponentials (divides O)
@@ -282,10 +307,19 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       float mx8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+#if FA_FWD_MAX3
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; e += 2)
+          mx8[(e >> 1) & 7] = fmax3(mx8[(e >> 1) & 7], __uint_as_float(s[c][e]),
+                                    __uint_as_float(s[c][e + 1]));
+#else
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(s[c][e]));
+#endif
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * p.scale_log2;
@@ -306,17 +340,30 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           f2unpack(ffma2(f2pack(__uint_as_float(s[c][2 * e]), __uint_as_float(s[c][2 * e + 1])),
                          sc2, nm2),
                    x0, x1);
-          // one pair in four goes through the FMA-pipe polynomial, the rest through MUFU
-          if ((e & 3) == 3) {
-            ex2_poly2(x0, x1, p0, p1);
+          // one pair in FA_FWD_POLY_EVERY goes through the FMA-pipe polynomial, the rest MUFU
+          if (FA_FWD_POLY_EVERY > 0 && (e % (FA_FWD_POLY_EVERY > 0 ? FA_FWD_POLY_EVERY : 1)) ==
+                                           FA_FWD_POLY_EVERY - 1) {
+            if (FA_FWD_POLY_CLAMPED)
+              ex2_poly2_clamped(fmaxf(x0, -126.f), fmaxf(x1, -126.f), p0, p1);
+            else
+              ex2_poly2(x0, x1, p0, p1);
           } else {
             p0 = ex2(x0);
             p1 = ex2(x1);
           }
           pk[e] = pack_bf16(p0, p1);
           sum_x[e & 1] = fadd2(sum_x[e & 1], f2pack(p0, p1));
+#if FA_FWD_RSUM == 1
           sum_r[e & 1] = fadd2(sum_r[e & 1], f2pack(__uint_as_float(pk[e] << 16),
                                                    __uint_as_float(pk[e] & 0xffff0000u)));
+#elif FA_FWD_RSUM == 2
+          {
+            float r0, r1;
+            f2unpack(sum_r[e & 1], r0, r1);
+            add_bf16pair_f32(pk[e], r0, r1);
+            sum_r[e & 1] = f2pack(r0, r1);
+          }
+#endif
         }
         // 32 keys -> 16 packed columns; two chunks share one 32-column store
         if (c & 1) {
@@ -335,7 +382,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         f2unpack(fadd2(sum_x[0], sum_x[1]), a0, a1);
         f2unpack(fadd2(sum_r[0], sum_r[1]), b0, b1);
         l = l * alpha + (a0 + a1);
-        lr = lr * alpha + (b0 + b1);
+        lr = (FA_FWD_RSUM == 0) ? l : lr * alpha + (b0 + b1);
       }
       m = m_use;
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {

@@ -18,6 +18,38 @@ namespace fattn {
 // ------------------------------------------------------------------------------------------
 __device__ int g_status[2];
 
+// ------------------------------------------------------------------------------------------
+// Optional pipeline trace (compiled in only with -DFA_TRACE): lane 0 of each warp of one chosen
+// CTA appends (SM clock, warp, event, iteration) records; fa_trace_read copies them out.
+// ------------------------------------------------------------------------------------------
+#ifdef FA_TRACE
+#ifndef FA_TRACE_CTA
+#define FA_TRACE_CTA 300
+#endif
+constexpr unsigned kTraceWarps = 16, kTracePerWarp = 4096, kTraceMax = kTraceWarps * kTracePerWarp;
+__device__ unsigned long long g_trace[2 * kTraceMax];
+__device__ unsigned int g_trace_n;
+// per-warp slots, plain stores (no atomics): the record costs a few issue cycles only
+#define FA_TRACE_EV(code, it)                                                                  \
+  do {                                                                                         \
+    if (blockIdx.x == FA_TRACE_CTA && (threadIdx.x & 31) == 0 && (threadIdx.x >> 5) < 16 &&    \
+        fa_trace_k < ::fattn::kTracePerWarp) {                                                 \
+      const unsigned k_ = (threadIdx.x >> 5) * ::fattn::kTracePerWarp + fa_trace_k++;          \
+      ::fattn::g_trace[2 * k_] = clock64();                                                    \
+      ::fattn::g_trace[2 * k_ + 1] = ((unsigned long long)(threadIdx.x >> 5) << 40) |          \
+                                     ((unsigned long long)(code) << 32) | (unsigned)(it);      \
+    }                                                                                          \
+  } while (0)
+#define FA_TRACE_DECL unsigned fa_trace_k = 0
+#else
+#define FA_TRACE_EV(code, it) \
+  do {                        \
+  } while (0)
+#define FA_TRACE_DECL \
+  do {                \
+  } while (0)
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -61,6 +93,22 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t bar, uint32_t parity)
   return ok;
 }
 
+// try_wait with a suspend-time hint: the waiting thread sleeps in hardware until the phase
+// completes or `hint_ns` elapses, instead of spinning and taking issue slots from the warps
+// that compute on the same SM sub-partition.
+__device__ __forceinline__ uint32_t mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                        uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok;
+}
+
 // Bounded wait shared by all roles of one CTA.  `abort_flag` lives in shared memory; once any
 // thread of the CTA gives up, every later wait returns false at once so all roles fall through
 // to the teardown instead of hanging.  Returns true when the phase completed.
@@ -68,11 +116,14 @@ struct Waiter {
   volatile int* abort_flag;
   uint64_t limit_ns;
 
+  // After the first failed try_wait the thread sleeps in try_wait (up to 1 ms per call, woken
+  // when the phase completes); between calls it checks the abort flag and the deadline.  A
+  // busy spin measurably slowed both kernels by taking issue slots from the computing warps.
   __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, int site) const {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
-      if (mbar_try_wait(bar, parity)) return true;
+      if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
       if (*abort_flag) return false;
       if (global_ns() - t0 > limit_ns) {
         *abort_flag = 1;
@@ -349,6 +400,27 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
+// Cheaper pair form for inputs already known to be >= -126 (callers clamp): no select, and
+// the exponent is inserted with one integer multiply-add per value.
+__device__ __forceinline__ void ex2_poly2_clamped(float x0, float x1, float& p0, float& p1) {
+  const float kShift = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t xc = f2pack(x0, x1);
+  const uint64_t t = fadd2(xc, f2pack(kShift, kShift));
+  const uint64_t nn = fadd2(t, f2pack(-kShift, -kShift));
+  float n0, n1;
+  f2unpack(nn, n0, n1);
+  const uint64_t f = fadd2(xc, f2pack(-n0, -n1));
+  uint64_t q = ffma2(f, f2pack(0.0551716685295105f, 0.0551716685295105f),
+                     f2pack(0.2426111251115799f, 0.2426111251115799f));
+  q = ffma2(q, f, f2pack(0.6932609677314758f, 0.6932609677314758f));
+  q = ffma2(q, f, f2pack(0.9999280571937561f, 0.9999280571937561f));
+  float q0, q1, t0, t1;
+  f2unpack(q, q0, q1);
+  f2unpack(t, t0, t1);
+  p0 = __uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(q0));
+  p1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(q1));
+}
+
 // ex2_poly on a pair, with the range reduction and polynomial in paired fp32 instructions.
 __device__ __forceinline__ void ex2_poly2(float x0, float x1, float& p0, float& p1) {
   const float kShift = 12582912.0f;  // 1.5 * 2^23
@@ -370,6 +442,20 @@ __device__ __forceinline__ void ex2_poly2(float x0, float x1, float& p0, float& 
   const float r1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
   p0 = x0 < -126.0f ? 0.f : r0;
   p1 = x1 < -126.0f ? 0.f : r1;
+}
+
+// acc0 += lo(bf16 pair), acc1 += hi(bf16 pair), with mixed-precision fp32 + bf16 adds.
+__device__ __forceinline__ void add_bf16pair_f32(uint32_t pk, float& acc0, float& acc1) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}\n"
+      : "+f"(acc0), "+f"(acc1)
+      : "r"(pk));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

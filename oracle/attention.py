@@ -178,3 +178,42 @@ def attention_head_subset(q, k, v, do, causal: bool, scale: float, heads):
             res += [dq[0, 0], dk[0, 0], dv[0, 0]]
         out[(b, h)] = tuple(res)
     return out
+
+
+def attention_rows(q, k, v, rows, causal: bool, scale: float):
+    """Forward outputs of selected query rows of ONE head (q, k, v: [N, d] arrays).
+
+    A row of the definition needs only its own scores against all keys ([P2], [P3] formula), so
+    sampled rows of very long sequences are computed exactly without the N x N matrix.
+    Returns (O_rows [len(rows), d], L_rows [len(rows)]).
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    rows = np.asarray(rows)
+    s = scale * (q[rows] @ k.T)
+    if causal:
+        s = np.where(np.arange(k.shape[0])[None, :] > rows[:, None], -np.inf, s)
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=1, keepdims=True)
+    return (e / l) @ v, (m + np.log(l))[:, 0]
+
+
+def attention_dq_rows(q, k, v, do, rows, causal: bool, scale: float):
+    """dQ of selected query rows of ONE head: dQ_i = scale * sum_j P_ij (dP_ij - D_i) k_j with
+    dP_ij = dO_i . v_j and D_i = dO_i . O_i -- row i needs only its own P row and O row."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    do = np.asarray(do, np.float64)
+    rows = np.asarray(rows)
+    O, L = attention_rows(q, k, v, rows, causal, scale)
+    s = scale * (q[rows] @ k.T)
+    if causal:
+        s = np.where(np.arange(k.shape[0])[None, :] > rows[:, None], -np.inf, s)
+    p = np.exp(s - L[:, None])
+    dp = do[rows] @ v.T
+    D = np.sum(do[rows] * O, axis=1)
+    ds = p * (dp - D[:, None])
+    return scale * (ds @ k)

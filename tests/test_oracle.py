@@ -413,3 +413,34 @@ def test_planted_mistake_is_caught(name, fwd, online, bwd):
 
 def test_oracle_passes_all_pins():
     assert run_pins(attention_forward, attention_forward_online, attention_backward) == []
+
+
+# --------------------------------------------------------------------------------------------
+# row-sampled oracle functions (used where a head is too long for the full N x N oracle)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_match_full_oracle(causal):
+    q, k, v, do = (rand((1, 1, 45, 8), s) for s in (80, 81, 82, 83))
+    O, L = attention_forward(q, k, v, causal, 0.3)
+    dq, _, _ = attention_backward(q, k, v, O, L, do, causal, 0.3)
+    rows = np.array([0, 1, 7, 30, 44])
+    Or, Lr = __import__("oracle").attention_rows(q[0, 0], k[0, 0], v[0, 0], rows, causal, 0.3)
+    dqr = __import__("oracle").attention_dq_rows(q[0, 0], k[0, 0], v[0, 0], do[0, 0], rows, causal,
+                                               0.3)
+    assert np.allclose(Or, O[0, 0, rows], atol=1e-13) and np.allclose(Lr, L[0, 0, rows], atol=1e-13)
+    assert np.allclose(dqr, dq[0, 0, rows], atol=1e-12)
+
+
+def test_rows_closed_forms():
+    """Q = 0 rows: L = ln(i+1) causal, O = prefix mean; dQ of row 0 (causal) is exactly 0."""
+    import oracle as orc
+    N = 33
+    q = np.zeros((N, 4))
+    k, v, do = rand((N, 4), 84), rand((N, 4), 85), rand((N, 4), 86)
+    rows = np.array([0, 5, 32])
+    O, L = orc.attention_rows(q, k, v, rows, True, 0.5)
+    assert np.allclose(L, np.log(rows + 1), atol=1e-14)
+    assert np.allclose(O, np.stack([v[:r + 1].mean(0) for r in rows]), atol=1e-14)
+    dq = orc.attention_dq_rows(rand((N, 4), 87), k, v, do, np.array([0]), True, 0.5)
+    assert np.allclose(dq, 0.0, atol=1e-15)
