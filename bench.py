@@ -57,7 +57,7 @@ def load_peaks():
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="fattn", choices=["fattn", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -36,6 +36,11 @@
 #ifndef FA_BWD_PAIRED
 #define FA_BWD_PAIRED 0
 #endif
+// FA_BWD_MASKFAST: query blocks entirely below the diagonal (and without padded keys) skip the
+// per-element mask test.
+#ifndef FA_BWD_MASKFAST
+#define FA_BWD_MASKFAST 1
+#endif
 
 namespace fattn {
 
@@ -405,17 +410,31 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         }
       }
 #else
+      const bool need_mask = !FA_BWD_MASKFAST || !key_ok || (CAUSAL && qbase < k0 + C::BC);
+      if (need_mask) {
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 l4 = reinterpret_cast<const float4*>(L2s)[c4];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l4 = reinterpret_cast<const float4*>(L2s)[c4];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * c4 + e;
-          const float x = fmaf(__uint_as_float(st[c >> 5][c & 31]), p.scale_log2, -lv[e]);
-          bool valid = key_ok;
-          if (CAUSAL) valid = valid && (key <= qbase + c);
-          pr[c] = valid ? ex2(x) : 0.f;
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            const float x = fmaf(__uint_as_float(st[c >> 5][c & 31]), p.scale_log2, -lv[e]);
+            bool valid = key_ok;
+            if (CAUSAL) valid = valid && (key <= qbase + c);
+            pr[c] = valid ? ex2(x) : 0.f;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l4 = reinterpret_cast<const float4*>(L2s)[c4];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            pr[c] = ex2(fmaf(__uint_as_float(st[c >> 5][c & 31]), p.scale_log2, -lv[e]));
+          }
         }
       }
 #endif

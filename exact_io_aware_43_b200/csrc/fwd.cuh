@@ -44,6 +44,21 @@
 #ifndef FA_FWD_MAX3
 #define FA_FWD_MAX3 0
 #endif
+// FA_FWD_MMA_SPLIT: 1 gives each query tile its own MMA-issuing warp (no head-of-line blocking
+// between the tiles); 0 issues both tiles' MMAs from one thread in a fixed interleaved order.
+#ifndef FA_FWD_MMA_SPLIT
+#define FA_FWD_MMA_SPLIT 0
+#endif
+// FA_FWD_TOKEN: the two softmax warpgroups take turns on the exponentials (0, 1, 0, 1, ...),
+// passing a token through an mbarrier.
+#ifndef FA_FWD_TOKEN
+#define FA_FWD_TOKEN 0
+#endif
+// FA_FWD_EAGER_PV: after PV_0(j) the single issuer probes (without blocking) whether P_1(j) is
+// already written and, if so, queues PV_1(j) before it waits for PV_0(j) to finish.
+#ifndef FA_FWD_EAGER_PV
+#define FA_FWD_EAGER_PV 0
+#endif
 
 namespace fattn {
 
@@ -87,7 +102,7 @@ struct FwdCfg {
   static constexpr int OFF_BAR = OFF_V + STAGES * KVTILE_BYTES;
   // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT], p_full[NQT],
   //           o_done[NQT], drain
-  static constexpr int NBAR = 1 + 4 * STAGES + 3 * NQT + 1;
+  static constexpr int NBAR = 1 + 4 * STAGES + 5 * NQT;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem address + abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);   // Q, K both K-major
@@ -133,25 +148,32 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
   auto BAR_SF = [&](int t) { return bar(1 + 4 * C::STAGES + t); };
   auto BAR_PF = [&](int t) { return bar(1 + 4 * C::STAGES + NQT + t); };
   auto BAR_OD = [&](int t) { return bar(1 + 4 * C::STAGES + 2 * NQT + t); };
-  const uint32_t BAR_DRAIN = bar(C::NBAR - 1);
+  auto BAR_DRAIN = [&](int t) { return bar(1 + 4 * C::STAGES + 3 * NQT + t); };
+  auto BAR_XU = [&](int t) { return bar(1 + 4 * C::STAGES + 4 * NQT + t); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   const Waiter W{abort_flag, p.limit_ns};
 
+  int n_active = 0;
+#pragma unroll
+  for (int t = 0; t < NQT; ++t) n_active += (nkv[t] > 0);
+  // with one MMA warp per tile every active tile's warp releases each K/V stage
+  const int kv_release = FA_FWD_MMA_SPLIT ? n_active : 1;
   if (threadIdx.x == 0) {
     mbar_init(BAR_Q, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(BAR_KF(s), 1);
-      mbar_init(BAR_KE(s), 1);
+      mbar_init(BAR_KE(s), kv_release);
       mbar_init(BAR_VF(s), 1);
-      mbar_init(BAR_VE(s), 1);
+      mbar_init(BAR_VE(s), kv_release);
     }
     for (int t = 0; t < NQT; ++t) {
       mbar_init(BAR_SF(t), 1);
       mbar_init(BAR_PF(t), 4);
       mbar_init(BAR_OD(t), 1);
     }
-    mbar_init(BAR_DRAIN, 1);
+    for (int t = 0; t < NQT; ++t) mbar_init(BAR_DRAIN(t), 1);
+    for (int t = 0; t < NQT; ++t) mbar_init(BAR_XU(t), 4);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -163,6 +185,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  FA_TRACE_EV(30, 0);
   if (warp >= C::SOFTMAX_WARPS) {
    // ================================================================ control warpgroup
    if constexpr (C::REALLOC) regs_dec<C::CTRL_REGS>();
@@ -186,6 +209,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         const int s = j % C::STAGES;
         const uint32_t ph = (j / C::STAGES) & 1;
         if (!W.wait(BAR_KE(s), ph ^ 1, 1)) break;
+        FA_TRACE_EV(20, j);
         mbar_arrive_expect_tx(BAR_KF(s), C::KVTILE_BYTES);
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_3d(sbase + C::OFF_K + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmK,
@@ -194,6 +218,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           ++j;  // the K load of tile j is in flight
           break;
         }
+        FA_TRACE_EV(21, j);
         mbar_arrive_expect_tx(BAR_VF(s), C::KVTILE_BYTES);
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_3d(sbase + C::OFF_V + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmV,
@@ -208,7 +233,59 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         }
       }
     }
-  } else if (warp == C::MMA_WARP) {
+  } else if (FA_FWD_MMA_SPLIT && warp >= C::MMA_WARP && warp < C::MMA_WARP + NQT) {
+    // ---------------------------------------------------------------- MMA issuer of tile t
+    // Each query tile has its own issuing warp, so one tile's wait never delays the other's
+    // MMAs.  Per KV tile j: PV_t(j) once softmax t has written P_t(j), then S_t(j+1), which
+    // overwrites the tensor memory holding P_t(j) and therefore waits for PV_t(j) to complete.
+    const int t = warp - C::MMA_WARP;
+    const int n = nkv[t];
+    if (lane == 0 && n > 0) {
+      const uint32_t q_addr = sbase + C::OFF_Q + t * C::QTILE_BYTES;
+      auto issue_s = [&](uint32_t k_addr) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ss(tmem + C::TMEM_S + t * C::BN, sdesc_sw128(q_addr + koff, 16, 1024),
+                 sdesc_sw128(k_addr + koff, 16, 1024), C::IDESC_S, kk > 0);
+        }
+        tc_commit(BAR_SF(t));
+      };
+      bool ok = W.wait(BAR_Q, 0, 10) && W.wait(BAR_KF(0), 0, 11);
+      if (ok) {
+        tc_fence_after();
+        issue_s(sbase + C::OFF_K);
+        tc_commit(BAR_KE(0));
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int s = j % C::STAGES;
+        const int s1 = (j + 1) % C::STAGES;
+        const uint32_t v_addr = sbase + C::OFF_V + s * C::KVTILE_BYTES;
+        if (!(ok = W.wait(BAR_VF(s), (j / C::STAGES) & 1, 13))) break;
+        FA_TRACE_EV(1 + 16 * t, j);
+        if (!(ok = W.wait(BAR_PF(t), j & 1, 14))) break;
+        FA_TRACE_EV(2 + 16 * t, j);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk)
+          mma_ts(tmem + C::TMEM_O + t * D, tmem + C::TMEM_S + t * C::BN + kk * 8,
+                 sdesc_sw128(v_addr + kk * 2048, C::BN * 128, 1024), C::IDESC_PV,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(BAR_OD(t));
+        tc_commit(BAR_VE(s));
+        if (j + 1 < n) {
+          if (!(ok = W.wait(BAR_KF(s1), ((j + 1) / C::STAGES) & 1, 11))) break;
+          if (!(ok = W.wait(BAR_OD(t), j & 1, 12))) break;  // P_t(j) consumed
+          FA_TRACE_EV(3 + 16 * t, j);
+          tc_fence_after();
+          issue_s(sbase + C::OFF_K + s1 * C::KVTILE_BYTES);
+          tc_commit(BAR_KE(s1));
+        }
+      }
+      tc_commit(BAR_DRAIN(t));
+      W.drain(BAR_DRAIN(t), 0);
+    }
+  } else if (!FA_FWD_MMA_SPLIT && warp == C::MMA_WARP) {
     // ---------------------------------------------------------------- MMA issuer
     // Order per KV tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  S_t(j+1) overwrites the tensor
     // memory that holds P_t(j), so it waits for PV_t(j) to complete; issuing it right behind
@@ -238,9 +315,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         const uint32_t k1_addr = sbase + C::OFF_K + s1 * C::KVTILE_BYTES;
         if (!(ok = W.wait(BAR_VF(s), (j / C::STAGES) & 1, 13))) break;
         bool k_ready = false;
-        for (int t = 0; t < NQT && ok; ++t) {
-          if (j >= nkv[t]) continue;
-          if (!(ok = W.wait(BAR_PF(t), j & 1, 14))) break;
+        bool pv_issued[NQT];
+#pragma unroll
+        for (int t = 0; t < NQT; ++t) pv_issued[t] = false;
+        auto issue_pv = [&](int t) {
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < C::BN / 16; ++kk) {
@@ -251,10 +329,24 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
                    (j > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(BAR_OD(t));
+          pv_issued[t] = true;
+        };
+        for (int t = 0; t < NQT && ok; ++t) {
+          if (j >= nkv[t]) continue;
+          if (!pv_issued[t]) {
+            FA_TRACE_EV(1 + 16 * t, j);
+            if (!(ok = W.wait(BAR_PF(t), j & 1, 14))) break;
+            FA_TRACE_EV(2 + 16 * t, j);
+            issue_pv(t);
+          }
+          if (FA_FWD_EAGER_PV && NQT == 2 && t == 0 && j < nkv[1] &&
+              mbar_test_wait(BAR_PF(1), j & 1))
+            issue_pv(1);
           if (j + 1 < nkv[t]) {
             if (!k_ready && !(ok = W.wait(BAR_KF(s1), ((j + 1) / C::STAGES) & 1, 11))) break;
             k_ready = true;
             if (!(ok = W.wait(BAR_OD(t), j & 1, 12))) break;  // P_t(j) consumed
+            FA_TRACE_EV(3 + 16 * t, j);
             tc_fence_after();
             issue_s(t, k1_addr);
           }
@@ -264,8 +356,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         if (k_ready) tc_commit(BAR_KE(s1));
       }
       // every MMA issued above has completed before the tensor memory is released
-      tc_commit(BAR_DRAIN);
-      W.drain(BAR_DRAIN, 0);
+      tc_commit(BAR_DRAIN(0));
+      W.drain(BAR_DRAIN(0), 0);
     }
    }
   } else {
@@ -287,13 +379,16 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     float lr = 0.f;  // sum of the bf16-rounded exponentials (divides O)
     bool ok = true;
     for (int j = 0; j < n; ++j) {
+      FA_TRACE_EV(10, j);
       if (!(ok = W.wait_warp(BAR_SF(t), j & 1, 20))) break;
+      FA_TRACE_EV(11, j);
       tc_fence_after();
       uint32_t s[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_wait_ld(s[c]);
+      FA_TRACE_EV(15, j);
       // mask keys past N and, on diagonal tiles, keys after the query (causal)
       const int key0 = j * C::BN;
       const int lim = CAUSAL ? min(row, p.N - 1) - key0 : (p.N - 1) - key0;  // last valid col
@@ -322,6 +417,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
 #endif
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      FA_TRACE_EV(16, j);
+      if (FA_FWD_TOKEN && NQT == 2) {
+        const int o = 1 - t;
+        const int jo = t == 0 ? j - 1 : j;  // the other tile's KV tile that goes first
+        if (jo >= 0 && jo < nkv[o] && !(ok = W.wait_warp(BAR_XU(o), jo & 1, 23))) break;
+      }
       const float m_tile = mx * p.scale_log2;
       const float m_use = (j == 0 || m_tile > m + kRescale) ? fmaxf(m, m_tile) : m;
       const float alpha = (j == 0 || m_use == m) ? 1.f : ex2(m - m_use);
@@ -374,6 +475,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           for (int e = 0; e < 16; ++e) s[c][e] = pk[e];
         }
       }
+      FA_TRACE_EV(12, j);
+      if (FA_FWD_TOKEN && NQT == 2) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR_XU(t));
+      }
       // P~ (bf16) over the first 64 columns of S_t
       tmem_st32(tS + 0, s[0]);
       tmem_st32(tS + 32, s[2]);
@@ -403,6 +509,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_PF(t));
+      FA_TRACE_EV(13, j);
     }
     if (ok && n > 0) {
       // ---- epilogue: O / l -> bf16 -> global; L = (m + log2 l) * ln 2
