@@ -24,22 +24,19 @@
 
 #include "sm100.cuh"
 
-// Tuning knobs (compile time).  FA_BWD_POLY_EVERY: one pair of exponentials in N goes through
-// the FMA-pipe polynomial (0: all MUFU).  FA_BWD_STAGES128: depth of the Q_i/dO_i ring for d=128.
-// FA_BWD_PAIRED: paired fp32 instructions and a block-level mask test in the P/dS arithmetic.
-#ifndef FA_BWD_POLY_EVERY
-#define FA_BWD_POLY_EVERY 0
-#endif
+// Tuning knobs (compile time).  FA_BWD_STAGES128: depth of the Q_i/dO_i ring for d=128.
 #ifndef FA_BWD_STAGES128
 #define FA_BWD_STAGES128 3
-#endif
-#ifndef FA_BWD_PAIRED
-#define FA_BWD_PAIRED 0
 #endif
 // FA_BWD_MASKFAST: query blocks entirely below the diagonal (and without padded keys) skip the
 // per-element mask test.
 #ifndef FA_BWD_MASKFAST
 #define FA_BWD_MASKFAST 1
+#endif
+// FA_BWD_SPLIT: two P/dS warpgroups, each owning 32 of the 64 query columns of S^T / dP^T (the
+// arithmetic is elementwise, so the halves are independent); 0: one warpgroup, all 64 columns.
+#ifndef FA_BWD_SPLIT
+#define FA_BWD_SPLIT 1
 #endif
 
 namespace fattn {
@@ -146,10 +143,13 @@ struct BwdCfg {
   static constexpr int KV_BYTES = KB * KV_BLK;
   static constexpr int Q_BYTES = KB * Q_BLK;
   static constexpr int STAGES = D == 64 ? 3 : (D == 128 ? FA_BWD_STAGES128 : 1);
-  static constexpr int THREADS = 320;
-  static constexpr int DQ_WARP0 = 4;
-  static constexpr int PRODUCER_WARP = 8;
-  static constexpr int MMA_WARP = 9;
+  static constexpr bool SPLIT = FA_BWD_SPLIT != 0;
+  static constexpr int CMP_WARPS = SPLIT ? 8 : 4;        // P/dS warps (one or two warpgroups)
+  static constexpr int NCOL = SPLIT ? 32 : 64;           // query columns per P/dS thread
+  static constexpr int THREADS = SPLIT ? 512 : 320;
+  static constexpr int DQ_WARP0 = CMP_WARPS;
+  static constexpr int PRODUCER_WARP = CMP_WARPS + 4;
+  static constexpr int MMA_WARP = CMP_WARPS + 5;
   // tensor memory columns
   static constexpr int T_S = 0, T_DP = 64, T_P = 128, T_DS = 160, T_DQ = 192, T_DV = 256,
                        T_DK = 256 + DO;
@@ -222,11 +222,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       mbar_init(BAR_QE(s), 1);
     }
     mbar_init(BAR_SF, 1);
-    mbar_init(BAR_SFREE, 4);
+    mbar_init(BAR_SFREE, C::CMP_WARPS);
     mbar_init(BAR_DPF, 1);
-    mbar_init(BAR_DPFREE, 4);
-    mbar_init(BAR_PF, 4);
-    mbar_init(BAR_DSF, 4);
+    mbar_init(BAR_DPFREE, C::CMP_WARPS);
+    mbar_init(BAR_PF, C::CMP_WARPS);
+    mbar_init(BAR_DSF, C::CMP_WARPS);
     mbar_init(BAR_DVD, 1);
     mbar_init(BAR_DQF, 1);
     mbar_init(BAR_DQE, 4);
@@ -261,6 +261,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const int i = i_start + it;
         const int s = it % C::STAGES;
         if (!W.wait(BAR_QE(s), ((it / C::STAGES) & 1) ^ 1, 31)) break;
+        FA_TRACE_EV(20, it);
         mbar_arrive_expect_tx(BAR_QF(s), 2 * C::Q_BYTES + 2 * C::BR * 4);
         for (int kb = 0; kb < C::KB; ++kb) {
           tma_load_3d(sbase + C::OFF_Q + s * C::Q_BYTES + kb * C::Q_BLK, &tmQ, BAR_QF(s), kb * 64,
@@ -317,7 +318,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const uint32_t q_addr = sbase + C::OFF_Q + s * C::Q_BYTES;
         const uint32_t do_addr = sbase + C::OFF_DO + s * C::Q_BYTES;
         // dV += P^T dO_i
+        FA_TRACE_EV(1, it);
         if (!(ok = W.wait(BAR_PF, it & 1, 42))) break;
+        FA_TRACE_EV(2, it);
         tc_fence_after();
         issue_kv(C::T_DV, C::T_P, do_addr, it > 0);
         tc_commit(BAR_DVD);
@@ -327,6 +330,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         auto issue_next_st = [&]() -> bool {
           if (!W.wait(BAR_QF(sn), ((it + 1) / C::STAGES) & 1, 43)) return false;
           if (!W.wait(BAR_SFREE, it & 1, 44)) return false;
+          FA_TRACE_EV(3, it);
           tc_fence_after();
           issue_st(C::T_S, k_addr, sbase + C::OFF_Q + sn * C::Q_BYTES);
           tc_commit(BAR_SF);
@@ -334,8 +338,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         };
         if (more && C::STAGES > 1 && !(ok = issue_next_st())) break;
         // dK += dS^T Q_i ; dQ_i^T = K_j^T dS^T
+        FA_TRACE_EV(4, it);
         if (!(ok = W.wait(BAR_DSF, it & 1, 45))) break;
+        FA_TRACE_EV(5, it);
         if (it > 0 && !(ok = W.wait(BAR_DQE, (it - 1) & 1, 46))) break;
+        FA_TRACE_EV(6, it);
         tc_fence_after();
         issue_kv(C::T_DK, C::T_DS, q_addr, it > 0);
 #pragma unroll
@@ -348,6 +355,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         if (more) {
           if (C::STAGES == 1 && !(ok = issue_next_st())) break;
           if (!(ok = W.wait(BAR_DPFREE, it & 1, 47))) break;
+          FA_TRACE_EV(7, it);
           tc_fence_after();
           issue_st(C::T_DP, v_addr, sbase + C::OFF_DO + sn * C::Q_BYTES);
           tc_commit(BAR_DPF);
@@ -356,64 +364,44 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tc_commit(BAR_DRAIN);
       W.drain(BAR_DRAIN, 0);
     }
-  } else if (warp < 4) {
-    // ---------------------------------------------------------------- P / dS warpgroup
-    const int r = threadIdx.x;               // key row within the block == TMEM lane
+  } else if (warp < C::CMP_WARPS) {
+    // ---------------------------------------------------------------- P / dS warpgroup(s)
+    // Thread = key row (TMEM lane).  With two warpgroups, warpgroup h owns query columns
+    // [32h, 32h+32) of every tile; the arithmetic is elementwise, so the halves never meet.
+    constexpr int NC = C::NCOL;
+    const int h = warp >> 2;                 // column half (0 when not split)
+    const int c0 = h * NC;                   // first query column of this thread
+    const int r = (warp & 3) * 32 + lane;    // key row within the block == TMEM lane
     const int key = k0 + r;
     const bool key_ok = key < p.N;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     uint8_t* ds_row = smem + C::OFF_DS + r * 128;
     bool ok = true;
     for (int it = 0; it < nit; ++it) {
       const int i = i_start + it;
       const int s = it % C::STAGES;
-      const float* L2s = rows_smem + s * 2 * C::BR;
-      const float* Ds = L2s + C::BR;
+      const float* L2s = rows_smem + s * 2 * C::BR + c0;
+      const float* Ds = rows_smem + s * 2 * C::BR + C::BR + c0;
+      FA_TRACE_EV(10, it);
       if (!(ok = W.wait_warp(BAR_SF, it & 1, 50))) break;
       if (!(ok = W.wait_warp(BAR_QF(s), (it / C::STAGES) & 1, 51))) break;
+      FA_TRACE_EV(11, it);
       tc_fence_after();
-      uint32_t st[2][32];
-      tmem_ld32(tmem + lane_base + C::T_S, st[0]);
-      tmem_ld32(tmem + lane_base + C::T_S + 32, st[1]);
-      tmem_wait_ld(st[0]);
-      tmem_wait_ld(st[1]);
+      uint32_t st[NC / 32][32];
+#pragma unroll
+      for (int q = 0; q < NC / 32; ++q) tmem_ld32(tmem + lane_base + C::T_S + c0 + 32 * q, st[q]);
+#pragma unroll
+      for (int q = 0; q < NC / 32; ++q) tmem_wait_ld(st[q]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_SFREE);
       // P^T = exp2(S^T s log2e - L2); zero for masked (causal key > query) and padded keys
-      float pr[64];
-      const int qbase = i * C::BR;
-#if FA_BWD_PAIRED
-      {
-        // only blocks that reach the diagonal (or padded keys) need the per-element mask
-        const bool need_mask = !key_ok || (CAUSAL && qbase < k0 + C::BC);
-        const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
-#pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          const int c = 2 * c2;
-          float x0, x1;
-          f2unpack(ffma2(f2pack(__uint_as_float(st[c >> 5][c & 31]),
-                                __uint_as_float(st[c >> 5][(c & 31) + 1])),
-                         sc2, f2pack(-L2s[c], -L2s[c + 1])),
-                   x0, x1);
-          if (need_mask) {
-            if (!key_ok || (CAUSAL && key > qbase + c)) x0 = -INFINITY;
-            if (!key_ok || (CAUSAL && key > qbase + c + 1)) x1 = -INFINITY;
-          }
-          if (FA_BWD_POLY_EVERY > 0 &&
-              (c2 % (FA_BWD_POLY_EVERY > 0 ? FA_BWD_POLY_EVERY : 1)) == FA_BWD_POLY_EVERY - 1) {
-            ex2_poly2(x0, x1, pr[c], pr[c + 1]);
-          } else {
-            pr[c] = ex2(x0);
-            pr[c + 1] = ex2(x1);
-          }
-        }
-      }
-#else
+      float pr[NC];
+      const int qbase = i * C::BR + c0;
       const bool need_mask = !FA_BWD_MASKFAST || !key_ok || (CAUSAL && qbase < k0 + C::BC);
       if (need_mask) {
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
+        for (int c4 = 0; c4 < NC / 4; ++c4) {
           const float4 l4 = reinterpret_cast<const float4*>(L2s)[c4];
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
@@ -427,7 +415,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         }
       } else {
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
+        for (int c4 = 0; c4 < NC / 4; ++c4) {
           const float4 l4 = reinterpret_cast<const float4*>(L2s)[c4];
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
@@ -437,30 +425,34 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           }
         }
       }
-#endif
-      uint32_t pk[32];
+      uint32_t pk[NC / 2];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
+      for (int c = 0; c < NC / 2; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
       // P^T columns are free once dV(it-1) has read them
       if (it > 0 && !(ok = W.wait_warp(BAR_DVD, (it - 1) & 1, 52))) break;
       tc_fence_after();
-      tmem_st32(tmem + lane_base + C::T_P, pk);
+      if (NC == 64)
+        tmem_st32(tmem + lane_base + C::T_P, *reinterpret_cast<uint32_t(*)[32]>(pk));
+      else
+        tmem_st16(tmem + lane_base + C::T_P + c0 / 2, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_PF);
+      FA_TRACE_EV(12, it);
       // dS^T = P^T * (dP^T - D)
       if (!(ok = W.wait_warp(BAR_DPF, it & 1, 53))) break;
+      FA_TRACE_EV(13, it);
       tc_fence_after();
-      tmem_ld32(tmem + lane_base + C::T_DP, st[0]);
-      tmem_ld32(tmem + lane_base + C::T_DP + 32, st[1]);
-      tmem_wait_ld(st[0]);
-      tmem_wait_ld(st[1]);
+#pragma unroll
+      for (int q = 0; q < NC / 32; ++q) tmem_ld32(tmem + lane_base + C::T_DP + c0 + 32 * q, st[q]);
+#pragma unroll
+      for (int q = 0; q < NC / 32; ++q) tmem_wait_ld(st[q]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_DPFREE);
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
+      for (int c4 = 0; c4 < NC / 4; ++c4) {
         const float4 d4 = reinterpret_cast<const float4*>(Ds)[c4];
         const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
@@ -474,26 +466,32 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       // dS^T columns and the dS smem tile are free once dK(it-1) and dQ(it-1) have read them
       if (it > 0 && !(ok = W.wait_warp(BAR_DQF, (it - 1) & 1, 54))) break;
       tc_fence_after();
-      tmem_st32(tmem + lane_base + C::T_DS, pk);
+      if (NC == 64)
+        tmem_st32(tmem + lane_base + C::T_DS, *reinterpret_cast<uint32_t(*)[32]>(pk));
+      else
+        tmem_st16(tmem + lane_base + C::T_DS + c0 / 2, pk);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < NC / 8; ++c) {
+        const int chunk = c0 / 8 + c;  // 16-byte chunk = 8 queries of this key's row
         const uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(ds_row + ((c ^ (r & 7)) << 4)) = v;
+        *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (r & 7)) << 4)) = v;
       }
       fence_async_smem();
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_DSF);
+      FA_TRACE_EV(14, it);
     }
     if (ok) {
-      // ---- epilogue: dV, dK (x scale) -> bf16 -> global
+      // ---- epilogue: dV, dK (x scale) -> bf16 -> global (split: warpgroup 0 dV, 1 dK)
       ok = W.wait_warp(BAR_DQF, (nit - 1) & 1, 55);
       if (ok) {
         tc_fence_after();
         const size_t base = (size_t(head) * p.N + key) * D + slice * C::DO;
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
+          if (C::SPLIT && which != h) continue;
           const uint32_t col = which == 0 ? C::T_DV : C::T_DK;
           const float mul = which == 0 ? 1.f : p.scale;
           __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + base;
@@ -517,7 +515,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       }
     }
     tc_fence_before();
-  } else if (warp < 8) {
+  } else if (warp < C::DQ_WARP0 + 4) {
     // ---------------------------------------------------------------- dQ drain warpgroup
     // dQ^T (d on TMEM lanes, 64 queries on columns) -> x scale -> shared staging slots laid out
     // [64 queries][64 d] fp32 -> TMA bulk reduce-add into the fp32 accumulator (rows past N are

@@ -135,7 +135,7 @@ int check_common(int B, int H, int N, int d, float scale) {
   if (bh > (1ll << 30) || (long long)N > (1ll << 30))
     return fail(FA_ERR_INVALID_ARG, "B*H or N too large");
   const long long blocks = bh * ((N + 127) / 128);
-  if (blocks > 0x7fffffffll) return fail(FA_ERR_INVALID_ARG, "problem too large for one grid");
+  if (blocks > 0x3fffffffll) return fail(FA_ERR_INVALID_ARG, "problem too large for one grid");
   return FA_OK;
 }
 
@@ -162,6 +162,20 @@ int set_smem(K kernel, int bytes) {
   return FA_OK;
 }
 
+#ifndef FA_FWD_PERSISTENT
+#define FA_FWD_PERSISTENT 1
+#endif
+
+int sm_count() {
+  static thread_local int dev_cached = -1, n = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev != dev_cached) {
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    dev_cached = dev;
+  }
+  return n;
+}
+
 template <int D, bool CAUSAL, int NQT>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                fattn::FwdParams p, int BH, cudaStream_t st) {
@@ -184,7 +198,11 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
                                       "register split");
   }
   p.nqb = (p.N + NQT * C::BM - 1) / (NQT * C::BM);
-  dim3 grid(unsigned(BH) * unsigned(p.nqb));
+  p.BH = BH;
+  p.units = BH * p.nqb;
+  // persistent: one CTA per SM (at most one unit each when there are fewer units than SMs)
+  const int G = FA_FWD_PERSISTENT ? (p.units < sm_count() ? p.units : sm_count()) : p.units;
+  dim3 grid(static_cast<unsigned>(G));
   TimedLaunch tl(FA_KERNEL_FWD, st);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, p);
   cudaError_t e = cudaGetLastError();
@@ -193,16 +211,6 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
-int sm_count() {
-  static thread_local int dev_cached = -1, n = 148;
-  int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess && dev != dev_cached) {
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    dev_cached = dev;
-  }
-  return n;
-}
 
 template <int D, bool CAUSAL>
 int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, cudaStream_t st) {

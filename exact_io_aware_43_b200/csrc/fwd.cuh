@@ -1,9 +1,9 @@
 // fwd.cuh -- fused attention forward for sm_100a.
 //
-// One CTA owns NQT query tiles of 128 rows of one (batch, head) and streams every K_j, V_j tile
-// of 128 keys through a shared-memory ring (chipfoundryservices.com glossary "Flash Attention",
-// "Tiling Algorithm" steps 1-2; robocikowo.com "Flash Attention": a Q block is loaded once, then
-// the loop runs over the K, V blocks).  Per KV tile and query tile:
+// A work unit is NQT query tiles of 128 rows of one (batch, head).  For each unit the CTA streams
+// every K_j, V_j tile of 128 keys through a shared-memory ring (chipfoundryservices.com glossary
+// "Flash Attention", "Tiling Algorithm" steps 1-2; robocikowo.com "Flash Attention": a Q block
+// is loaded once, then the loop runs over the K, V blocks).  Per KV tile and query tile:
 //   S   = Q_t K_j^T                  tcgen05.mma, bf16 x bf16 -> fp32 in tensor memory (step 3)
 //   m   = max(m, rowmax(S*s))        one softmax thread owns one row (one TMEM lane)   (step 4)
 //   P~  = exp2(S*s*log2e - m)        rounded to bf16 and written back into tensor memory
@@ -13,51 +13,38 @@
 // The score tile lives only in tensor memory: the N x N matrix never reaches HBM
 // (systems-analysis.info "FlashAttention (PL)", "Scalanie operacji w jedno jadro CUDA").
 //
-// Warp roles: warps [0, 4*NQT) are the softmax warpgroups (warpgroup t owns query tile t),
-// warp 4*NQT issues TMA loads, warp 4*NQT+1 allocates tensor memory and issues the MMAs.
-// With NQT = 2 the two query tiles ping-pong: the tensor core works on one tile while the
-// softmax warpgroup of the other computes its exponentials.
+// The kernel is persistent: CTA c takes units c, 2G-1-c, 2G+c, ... (a zig-zag over rounds of G =
+// gridDim.x units, with the units ordered heaviest first when causal), keeping its tensor memory
+// and barriers across units.  Q of the next unit is loaded as soon as the current unit's last S
+// MMA has been issued, so its latency hides behind the last PV and the epilogue.  With a grid of
+// one CTA per unit the same code runs one unit per CTA.
+//
+// Warp roles: warps [0, 4*NQT) are the softmax warpgroups (warpgroup t owns query tile t); the
+// next warpgroup holds the TMA producer warp and the MMA-issuing warp (which also allocates
+// tensor memory).  With NQT = 2 the two query tiles ping-pong: the tensor core works on one tile
+// while the softmax warpgroup of the other computes its exponentials.
 #pragma once
 
 #include "sm100.cuh"
 
-// Tuning knobs (compile time).  One pair of exponentials in FA_FWD_POLY_EVERY goes through the
-// FMA-pipe polynomial instead of MUFU (0: none); FA_FWD_POLY_CLAMPED picks the cheaper form
-// (masked scores are clamped to -126 first, giving ~2^-126 instead of 0 -- far below the bf16
-// resolution of P); FA_FWD_MAX3 uses the three-input max for the row maximum.
+// Tuning knobs (compile time), each chosen by measurement on the long-context workload.
+// FA_FWD_POLY_EVERY: one pair of exponentials in N goes through the FMA-pipe polynomial instead of
+// MUFU (0: none).  FA_FWD_RSUM: how O's normaliser is formed -- 0: the fp32 sum (also used for
+// L); 1: sum of the bf16-rounded weights via integer unpack; 2: the same sum with mixed
+// bf16 + fp32 adds.  FA_FWD_RESCALE: the reference max moves (and O is rescaled) only when a row's
+// max grows by more than this many log2 units (0: on every increase).  FA_FWD_MAX3: three-input
+// max for the row maximum.
 #ifndef FA_FWD_POLY_EVERY
 #define FA_FWD_POLY_EVERY 0
 #endif
-// FA_FWD_RSUM: how O's normaliser is formed.  0: the fp32 sum (also used for L); 1: sum of the
-// bf16-rounded weights via integer unpack; 2: the same sum with mixed bf16+fp32 adds.
 #ifndef FA_FWD_RSUM
 #define FA_FWD_RSUM 2
 #endif
-// FA_FWD_RESCALE: the reference max moves (and O is rescaled) only when a row's max grows by more
-// than this many log2 units; 0 rescales on every increase.
 #ifndef FA_FWD_RESCALE
 #define FA_FWD_RESCALE 8.0f
 #endif
-#ifndef FA_FWD_POLY_CLAMPED
-#define FA_FWD_POLY_CLAMPED 0
-#endif
 #ifndef FA_FWD_MAX3
 #define FA_FWD_MAX3 0
-#endif
-// FA_FWD_MMA_SPLIT: 1 gives each query tile its own MMA-issuing warp (no head-of-line blocking
-// between the tiles); 0 issues both tiles' MMAs from one thread in a fixed interleaved order.
-#ifndef FA_FWD_MMA_SPLIT
-#define FA_FWD_MMA_SPLIT 0
-#endif
-// FA_FWD_TOKEN: the two softmax warpgroups take turns on the exponentials (0, 1, 0, 1, ...),
-// passing a token through an mbarrier.
-#ifndef FA_FWD_TOKEN
-#define FA_FWD_TOKEN 0
-#endif
-// FA_FWD_EAGER_PV: after PV_0(j) the single issuer probes (without blocking) whether P_1(j) is
-// already written and, if so, queues PV_1(j) before it waits for PV_0(j) to finish.
-#ifndef FA_FWD_EAGER_PV
-#define FA_FWD_EAGER_PV 0
 #endif
 
 namespace fattn {
@@ -66,7 +53,9 @@ struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
   int N;            // sequence length (queries = keys)
+  int BH;           // batch * heads
   int nqb;          // query blocks (of NQT*128 rows) per head
+  int units;        // BH * nqb
   float scale_log2; // scale * log2(e)
   uint64_t limit_ns;
 };
@@ -84,11 +73,11 @@ struct FwdCfg {
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
   static constexpr int THREADS = (SOFTMAX_WARPS + 4) * 32;
   // Register split with two softmax warpgroups (384 threads launched at 168 registers each):
-  // control warpgroup 40, softmax warpgroups 232; 40*128 + 232*256 = 384*168.
+  // control warpgroup 104, softmax warpgroups 200; 104*128 + 200*256 <= 384*168.
   static constexpr bool REALLOC = NQT == 2;
   static constexpr int LAUNCH_REGS = 168;
-  static constexpr int CTRL_REGS = 40;
-  static constexpr int SOFTMAX_REGS = 232;
+  static constexpr int CTRL_REGS = 104;
+  static constexpr int SOFTMAX_REGS = 200;
   static_assert(!REALLOC || CTRL_REGS * 128 + SOFTMAX_REGS * 256 <= LAUNCH_REGS * THREADS,
                 "register split exceeds the launch allocation");
   static constexpr int TMEM_S = 0;               // S_t at column t*BN (P_t aliases its first BN/2)
@@ -100,13 +89,43 @@ struct FwdCfg {
   static constexpr int OFF_K = OFF_Q + NQT * QTILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KVTILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * KVTILE_BYTES;
-  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT], p_full[NQT],
-  //           o_done[NQT], drain
-  static constexpr int NBAR = 1 + 4 * STAGES + 5 * NQT;
+  // barriers: q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT],
+  //           p_full[NQT], o_done[NQT], o_free[NQT], drain
+  static constexpr int NBAR = 2 + 4 * STAGES + 4 * NQT + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem address + abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);   // Q, K both K-major
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);   // P (tmem), V MN-major
+};
+
+// The k-th unit of CTA c among G CTAs (zig-zag over rounds of G units), or -1 when none is left.
+__device__ __forceinline__ int fwd_unit_of(int k, int c, int G, int units) {
+  const int u = k * G + ((k & 1) ? (G - 1 - c) : c);
+  return u < units ? u : -1;
+}
+
+// Unit u -> (head, first query row, KV tiles per query tile).  Units are numbered query block
+// major, heaviest (latest) query blocks first when causal, heads inner.
+template <int NQT, bool CAUSAL>
+struct FwdUnit {
+  int head, q0, J;
+  int nkv[NQT];
+  __device__ __forceinline__ FwdUnit(int u, const FwdParams& p) {
+    const int qi = u / p.BH;
+    head = u - qi * p.BH;
+    const int qb = CAUSAL ? (p.nqb - 1 - qi) : qi;
+    q0 = qb * NQT * 128;
+    const int n_kv_total = (p.N + 127) / 128;
+    J = 0;
+#pragma unroll
+    for (int t = 0; t < NQT; ++t) {
+      const int r0 = q0 + t * 128;
+      int n = 0;
+      if (r0 < p.N) n = CAUSAL ? min(n_kv_total, (r0 + 127) / 128 + 1) : n_kv_total;
+      nkv[t] = n;
+      J = max(J, n);
+    }
+  }
 };
 
 template <int D, bool CAUSAL, int NQT>
@@ -114,66 +133,49 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D, NQT>;
+  using Unit = FwdUnit<NQT, CAUSAL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const int cta = blockIdx.x;
   FA_TRACE_DECL;
-
-  // ---- work unit: (head, query block), heaviest query blocks first when causal
-  const int head = blockIdx.x / p.nqb;
-  const int qb_lin = blockIdx.x % p.nqb;
-  const int qb = CAUSAL ? (p.nqb - 1 - qb_lin) : qb_lin;
-  const int q0 = qb * NQT * C::BM;
-  const int n_kv_total = (p.N + C::BN - 1) / C::BN;
-  int nkv[NQT];
-  int J = 0;
-#pragma unroll
-  for (int t = 0; t < NQT; ++t) {
-    const int r0 = q0 + t * C::BM;
-    int n = 0;
-    if (r0 < p.N) n = CAUSAL ? min(n_kv_total, (r0 + C::BM - 1) / C::BN + 1) : n_kv_total;
-    nkv[t] = n;
-    J = max(J, n);
-  }
 
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
   const uint32_t BAR_Q = bar(0);
-  auto BAR_KF = [&](int s) { return bar(1 + s); };
-  auto BAR_KE = [&](int s) { return bar(1 + C::STAGES + s); };
-  auto BAR_VF = [&](int s) { return bar(1 + 2 * C::STAGES + s); };
-  auto BAR_VE = [&](int s) { return bar(1 + 3 * C::STAGES + s); };
-  auto BAR_SF = [&](int t) { return bar(1 + 4 * C::STAGES + t); };
-  auto BAR_PF = [&](int t) { return bar(1 + 4 * C::STAGES + NQT + t); };
-  auto BAR_OD = [&](int t) { return bar(1 + 4 * C::STAGES + 2 * NQT + t); };
-  auto BAR_DRAIN = [&](int t) { return bar(1 + 4 * C::STAGES + 3 * NQT + t); };
-  auto BAR_XU = [&](int t) { return bar(1 + 4 * C::STAGES + 4 * NQT + t); };
+  const uint32_t BAR_QE = bar(1);
+  auto BAR_KF = [&](int s) { return bar(2 + s); };
+  auto BAR_KE = [&](int s) { return bar(2 + C::STAGES + s); };
+  auto BAR_VF = [&](int s) { return bar(2 + 2 * C::STAGES + s); };
+  auto BAR_VE = [&](int s) { return bar(2 + 3 * C::STAGES + s); };
+  auto BAR_SF = [&](int t) { return bar(2 + 4 * C::STAGES + t); };
+  auto BAR_PF = [&](int t) { return bar(2 + 4 * C::STAGES + NQT + t); };
+  auto BAR_OD = [&](int t) { return bar(2 + 4 * C::STAGES + 2 * NQT + t); };
+  auto BAR_OF = [&](int t) { return bar(2 + 4 * C::STAGES + 3 * NQT + t); };
+  const uint32_t BAR_DRAIN = bar(C::NBAR - 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   const Waiter W{abort_flag, p.limit_ns};
 
-  int n_active = 0;
-#pragma unroll
-  for (int t = 0; t < NQT; ++t) n_active += (nkv[t] > 0);
-  // with one MMA warp per tile every active tile's warp releases each K/V stage
-  const int kv_release = FA_FWD_MMA_SPLIT ? n_active : 1;
   if (threadIdx.x == 0) {
     mbar_init(BAR_Q, 1);
+    mbar_init(BAR_QE, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(BAR_KF(s), 1);
-      mbar_init(BAR_KE(s), kv_release);
+      mbar_init(BAR_KE(s), 1);
       mbar_init(BAR_VF(s), 1);
-      mbar_init(BAR_VE(s), kv_release);
+      mbar_init(BAR_VE(s), 1);
     }
     for (int t = 0; t < NQT; ++t) {
       mbar_init(BAR_SF(t), 1);
       mbar_init(BAR_PF(t), 4);
       mbar_init(BAR_OD(t), 1);
+      mbar_init(BAR_OF(t), 4);
     }
-    for (int t = 0; t < NQT; ++t) mbar_init(BAR_DRAIN(t), 1);
-    for (int t = 0; t < NQT; ++t) mbar_init(BAR_XU(t), 4);
+    mbar_init(BAR_DRAIN, 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -186,357 +188,332 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   FA_TRACE_EV(30, 0);
+
   if (warp >= C::SOFTMAX_WARPS) {
-   // ================================================================ control warpgroup
-   if constexpr (C::REALLOC) regs_dec<C::CTRL_REGS>();
-   if (warp == C::PRODUCER_WARP) {
-    // ---------------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      int q_tiles = 0;
-      for (int t = 0; t < NQT; ++t) q_tiles += (nkv[t] > 0);
-      mbar_arrive_expect_tx(BAR_Q, q_tiles * C::QTILE_BYTES);
-      for (int t = 0; t < NQT; ++t) {
-        if (nkv[t] == 0) continue;
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(sbase + C::OFF_Q + t * C::QTILE_BYTES + kb * (C::BM * 128), &tmQ, BAR_Q,
-                      kb * 64, q0 + t * C::BM, head);
-      }
-      int j = 0;
-      for (; j < J; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = (j / C::STAGES) & 1;
-        if (!W.wait(BAR_KE(s), ph ^ 1, 1)) break;
-        FA_TRACE_EV(20, j);
-        mbar_arrive_expect_tx(BAR_KF(s), C::KVTILE_BYTES);
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(sbase + C::OFF_K + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmK,
-                      BAR_KF(s), kb * 64, j * C::BN, head);
-        if (!W.wait(BAR_VE(s), ph ^ 1, 2)) {
-          ++j;  // the K load of tile j is in flight
-          break;
-        }
-        FA_TRACE_EV(21, j);
-        mbar_arrive_expect_tx(BAR_VF(s), C::KVTILE_BYTES);
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(sbase + C::OFF_V + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmV,
-                      BAR_VF(s), kb * 64, j * C::BN, head);
-      }
-      if (W.aborted()) {
-        // drain: wait (bounded) for every load already issued before the CTA exits
-        W.drain(BAR_Q, 0);
-        for (int jj = max(0, j - C::STAGES); jj < j; ++jj) {
-          W.drain(BAR_KF(jj % C::STAGES), (jj / C::STAGES) & 1);
-          W.drain(BAR_VF(jj % C::STAGES), (jj / C::STAGES) & 1);
-        }
-      }
-    }
-  } else if (FA_FWD_MMA_SPLIT && warp >= C::MMA_WARP && warp < C::MMA_WARP + NQT) {
-    // ---------------------------------------------------------------- MMA issuer of tile t
-    // Each query tile has its own issuing warp, so one tile's wait never delays the other's
-    // MMAs.  Per KV tile j: PV_t(j) once softmax t has written P_t(j), then S_t(j+1), which
-    // overwrites the tensor memory holding P_t(j) and therefore waits for PV_t(j) to complete.
-    const int t = warp - C::MMA_WARP;
-    const int n = nkv[t];
-    if (lane == 0 && n > 0) {
-      const uint32_t q_addr = sbase + C::OFF_Q + t * C::QTILE_BYTES;
-      auto issue_s = [&](uint32_t k_addr) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ss(tmem + C::TMEM_S + t * C::BN, sdesc_sw128(q_addr + koff, 16, 1024),
-                 sdesc_sw128(k_addr + koff, 16, 1024), C::IDESC_S, kk > 0);
-        }
-        tc_commit(BAR_SF(t));
-      };
-      bool ok = W.wait(BAR_Q, 0, 10) && W.wait(BAR_KF(0), 0, 11);
-      if (ok) {
-        tc_fence_after();
-        issue_s(sbase + C::OFF_K);
-        tc_commit(BAR_KE(0));
-      }
-      for (int j = 0; ok && j < n; ++j) {
-        const int s = j % C::STAGES;
-        const int s1 = (j + 1) % C::STAGES;
-        const uint32_t v_addr = sbase + C::OFF_V + s * C::KVTILE_BYTES;
-        if (!(ok = W.wait(BAR_VF(s), (j / C::STAGES) & 1, 13))) break;
-        FA_TRACE_EV(1 + 16 * t, j);
-        if (!(ok = W.wait(BAR_PF(t), j & 1, 14))) break;
-        FA_TRACE_EV(2 + 16 * t, j);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk)
-          mma_ts(tmem + C::TMEM_O + t * D, tmem + C::TMEM_S + t * C::BN + kk * 8,
-                 sdesc_sw128(v_addr + kk * 2048, C::BN * 128, 1024), C::IDESC_PV,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(BAR_OD(t));
-        tc_commit(BAR_VE(s));
-        if (j + 1 < n) {
-          if (!(ok = W.wait(BAR_KF(s1), ((j + 1) / C::STAGES) & 1, 11))) break;
-          if (!(ok = W.wait(BAR_OD(t), j & 1, 12))) break;  // P_t(j) consumed
-          FA_TRACE_EV(3 + 16 * t, j);
-          tc_fence_after();
-          issue_s(sbase + C::OFF_K + s1 * C::KVTILE_BYTES);
-          tc_commit(BAR_KE(s1));
-        }
-      }
-      tc_commit(BAR_DRAIN(t));
-      W.drain(BAR_DRAIN(t), 0);
-    }
-  } else if (!FA_FWD_MMA_SPLIT && warp == C::MMA_WARP) {
-    // ---------------------------------------------------------------- MMA issuer
-    // Order per KV tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  S_t(j+1) overwrites the tensor
-    // memory that holds P_t(j), so it waits for PV_t(j) to complete; issuing it right behind
-    // PV_t(j) lets softmax t start on tile j+1 while the other query tile's PV runs.
-    if (lane == 0) {
-      auto issue_s = [&](int t, uint32_t k_addr) {
-        const uint32_t q_addr = sbase + C::OFF_Q + t * C::QTILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ss(tmem + C::TMEM_S + t * C::BN, sdesc_sw128(q_addr + koff, 16, 1024),
-                 sdesc_sw128(k_addr + koff, 16, 1024), C::IDESC_S, kk > 0);
-        }
-        tc_commit(BAR_SF(t));
-      };
-      bool ok = W.wait(BAR_Q, 0, 10) && W.wait(BAR_KF(0), 0, 11);
-      if (ok) {
-        tc_fence_after();
-        for (int t = 0; t < NQT; ++t)
-          if (nkv[t] > 0) issue_s(t, sbase + C::OFF_K);
-        tc_commit(BAR_KE(0));
-      }
-      for (int j = 0; ok && j < J; ++j) {
-        const int s = j % C::STAGES;
-        const int s1 = (j + 1) % C::STAGES;
-        const uint32_t v_addr = sbase + C::OFF_V + s * C::KVTILE_BYTES;
-        const uint32_t k1_addr = sbase + C::OFF_K + s1 * C::KVTILE_BYTES;
-        if (!(ok = W.wait(BAR_VF(s), (j / C::STAGES) & 1, 13))) break;
-        bool k_ready = false;
-        bool pv_issued[NQT];
-#pragma unroll
-        for (int t = 0; t < NQT; ++t) pv_issued[t] = false;
-        auto issue_pv = [&](int t) {
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk) {
-            // P~ is packed bf16: 16 keys = 8 columns; V rows (keys) are 128 B apart, so a
-            // 16-key slice is 2048 B further on; 64-wide d blocks are BN*128 B apart.
-            mma_ts(tmem + C::TMEM_O + t * D, tmem + C::TMEM_S + t * C::BN + kk * 8,
-                   sdesc_sw128(v_addr + kk * 2048, C::BN * 128, 1024), C::IDESC_PV,
-                   (j > 0 || kk > 0) ? 1u : 0u);
+    // ================================================================ control warpgroup
+    if constexpr (C::REALLOC) regs_dec<C::CTRL_REGS>();
+    if (warp == C::PRODUCER_WARP) {
+      // -------------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        int kv_it = 0;   // KV tiles loaded so far (ring position)
+        int k = 0;
+        bool ok = true;
+        for (;; ++k) {
+          const int u = fwd_unit_of(k, cta, G, p.units);
+          if (u < 0) break;
+          const Unit un(u, p);
+          // Q of this unit replaces the previous unit's once its last S MMA has completed
+          if (k > 0 && !(ok = W.wait(BAR_QE, (k - 1) & 1, 3))) break;
+          int q_tiles = 0;
+          for (int t = 0; t < NQT; ++t) q_tiles += (un.nkv[t] > 0);
+          mbar_arrive_expect_tx(BAR_Q, q_tiles * C::QTILE_BYTES);
+          for (int t = 0; t < NQT; ++t) {
+            if (un.nkv[t] == 0) continue;
+            for (int kb = 0; kb < C::KB; ++kb)
+              tma_load_3d(sbase + C::OFF_Q + t * C::QTILE_BYTES + kb * (C::BM * 128), &tmQ, BAR_Q,
+                          kb * 64, un.q0 + t * C::BM, un.head);
           }
-          tc_commit(BAR_OD(t));
-          pv_issued[t] = true;
+          for (int j = 0; j < un.J; ++j) {
+            const int g = kv_it + j;
+            const int s = g % C::STAGES;
+            const uint32_t ph = (g / C::STAGES) & 1;
+            if (!(ok = W.wait(BAR_KE(s), ph ^ 1, 1))) break;
+            FA_TRACE_EV(20, j);
+            mbar_arrive_expect_tx(BAR_KF(s), C::KVTILE_BYTES);
+            for (int kb = 0; kb < C::KB; ++kb)
+              tma_load_3d(sbase + C::OFF_K + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmK,
+                          BAR_KF(s), kb * 64, j * C::BN, un.head);
+            if (!(ok = W.wait(BAR_VE(s), ph ^ 1, 2))) break;
+            FA_TRACE_EV(21, j);
+            mbar_arrive_expect_tx(BAR_VF(s), C::KVTILE_BYTES);
+            for (int kb = 0; kb < C::KB; ++kb)
+              tma_load_3d(sbase + C::OFF_V + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmV,
+                          BAR_VF(s), kb * 64, j * C::BN, un.head);
+          }
+          if (!ok) break;
+          kv_it += un.J;
+        }
+        if (!ok) {
+          // drain (bounded): every load issued so far lands before the CTA exits
+          W.drain(BAR_Q, k & 1);
+          for (int s = 0; s < C::STAGES; ++s) {
+            W.drain(BAR_KF(s), 0);
+            W.drain(BAR_KF(s), 1);
+            W.drain(BAR_VF(s), 0);
+            W.drain(BAR_VF(s), 1);
+          }
+        }
+      }
+    } else if (warp == C::MMA_WARP) {
+      // -------------------------------------------------------------- MMA issuer
+      // Order per KV tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  S_t(j+1) overwrites the
+      // tensor memory that holds P_t(j), so it waits for PV_t(j) to complete; issuing it right
+      // behind PV_t(j) lets softmax t start on tile j+1 while the other query tile's PV runs.
+      if (lane == 0) {
+        auto issue_s = [&](int t, uint32_t k_addr) {
+          const uint32_t q_addr = sbase + C::OFF_Q + t * C::QTILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_ss(tmem + C::TMEM_S + t * C::BN, sdesc_sw128(q_addr + koff, 16, 1024),
+                   sdesc_sw128(k_addr + koff, 16, 1024), C::IDESC_S, kk > 0);
+          }
+          tc_commit(BAR_SF(t));
         };
-        for (int t = 0; t < NQT && ok; ++t) {
-          if (j >= nkv[t]) continue;
-          if (!pv_issued[t]) {
-            FA_TRACE_EV(1 + 16 * t, j);
-            if (!(ok = W.wait(BAR_PF(t), j & 1, 14))) break;
-            FA_TRACE_EV(2 + 16 * t, j);
-            issue_pv(t);
-          }
-          if (FA_FWD_EAGER_PV && NQT == 2 && t == 0 && j < nkv[1] &&
-              mbar_test_wait(BAR_PF(1), j & 1))
-            issue_pv(1);
-          if (j + 1 < nkv[t]) {
-            if (!k_ready && !(ok = W.wait(BAR_KF(s1), ((j + 1) / C::STAGES) & 1, 11))) break;
-            k_ready = true;
-            if (!(ok = W.wait(BAR_OD(t), j & 1, 12))) break;  // P_t(j) consumed
-            FA_TRACE_EV(3 + 16 * t, j);
+        int kv_it = 0;
+        int tit[NQT], tun[NQT];  // per tile: KV iterations and units processed so far
+#pragma unroll
+        for (int t = 0; t < NQT; ++t) tit[t] = tun[t] = 0;
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+          const int u = fwd_unit_of(k, cta, G, p.units);
+          if (u < 0) break;
+          const Unit un(u, p);
+          const int J = un.J;
+          const int s0 = kv_it % C::STAGES;
+          if (!(ok = W.wait(BAR_Q, k & 1, 10))) break;
+          if (!(ok = W.wait(BAR_KF(s0), (kv_it / C::STAGES) & 1, 11))) break;
+          for (int t = 0; t < NQT && ok; ++t) {
+            if (un.nkv[t] == 0) continue;
+            // S_t's columns hold P_t of the previous unit's last tile until its PV completed
+            if (tit[t] > 0 && !(ok = W.wait(BAR_OD(t), (tit[t] - 1) & 1, 12))) break;
             tc_fence_after();
-            issue_s(t, k1_addr);
+            issue_s(t, sbase + C::OFF_K + s0 * C::KVTILE_BYTES);
           }
+          if (!ok) break;
+          tc_commit(BAR_KE(s0));
+          if (J == 1) tc_commit(BAR_QE);  // every S of this unit is issued: Q may be replaced
+          for (int j = 0; ok && j < J; ++j) {
+            const int g = kv_it + j;
+            const int s = g % C::STAGES;
+            const int s1 = (g + 1) % C::STAGES;
+            const uint32_t v_addr = sbase + C::OFF_V + s * C::KVTILE_BYTES;
+            const uint32_t k1_addr = sbase + C::OFF_K + s1 * C::KVTILE_BYTES;
+            if (!(ok = W.wait(BAR_VF(s), (g / C::STAGES) & 1, 13))) break;
+            bool k_ready = false;
+            for (int t = 0; t < NQT && ok; ++t) {
+              if (j >= un.nkv[t]) continue;
+              FA_TRACE_EV(1 + 16 * t, j);
+              if (!(ok = W.wait(BAR_PF(t), tit[t] & 1, 14))) break;
+              // the first PV of a unit overwrites O_t: the previous epilogue must have read it
+              if (j == 0 && tun[t] > 0 && !(ok = W.wait(BAR_OF(t), (tun[t] - 1) & 1, 15))) break;
+              FA_TRACE_EV(2 + 16 * t, j);
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < C::BN / 16; ++kk) {
+                // P~ is packed bf16: 16 keys = 8 columns; V rows (keys) are 128 B apart, so a
+                // 16-key slice is 2048 B further on; 64-wide d blocks are BN*128 B apart.
+                mma_ts(tmem + C::TMEM_O + t * D, tmem + C::TMEM_S + t * C::BN + kk * 8,
+                       sdesc_sw128(v_addr + kk * 2048, C::BN * 128, 1024), C::IDESC_PV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+              }
+              tc_commit(BAR_OD(t));
+              if (j + 1 < un.nkv[t]) {
+                if (!k_ready &&
+                    !(ok = W.wait(BAR_KF(s1), ((g + 1) / C::STAGES) & 1, 16)))
+                  break;
+                k_ready = true;
+                if (!(ok = W.wait(BAR_OD(t), tit[t] & 1, 17))) break;  // P_t(j) consumed
+                FA_TRACE_EV(3 + 16 * t, j);
+                tc_fence_after();
+                issue_s(t, k1_addr);
+              }
+              ++tit[t];
+            }
+            if (!ok) break;
+            tc_commit(BAR_VE(s));
+            if (k_ready) tc_commit(BAR_KE(s1));
+            // S MMAs of the last KV tile are issued during tile J-2: Q may then be replaced
+            if (j == J - 2) tc_commit(BAR_QE);
+          }
+          if (!ok) break;
+#pragma unroll
+          for (int t = 0; t < NQT; ++t) tun[t] += (un.nkv[t] > 0);
+          kv_it += J;
         }
-        if (!ok) break;
-        tc_commit(BAR_VE(s));
-        if (k_ready) tc_commit(BAR_KE(s1));
+        // every MMA issued above has completed before the tensor memory is released
+        tc_commit(BAR_DRAIN);
+        W.drain(BAR_DRAIN, 0);
       }
-      // every MMA issued above has completed before the tensor memory is released
-      tc_commit(BAR_DRAIN(0));
-      W.drain(BAR_DRAIN(0), 0);
     }
-   }
   } else {
     // ---------------------------------------------------------------- softmax warpgroups
     if constexpr (C::REALLOC) regs_inc<C::SOFTMAX_REGS>();
     const int t = warp >> 2;                  // query tile of this warpgroup
     const int r = threadIdx.x & 127;          // row within the tile == TMEM lane
-    const int row = q0 + t * C::BM + r;       // query index
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + C::TMEM_S + t * C::BN;
     const uint32_t tO = tmem + lane_base + C::TMEM_O + t * D;
-    const int n = nkv[t];
     // m: reference max (log2 units of the scaled scores) that the exponentials and l are taken
     // against.  It only moves when a row's max grows by more than kRescale (2^8 in value): the
     // result is the same exact softmax, P~ stays <= 256, and O is rescaled far less often.
     constexpr float kRescale = FA_FWD_RESCALE;
-    float m = -INFINITY;
-    float l = 0.f;   // sum of the fp32 exponentials (for L)
-    float lr = 0.f;  // sum of the bf16-rounded exponentials (divides O)
+    int tit = 0;  // KV iterations of this tile so far (barrier phases continue across units)
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      FA_TRACE_EV(10, j);
-      if (!(ok = W.wait_warp(BAR_SF(t), j & 1, 20))) break;
-      FA_TRACE_EV(11, j);
-      tc_fence_after();
-      uint32_t s[4][32];
+    for (int k = 0; ok; ++k) {
+      const int u = fwd_unit_of(k, cta, G, p.units);
+      if (u < 0) break;
+      const Unit un(u, p);
+      const int n = un.nkv[t];
+      if (n == 0) continue;
+      const int row = un.q0 + t * C::BM + r;  // query index
+      float m = -INFINITY;
+      float l = 0.f;   // sum of the fp32 exponentials (for L)
+      float lr = 0.f;  // sum of the bf16-rounded exponentials (divides O)
+      for (int j = 0; j < n; ++j, ++tit) {
+        FA_TRACE_EV(10, j);
+        if (!(ok = W.wait_warp(BAR_SF(t), tit & 1, 20))) break;
+        FA_TRACE_EV(11, j);
+        tc_fence_after();
+        uint32_t s[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_wait_ld(s[c]);
-      FA_TRACE_EV(15, j);
-      // mask keys past N and, on diagonal tiles, keys after the query (causal)
-      const int key0 = j * C::BN;
-      const int lim = CAUSAL ? min(row, p.N - 1) - key0 : (p.N - 1) - key0;  // last valid col
-      if (lim < C::BN - 1) {
+        for (int c = 0; c < 4; ++c) tmem_wait_ld(s[c]);
+        FA_TRACE_EV(15, j);
+        // mask keys past N and, on diagonal tiles, keys after the query (causal)
+        const int key0 = j * C::BN;
+        const int lim = CAUSAL ? min(row, p.N - 1) - key0 : (p.N - 1) - key0;  // last valid col
+        if (lim < C::BN - 1) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (32 * c + e > lim) s[c][e] = __float_as_uint(-INFINITY);
+        }
+        float mx8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+#if FA_FWD_MAX3
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (32 * c + e > lim) s[c][e] = __float_as_uint(-INFINITY);
-      }
-      float mx8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
-#if FA_FWD_MAX3
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; e += 2)
-          mx8[(e >> 1) & 7] = fmax3(mx8[(e >> 1) & 7], __uint_as_float(s[c][e]),
-                                    __uint_as_float(s[c][e + 1]));
+          for (int e = 0; e < 32; e += 2)
+            mx8[(e >> 1) & 7] = fmax3(mx8[(e >> 1) & 7], __uint_as_float(s[c][e]),
+                                      __uint_as_float(s[c][e + 1]));
 #else
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(s[c][e]));
+          for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(s[c][e]));
 #endif
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      FA_TRACE_EV(16, j);
-      if (FA_FWD_TOKEN && NQT == 2) {
-        const int o = 1 - t;
-        const int jo = t == 0 ? j - 1 : j;  // the other tile's KV tile that goes first
-        if (jo >= 0 && jo < nkv[o] && !(ok = W.wait_warp(BAR_XU(o), jo & 1, 23))) break;
-      }
-      const float m_tile = mx * p.scale_log2;
-      const float m_use = (j == 0 || m_tile > m + kRescale) ? fmaxf(m, m_tile) : m;
-      const float alpha = (j == 0 || m_use == m) ? 1.f : ex2(m - m_use);
-      // exact fp32 sum (for L) and the sum of the bf16-rounded weights the PV MMA uses (for O's
-      // normalisation: numerator and denominator then agree, so a row dominated by one key
-      // reproduces that key's V), both accumulated in paired fp32
-      uint64_t sum_x[2] = {0ull, 0ull}, sum_r[2] = {0ull, 0ull};
-      const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
-      const uint64_t nm2 = f2pack(-m_use, -m_use);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        FA_TRACE_EV(16, j);
+        const float m_tile = mx * p.scale_log2;
+        const float m_use = (j == 0 || m_tile > m + kRescale) ? fmaxf(m, m_tile) : m;
+        const float alpha = (j == 0 || m_use == m) ? 1.f : ex2(m - m_use);
+        // exact fp32 sum (for L) and the sum of the bf16-rounded weights the PV MMA uses (for
+        // O's normalisation: numerator and denominator then agree, so a row dominated by one
+        // key reproduces that key's V), both accumulated in paired fp32
+        uint64_t sum_x[2] = {0ull, 0ull}, sum_r[2] = {0ull, 0ull};
+        const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2pack(-m_use, -m_use);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float x0, x1, p0, p1;
-          f2unpack(ffma2(f2pack(__uint_as_float(s[c][2 * e]), __uint_as_float(s[c][2 * e + 1])),
-                         sc2, nm2),
-                   x0, x1);
-          // one pair in FA_FWD_POLY_EVERY goes through the FMA-pipe polynomial, the rest MUFU
-          if (FA_FWD_POLY_EVERY > 0 && (e % (FA_FWD_POLY_EVERY > 0 ? FA_FWD_POLY_EVERY : 1)) ==
-                                           FA_FWD_POLY_EVERY - 1) {
-            if (FA_FWD_POLY_CLAMPED)
-              ex2_poly2_clamped(fmaxf(x0, -126.f), fmaxf(x1, -126.f), p0, p1);
-            else
+          for (int e = 0; e < 16; ++e) {
+            float x0, x1, p0, p1;
+            f2unpack(ffma2(f2pack(__uint_as_float(s[c][2 * e]), __uint_as_float(s[c][2 * e + 1])),
+                           sc2, nm2),
+                     x0, x1);
+            // one pair in FA_FWD_POLY_EVERY goes through the FMA-pipe polynomial, the rest MUFU
+            if (FA_FWD_POLY_EVERY > 0 &&
+                (e % (FA_FWD_POLY_EVERY > 0 ? FA_FWD_POLY_EVERY : 1)) == FA_FWD_POLY_EVERY - 1) {
               ex2_poly2(x0, x1, p0, p1);
-          } else {
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
-          pk[e] = pack_bf16(p0, p1);
-          sum_x[e & 1] = fadd2(sum_x[e & 1], f2pack(p0, p1));
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            pk[e] = pack_bf16(p0, p1);
+            sum_x[e & 1] = fadd2(sum_x[e & 1], f2pack(p0, p1));
 #if FA_FWD_RSUM == 1
-          sum_r[e & 1] = fadd2(sum_r[e & 1], f2pack(__uint_as_float(pk[e] << 16),
-                                                   __uint_as_float(pk[e] & 0xffff0000u)));
+            sum_r[e & 1] = fadd2(sum_r[e & 1], f2pack(__uint_as_float(pk[e] << 16),
+                                                     __uint_as_float(pk[e] & 0xffff0000u)));
 #elif FA_FWD_RSUM == 2
-          {
-            float r0, r1;
-            f2unpack(sum_r[e & 1], r0, r1);
-            add_bf16pair_f32(pk[e], r0, r1);
-            sum_r[e & 1] = f2pack(r0, r1);
-          }
+            {
+              float r0, r1;
+              f2unpack(sum_r[e & 1], r0, r1);
+              add_bf16pair_f32(pk[e], r0, r1);
+              sum_r[e & 1] = f2pack(r0, r1);
+            }
 #endif
-        }
-        // 32 keys -> 16 packed columns; two chunks share one 32-column store
-        if (c & 1) {
+          }
+          // 32 keys -> 16 packed columns; two chunks share one 32-column store
+          if (c & 1) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) s[c - 1][16 + e] = pk[e];
-        } else {
+            for (int e = 0; e < 16; ++e) s[c - 1][16 + e] = pk[e];
+          } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) s[c][e] = pk[e];
-        }
-      }
-      FA_TRACE_EV(12, j);
-      if (FA_FWD_TOKEN && NQT == 2) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR_XU(t));
-      }
-      // P~ (bf16) over the first 64 columns of S_t
-      tmem_st32(tS + 0, s[0]);
-      tmem_st32(tS + 32, s[2]);
-      {
-        float a0, a1, b0, b1;
-        f2unpack(fadd2(sum_x[0], sum_x[1]), a0, a1);
-        f2unpack(fadd2(sum_r[0], sum_r[1]), b0, b1);
-        l = l * alpha + (a0 + a1);
-        lr = (FA_FWD_RSUM == 0) ? l : lr * alpha + (b0 + b1);
-      }
-      m = m_use;
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // O_t holds PV_t(j-1) (S_t(j) was issued only after it completed); rescale it
-        if (!(ok = W.wait_warp(BAR_OD(t), (j - 1) & 1, 21))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_wait_ld(o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + 32 * c, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR_PF(t));
-      FA_TRACE_EV(13, j);
-    }
-    if (ok && n > 0) {
-      // ---- epilogue: O / l -> bf16 -> global; L = (m + log2 l) * ln 2
-      ok = W.wait_warp(BAR_OD(t), (n - 1) & 1, 22);
-      if (ok) {
-        tc_fence_after();
-        const float inv_l = 1.f / lr;
-        __nv_bfloat16* orow = p.o + (size_t(head) * p.N + row) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_wait_ld(o);
-          uint4 pk[4];
-          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pw[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l,
-                              __uint_as_float(o[2 * e + 1]) * inv_l);
-          if (row < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = pk[e];
+            for (int e = 0; e < 16; ++e) s[c][e] = pk[e];
           }
         }
-        if (row < p.N) p.lse[size_t(head) * p.N + row] = (m + lg2(l)) * 0.69314718055994531f;
+        FA_TRACE_EV(12, j);
+        // P~ (bf16) over the first 64 columns of S_t
+        tmem_st32(tS + 0, s[0]);
+        tmem_st32(tS + 32, s[2]);
+        {
+          float a0, a1, b0, b1;
+          f2unpack(fadd2(sum_x[0], sum_x[1]), a0, a1);
+          f2unpack(fadd2(sum_r[0], sum_r[1]), b0, b1);
+          l = l * alpha + (a0 + a1);
+          lr = (FA_FWD_RSUM == 0) ? l : lr * alpha + (b0 + b1);
+        }
+        m = m_use;
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          FA_TRACE_EV(14, j);
+          // O_t holds PV_t(j-1) (S_t(j) was issued only after it completed); rescale it
+          if (!(ok = W.wait_warp(BAR_OD(t), (tit - 1) & 1, 21))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_wait_ld(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + 32 * c, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR_PF(t));
+        FA_TRACE_EV(13, j);
       }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16 -> global; L = (m + log2 l) * ln 2.  O_t is released to the
+      // next unit's first PV once its last chunk has been read.
+      if (!(ok = W.wait_warp(BAR_OD(t), (tit - 1) & 1, 22))) break;
+      tc_fence_after();
+      const float inv_l = 1.f / lr;
+      __nv_bfloat16* orow = p.o + (size_t(un.head) * p.N + row) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_wait_ld(o);
+        if (c == D / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR_OF(t));
+        }
+        uint4 pk[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pw[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        if (row < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = pk[e];
+        }
+      }
+      if (row < p.N) p.lse[size_t(un.head) * p.N + row] = (m + lg2(l)) * 0.69314718055994531f;
     }
     tc_fence_before();
   }
