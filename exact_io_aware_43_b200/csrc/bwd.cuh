@@ -38,6 +38,11 @@
 #ifndef FA_BWD_SPLIT
 #define FA_BWD_SPLIT 1
 #endif
+// FA_BWD_ORDER: 1 issues dP^T(i+1) as soon as the dS warps have read dP^T(i), ahead of dK(i) and
+// dQ^T(i) (which wait for dS(i)); 0 issues it after them.
+#ifndef FA_BWD_ORDER
+#define FA_BWD_ORDER 0
+#endif
 
 namespace fattn {
 
@@ -337,6 +342,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           return true;
         };
         if (more && C::STAGES > 1 && !(ok = issue_next_st())) break;
+        const bool early_dp = FA_BWD_ORDER && C::STAGES > 1 && more;
+        if (early_dp) {
+          if (!(ok = W.wait(BAR_DPFREE, it & 1, 47))) break;
+          FA_TRACE_EV(7, it);
+          tc_fence_after();
+          issue_st(C::T_DP, v_addr, sbase + C::OFF_DO + sn * C::Q_BYTES);
+          tc_commit(BAR_DPF);
+        }
         // dK += dS^T Q_i ; dQ_i^T = K_j^T dS^T
         FA_TRACE_EV(4, it);
         if (!(ok = W.wait(BAR_DSF, it & 1, 45))) break;
@@ -352,7 +365,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                  sdesc_sw128(ds_addr + kk * 2048, C::Q_BLK, 1024), C::IDESC_DQ, kk > 0);
         tc_commit(BAR_DQF);
         tc_commit(BAR_QE(s));
-        if (more) {
+        if (more && !early_dp) {
           if (C::STAGES == 1 && !(ok = issue_next_st())) break;
           if (!(ok = W.wait(BAR_DPFREE, it & 1, 47))) break;
           FA_TRACE_EV(7, it);
