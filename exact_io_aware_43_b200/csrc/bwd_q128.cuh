@@ -1,0 +1,551 @@
+// bwd_q128.cuh -- attention backward main kernel for d = 128 with 128-query steps (sm_100a).
+//
+// Same mathematics as fa_bwd_kernel (robocikowo.com "Flash Attention": the backward recomputes
+// P from the saved L; the gradient formulas are those of the definition), with a different
+// tiling: each step takes 128 queries instead of 64, so every one of the five GEMMs of a step is
+// a 128 x 128 x 128 tcgen05.mma group.  At N = 64 the tensor core's operand fetch from shared
+// memory (6 KB per 16-deep instruction) is what limits it; at N = 128 the K_j / V_j operand is
+// read once per 128 queries, which cuts shared-memory bytes per FLOP by a quarter.
+//
+// Tensor memory (512 columns) holds, per step:
+//   R1 [0,128)    S^T = K_j Q_i^T (fp32).  Each query half h (64 columns, one warpgroup) then
+//                 overwrites its own columns with P^T in bf16 at [96h, 96h+32).
+//   R2 [128,256)  dP^T = V_j dO_i^T (fp32); once the dS^T warps have read it, dQ_i^T =
+//                 K_j^T dS^T (fp32, d on lanes, 128 query columns).
+//   [256,384) dV accumulator, [384,512) dK accumulator.
+// dS^T (bf16) goes to a shared tile, from which both dQ^T and dK (dS^T Q_i, both operands in
+// shared memory) read it.  Reuse is ordered by completion barriers, never by issue order:
+// S^T(i+1) is issued once dV(i) has completed, dP^T(i+1) once dQ^T(i) has been read out.
+// (Compile-time alternatives keep dS^T in tensor memory for dK -- dQ^T then waits for dK -- or
+// stage dQ in the dS^T tile's space.)
+//
+// Warp roles (512 threads): warps 0-7 compute P^T and dS^T (warpgroup h owns query columns
+// [64h, 64h+64); thread = key row = TMEM lane), warps 8-11 drain dQ^T (TMEM -> x scale ->
+// shared staging -> TMA bulk reduce-add into the fp32 accumulator),
+// warp 12 issues TMA loads, warp 13 allocates tensor memory and issues the MMAs.
+#pragma once
+
+#include "bwd.cuh"
+
+// FA_BWDQ_EARLY_S: 1 issues S^T(i+1) right after dV(i) completes (before dK(i)); 0 issues it
+// after dK(i), which leaves the tensor core no gap while the MMA thread waits for dV(i).
+#ifndef FA_BWDQ_EARLY_S
+#define FA_BWDQ_EARLY_S 1
+#endif
+// FA_BWDQ_DO_STAGES: dO_i buffers (1 or 2).  FA_BWDQ_SEP_STAGE: 1 gives the dQ staging its own
+// 32 KB instead of the dS^T tile's space (then the dS^T writes need not wait for the reduce to
+// read the staging).  Shared memory holds at most one of the two extra tiles.
+#ifndef FA_BWDQ_DO_STAGES
+#define FA_BWDQ_DO_STAGES 1
+#endif
+#ifndef FA_BWDQ_SEP_STAGE
+#define FA_BWDQ_SEP_STAGE 1
+#endif
+// FA_BWDQ_DK_SS: 1 reads dS^T for dK from the shared tile (both operands in shared memory), so
+// dQ^T may overwrite R2 as soon as dS^T is ready and is issued first; 0 reads dS^T from tensor
+// memory, and dQ^T then waits for dK to complete.
+#ifndef FA_BWDQ_DK_SS
+#define FA_BWDQ_DK_SS 1
+#endif
+// FA_BWDQ_PREFETCH: the producer asks L2 for the Q and dO tiles this many steps ahead of the
+// ones it loads into shared memory (0: no prefetch).
+#ifndef FA_BWDQ_PREFETCH
+#define FA_BWDQ_PREFETCH 0
+#endif
+
+namespace fattn {
+
+struct BwdQ128Cfg {
+  static constexpr int D = 128;
+  static constexpr int BC = 128;          // keys per CTA
+  static constexpr int BR = 128;          // queries per step
+  static constexpr int BLK = 128 * 128;   // one 64-column (128-byte-row) block of a 128-row tile
+  static constexpr int TILE = 2 * BLK;    // a 128 x 128 bf16 tile
+  static constexpr int THREADS = 512;
+  static constexpr int CMP_WARPS = 8;
+  static constexpr int DQ_WARP0 = 8;
+  static constexpr int PRODUCER_WARP = 12;
+  static constexpr int MMA_WARP = 13;
+  // register split over the four warpgroups (launch: 512 threads x 128 registers)
+  static constexpr int LAUNCH_REGS = 128;
+#ifndef FA_BWDQ_CMP_REGS
+#define FA_BWDQ_CMP_REGS 136
+#endif
+#ifndef FA_BWDQ_DQ_REGS
+#define FA_BWDQ_DQ_REGS 144
+#endif
+#ifndef FA_BWDQ_CTRL_REGS
+#define FA_BWDQ_CTRL_REGS 96
+#endif
+  static constexpr int CMP_REGS = FA_BWDQ_CMP_REGS, DQ_REGS = FA_BWDQ_DQ_REGS,
+                       CTRL_REGS = FA_BWDQ_CTRL_REGS;
+  static_assert(2 * 128 * CMP_REGS + 128 * DQ_REGS + 128 * CTRL_REGS <= THREADS * LAUNCH_REGS,
+                "register split exceeds the launch allocation");
+  // tensor memory columns
+  static constexpr int T_S = 0, T_DP = 128, T_DQ = 128, T_DV = 256, T_DK = 384;
+  static constexpr int TMEM_COLS = 512;
+  // shared memory map (offsets from a 1024-aligned base)
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;        // 2 stages
+  static constexpr int DO_STAGES = FA_BWDQ_DO_STAGES;
+  static constexpr bool SEP = FA_BWDQ_SEP_STAGE != 0;
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;            // DO_STAGES x dO_i
+  static constexpr int OFF_DS = OFF_DO + DO_STAGES * TILE;   // dS^T [2 q halves][128 keys][64 q]
+  static constexpr int OFF_STG = SEP ? OFF_DS + TILE : OFF_DS;  // dQ staging: 2 x [64 q][64 d] f32
+  static constexpr int OFF_ROWS = OFF_STG + TILE;            // 2 stages x (L2[128], D[128]) fp32
+  // barriers: kv, q_full[2], q_empty[2], do_full[2], do_empty[2], s_full, p_full, dp_full,
+  //           ds_full, dv_done, dk_done, dq_full, dq_empty, ds_free, drain
+  static constexpr int NBAR = 19;
+  static constexpr int OFF_BAR = OFF_ROWS + 2 * 2 * BR * 4;
+  static constexpr int OFF_MISC = OFF_BAR + 160;
+  static constexpr int SMEM_NEED = OFF_MISC + 16;             // from a 1024-aligned base
+  static constexpr int SMEM_MAX = 227 * 1024;                 // opt-in limit per CTA on sm_100
+  // up to 1 KB of slack for aligning the base; the kernel checks what it actually got
+  static constexpr int SMEM_BYTES = SMEM_NEED + 1024 < SMEM_MAX ? SMEM_NEED + 1024 : SMEM_MAX;
+  static_assert(NBAR * 8 <= 160, "barrier area");
+  static_assert(SMEM_NEED <= SMEM_MAX, "shared memory budget");
+  static_assert(DO_STAGES == 1 || DO_STAGES == 2, "dO stages");
+  // dK reading the dS^T tile after dQ^T's completion is signalled: the staging must not share it
+  static_assert(SEP || !FA_BWDQ_DK_SS, "dK from shared dS^T needs separate dQ staging");
+  static constexpr uint32_t IDESC_ST = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+  static constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, 0, 1);  // dV, dK (A in TMEM)
+  static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, 128, 1, 1);  // dQ^T = K^T dS^T
+};
+
+template <bool CAUSAL>
+__global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
+    fa_bwd_kernel_q128(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmdO,
+                       const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
+  using C = BwdQ128Cfg;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the swizzled tiles need a 1024-byte-aligned base; with the largest layouts there is less
+  // than 1 KB of slack, so a base that cannot be aligned within it is reported, not used
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  if (pad + C::SMEM_NEED > C::SMEM_BYTES) {
+    if (threadIdx.x == 0 && atomicCAS(&g_status[0], 0, 2 /* FA_ERR_UNSUPPORTED */) == 0)
+      g_status[1] = 90;
+    return;
+  }
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  FA_TRACE_DECL;
+
+  // ---- work unit: (head, key block j); query blocks i from j (causal) or 0 to the last
+  const int head = blockIdx.x / p.nkb;
+  const int j = blockIdx.x % p.nkb;
+  const int k0 = j * C::BC;
+  const int nqb = (p.N + C::BR - 1) / C::BR;
+  const int i_start = CAUSAL ? j : 0;
+  const int nit = nqb - i_start;  // >= 1
+
+  auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
+  const uint32_t BAR_KV = bar(0);
+  auto BAR_QF = [&](int s) { return bar(1 + s); };
+  auto BAR_QE = [&](int s) { return bar(3 + s); };
+  auto BAR_DOF = [&](int s) { return bar(5 + s); };
+  auto BAR_DOE = [&](int s) { return bar(7 + s); };
+  const uint32_t BAR_SF = bar(9), BAR_PF = bar(10), BAR_DPF = bar(11), BAR_DSF = bar(12),
+                 BAR_DVD = bar(13), BAR_DKD = bar(14), BAR_DQF = bar(15), BAR_DQE = bar(16),
+                 BAR_DSFREE = bar(17), BAR_DRAIN = bar(18);
+  constexpr int DS_ = C::DO_STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  const Waiter W{abort_flag, p.limit_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR_KV, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR_QF(s), 1);
+      mbar_init(BAR_QE(s), 1);
+      mbar_init(BAR_DOF(s), 1);
+      mbar_init(BAR_DOE(s), 1);
+    }
+    mbar_init(BAR_SF, 1);
+    mbar_init(BAR_PF, C::CMP_WARPS);
+    mbar_init(BAR_DPF, 1);
+    mbar_init(BAR_DSF, C::CMP_WARPS);
+    mbar_init(BAR_DVD, 1);
+    mbar_init(BAR_DKD, 1);
+    mbar_init(BAR_DQF, 1);
+    mbar_init(BAR_DQE, 4);
+    mbar_init(BAR_DSFREE, 1);
+    mbar_init(BAR_DRAIN, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const float* rows_smem = reinterpret_cast<const float*>(smem + C::OFF_ROWS);
+
+  if (warp >= C::PRODUCER_WARP) {
+    // ================================================================ control warpgroup
+    regs_dec<C::CTRL_REGS>();
+    if (warp == C::PRODUCER_WARP && lane == 0) {
+      // -------------------------------------------------------------- TMA producer
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      mbar_arrive_expect_tx(BAR_KV, 2 * C::TILE);
+      for (int kb = 0; kb < 2; ++kb) {
+        tma_load_3d(sbase + C::OFF_K + kb * C::BLK, &tmK, BAR_KV, kb * 64, k0, head);
+        tma_load_3d(sbase + C::OFF_V + kb * C::BLK, &tmV, BAR_KV, kb * 64, k0, head);
+      }
+      int tq = 0, td = 0;  // Q / dO tiles issued
+      for (int t = 0; t < nit; ++t) {
+        const int i = i_start + t;
+        const int s = t & 1;
+        if (FA_BWDQ_PREFETCH > 0) {
+          // tiles t+1 .. t+PREFETCH are in flight to L2 after the first step; one more per step
+          for (int u = (t == 0 ? 1 : FA_BWDQ_PREFETCH); u <= FA_BWDQ_PREFETCH; ++u) {
+            if (t + u >= nit) break;
+            for (int kb = 0; kb < 2; ++kb) {
+              tma_prefetch_3d(&tmQ, kb * 64, (i + u) * C::BR, head);
+              tma_prefetch_3d(&tmdO, kb * 64, (i + u) * C::BR, head);
+            }
+          }
+        }
+        // Q_i, L2_i and D_i into stage s once dK of step t-2 has released it
+        if (!W.wait(BAR_QE(s), ((t >> 1) & 1) ^ 1, 31)) break;
+        mbar_arrive_expect_tx(BAR_QF(s), C::TILE + 2 * C::BR * 4);
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_3d(sbase + C::OFF_Q + s * C::TILE + kb * C::BLK, &tmQ, BAR_QF(s), kb * 64,
+                      i * C::BR, head);
+        const size_t roff = size_t(head) * p.Npad + size_t(i) * C::BR;
+        const uint32_t rdst = sbase + C::OFF_ROWS + s * 2 * C::BR * 4;
+        bulk_load(rdst, p.L2 + roff, C::BR * 4, BAR_QF(s));
+        bulk_load(rdst + C::BR * 4, p.Drow + roff, C::BR * 4, BAR_QF(s));
+        ++tq;
+        FA_TRACE_EV(20, t);
+        // dO_i into its buffer once dP^T and dV of the step that used it last have read it
+        const int sd = t % DS_;
+        if (!W.wait(BAR_DOE(sd), ((t / DS_) & 1) ^ 1, 32)) break;
+        mbar_arrive_expect_tx(BAR_DOF(sd), C::TILE);
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_3d(sbase + C::OFF_DO + sd * C::TILE + kb * C::BLK, &tmdO, BAR_DOF(sd), kb * 64,
+                      i * C::BR, head);
+        ++td;
+      }
+      if (W.aborted()) {
+        // let the copies already issued land before the CTA's shared memory goes away
+        W.drain(BAR_KV, 0);
+        for (int jj = tq > 2 ? tq - 2 : 0; jj < tq; ++jj) W.drain(BAR_QF(jj & 1), (jj >> 1) & 1);
+        for (int jj = td > DS_ ? td - DS_ : 0; jj < td; ++jj)
+          W.drain(BAR_DOF(jj % DS_), (jj / DS_) & 1);
+      }
+    } else if (warp == C::MMA_WARP && lane == 0) {
+      // -------------------------------------------------------------- MMA issuer
+      const uint32_t k_addr = sbase + C::OFF_K, v_addr = sbase + C::OFF_V;
+      const uint32_t ds_addr = sbase + C::OFF_DS;
+      auto q_addr = [&](int s) { return sbase + C::OFF_Q + s * C::TILE; };
+      auto do_addr = [&](int t) { return sbase + C::OFF_DO + (t % DS_) * C::TILE; };
+      // [S^T | dP^T] (128 keys x 128 queries) = A (keys x d) * B (queries x d)^T, both K-major
+      auto issue_st = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+          mma_ss(tmem + d_col, sdesc_sw128(a_base + off, 16, 1024),
+                 sdesc_sw128(b_base + off, 16, 1024), C::IDESC_ST, kk > 0 ? 1u : 0u);
+        }
+      };
+      // [dV | dK] (128 keys x 128 d) += A (TMEM, bf16 keys x queries: query half h packed at
+      // columns 96h..96h+31) * B (queries x d, MN-major; the two 64-wide d blocks BLK apart)
+      auto issue_kv = [&](uint32_t d_col, uint32_t a_col, uint32_t b_base, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + d_col, tmem + a_col + 96 * (kk >> 2) + (kk & 3) * 8,
+                 sdesc_sw128(b_base + kk * 2048, C::BLK, 1024), C::IDESC_KV,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      // dK (128 keys x 128 d) += dS^T (keys x queries, K-major, shared) * Q_i (queries x d)
+      auto issue_dk_ss = [&](uint32_t b_base, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + C::T_DK, sdesc_sw128(ds_addr + (kk >> 2) * C::BLK + (kk & 3) * 32, 16, 1024),
+                 sdesc_sw128(b_base + kk * 2048, C::BLK, 1024), C::IDESC_KV,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      // dQ^T (128 d x 128 queries) = K^T (d x keys, MN-major) * dS^T (keys x queries, MN-major)
+      auto issue_dq = [&]() {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + C::T_DQ, sdesc_sw128(k_addr + kk * 2048, C::BLK, 1024),
+                 sdesc_sw128(ds_addr + kk * 2048, C::BLK, 1024), C::IDESC_DQ, kk > 0 ? 1u : 0u);
+      };
+      auto next_s = [&](int t) -> bool {  // S^T(t+1) into R1 once dV(t) has read P^T(t)
+        if (!W.wait(BAR_DVD, t & 1, 44)) return false;
+        if (!W.wait(BAR_QF((t + 1) & 1), ((t + 1) >> 1) & 1, 45)) return false;
+        FA_TRACE_EV(3, t);
+        tc_fence_after();
+        issue_st(C::T_S, k_addr, q_addr((t + 1) & 1));
+        tc_commit(BAR_SF);
+        return true;
+      };
+      bool ok = W.wait(BAR_KV, 0, 40);
+      if (ok) ok = W.wait(BAR_QF(0), 0, 41);
+      if (ok) {
+        tc_fence_after();
+        issue_st(C::T_S, k_addr, q_addr(0));
+        tc_commit(BAR_SF);
+        ok = W.wait(BAR_DOF(0), 0, 42);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_st(C::T_DP, v_addr, do_addr(0));
+        tc_commit(BAR_DPF);
+      }
+      for (int t = 0; ok && t < nit; ++t) {
+        const int s = t & 1;
+        const bool more = t + 1 < nit;
+        // dV += P^T dO_i
+        FA_TRACE_EV(1, t);
+        if (!(ok = W.wait(BAR_PF, t & 1, 43))) break;
+        FA_TRACE_EV(2, t);
+        tc_fence_after();
+        issue_kv(C::T_DV, C::T_S, do_addr(t), t > 0);
+        tc_commit(BAR_DVD);
+        tc_commit(BAR_DOE(t % DS_));
+        if (FA_BWDQ_EARLY_S && more && !(ok = next_s(t))) break;
+        FA_TRACE_EV(4, t);
+        if (!(ok = W.wait(BAR_DSF, t & 1, 46))) break;
+        FA_TRACE_EV(5, t);
+        tc_fence_after();
+        if (FA_BWDQ_DK_SS) {
+          // dQ_i^T = K_j^T dS^T into R2 (the dP^T columns, read by now), then dK += dS^T Q_i;
+          // both take dS^T from the shared tile
+          issue_dq();
+          tc_commit(BAR_DQF);
+          issue_dk_ss(q_addr(s), t > 0);
+          tc_commit(BAR_DKD);
+          tc_commit(BAR_QE(s));
+          FA_TRACE_EV(6, t);
+          if (!FA_BWDQ_EARLY_S && more && !(ok = next_s(t))) break;
+        } else {
+          // dK += dS^T Q_i (dS^T from tensor memory)
+          issue_kv(C::T_DK, C::T_DP, q_addr(s), t > 0);
+          tc_commit(BAR_DKD);
+          tc_commit(BAR_QE(s));
+          if (!FA_BWDQ_EARLY_S && more && !(ok = next_s(t))) break;
+          // dQ_i^T = K_j^T dS^T into R2 once dK has read dS^T
+          if (!(ok = W.wait(BAR_DKD, t & 1, 47))) break;
+          FA_TRACE_EV(6, t);
+          tc_fence_after();
+          issue_dq();
+          tc_commit(BAR_DQF);
+        }
+        if (more) {
+          // dP^T(t+1) into R2 once dQ^T(t) has been read out
+          if (!(ok = W.wait(BAR_DQE, t & 1, 48))) break;
+          if (!(ok = W.wait(BAR_DOF((t + 1) % DS_), ((t + 1) / DS_) & 1, 49))) break;
+          FA_TRACE_EV(7, t);
+          tc_fence_after();
+          issue_st(C::T_DP, v_addr, do_addr(t + 1));
+          tc_commit(BAR_DPF);
+        }
+      }
+      // every MMA issued above has completed before the tensor memory is released
+      tc_commit(BAR_DRAIN);
+      W.drain(BAR_DRAIN, 0);
+    }
+  } else if (warp < C::CMP_WARPS) {
+    // ================================================================ P / dS warpgroups
+    regs_inc<C::CMP_REGS>();
+    const int h = warp >> 2;                // query half
+    const int c0 = 64 * h;                  // first query column of this thread
+    const int r = (warp & 3) * 32 + lane;   // key row within the block == TMEM lane
+    const int key = k0 + r;
+    const bool key_ok = key < p.N;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    uint8_t* ds_row = smem + C::OFF_DS + h * C::BLK + r * 128;
+    bool ok = true;
+    for (int t = 0; t < nit; ++t) {
+      const int i = i_start + t;
+      const int s = t & 1;
+      const float* L2s = rows_smem + s * 2 * C::BR + c0;
+      const float* Ds = rows_smem + s * 2 * C::BR + C::BR + c0;
+      if (!(ok = W.wait_warp(BAR_SF, t & 1, 50))) break;
+      if (!(ok = W.wait_warp(BAR_QF(s), (t >> 1) & 1, 51))) break;
+      FA_TRACE_EV(11, t);
+      tc_fence_after();
+      uint32_t sv[2][32];
+      tmem_ld32(tmem + lane_base + C::T_S + c0, sv[0]);
+      tmem_ld32(tmem + lane_base + C::T_S + c0 + 32, sv[1]);
+      tmem_wait_ld(sv[0]);
+      tmem_wait_ld(sv[1]);
+      // P^T = exp2(S^T s log2e - L2); zero for masked (causal key > query) and padded keys.
+      // Only the diagonal block (i == j) and a ragged last key block need the test.
+      uint32_t pk[32];
+      const bool need_mask = !key_ok || (CAUSAL && i == j);
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 l4 = reinterpret_cast<const float4*>(L2s)[c4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        float pr[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * c4 + e;
+          pr[e] = ex2(fmaf(__uint_as_float(sv[c >> 5][c & 31]), p.scale_log2, -lv[e]));
+          if (need_mask) {
+            const bool valid = key_ok && (!CAUSAL || r <= c0 + c);
+            pr[e] = valid ? pr[e] : 0.f;
+          }
+        }
+        pk[2 * c4] = pack_bf16(pr[0], pr[1]);
+        pk[2 * c4 + 1] = pack_bf16(pr[2], pr[3]);
+      }
+      // P^T over this thread's own S^T columns (the whole warpgroup has read them)
+      tmem_st32(tmem + lane_base + C::T_S + 96 * h, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR_PF);
+      FA_TRACE_EV(12, t);
+      // dS^T = P^T * (dP^T - D), with P^T as rounded to bf16 for the dV product
+      if (!(ok = W.wait_warp(BAR_DPF, t & 1, 53))) break;
+      FA_TRACE_EV(13, t);
+      tc_fence_after();
+      tmem_ld32(tmem + lane_base + C::T_DP + c0, sv[0]);
+      tmem_ld32(tmem + lane_base + C::T_DP + c0 + 32, sv[1]);
+      tmem_wait_ld(sv[0]);
+      tmem_wait_ld(sv[1]);
+      uint32_t dsk[32];
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 d4 = reinterpret_cast<const float4*>(Ds)[c4];
+        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = 4 * c4 + 2 * e;
+          const uint32_t pp = pk[c >> 1];
+          const float p0 = __uint_as_float(pp << 16);
+          const float p1 = __uint_as_float(pp & 0xffff0000u);
+          const float d0 = p0 * (__uint_as_float(sv[c >> 5][c & 31]) - dv4[2 * e]);
+          const float d1 = p1 * (__uint_as_float(sv[(c + 1) >> 5][(c + 1) & 31]) - dv4[2 * e + 1]);
+          dsk[c >> 1] = pack_bf16(d0, d1);
+        }
+      }
+      // dS^T into the shared tile (for dQ^T, and for dK when it reads shared memory) and, when dK
+      // reads tensor memory, over this thread's own dP^T columns; with shared staging the tile
+      // is free once the drain warps' reduce of the previous step has read its staging
+      if (!FA_BWDQ_DK_SS) tmem_st32(tmem + lane_base + C::T_DP + 96 * h, dsk);
+      if (!C::SEP && t > 0 && !(ok = W.wait_warp(BAR_DSFREE, (t - 1) & 1, 54))) {
+        if (!FA_BWDQ_DK_SS) tmem_wait_st();
+        break;
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 v = make_uint4(dsk[4 * c], dsk[4 * c + 1], dsk[4 * c + 2], dsk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(ds_row + ((c ^ (r & 7)) << 4)) = v;
+      }
+      fence_async_smem();
+      if (!FA_BWDQ_DK_SS) tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR_DSF);
+      FA_TRACE_EV(14, t);
+    }
+    if (ok) {
+      // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale), bf16
+      ok = W.wait_warp(BAR_DKD, (nit - 1) & 1, 55);
+      if (ok) {
+        tc_fence_after();
+        const size_t base = (size_t(head) * p.N + key) * C::D;
+        const uint32_t col = h == 0 ? C::T_DV : C::T_DK;
+        const float mul = h == 0 ? 1.f : p.scale;
+        __nv_bfloat16* dst = (h == 0 ? p.dv : p.dk) + base;
+#pragma unroll
+        for (int c = 0; c < C::D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + col + 32 * c, v);
+          tmem_wait_ld(v);
+          uint4 pkd[4];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pw[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+          if (key_ok) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d4[e] = pkd[e];
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  } else {
+    // ================================================================ dQ drain warpgroup
+    // dQ^T (d on TMEM lanes, 128 query columns) -> x scale -> two [64 queries][64 d] fp32
+    // staging slots in the dS^T tile's space -> TMA bulk reduce-add into the accumulator, one
+    // query half at a time (rows past N are clipped by the tensor map; halves wholly past N
+    // are skipped).
+    regs_inc<C::DQ_REGS>();
+    const int wq = warp - C::DQ_WARP0;
+    const int tq = threadIdx.x - C::DQ_WARP0 * 32;  // 0..127
+    const bool issuer = tq == 0;
+    const uint32_t lane_base = uint32_t(wq * 32) << 16;
+    const int drow = wq * 32 + lane;                // d index == TMEM lane
+    float* slots = reinterpret_cast<float*>(smem + C::OFF_STG);
+    float* my_slot = slots + (drow >> 6) * (64 * 64) + (drow & 63);
+    if (issuer) tma_prefetch_desc(&tmdQ);
+    for (int t = 0; t < nit; ++t) {
+      const int i = i_start + t;
+      // the four drain warps leave the loop together (they share named barriers below)
+      if (!named_bar_and(1, 128, W.wait_warp(BAR_DQF, t & 1, 60))) break;
+      tc_fence_after();
+      uint32_t v[4][32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld32(tmem + lane_base + C::T_DQ + 32 * q, v[q]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_wait_ld(v[q]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR_DQE);
+#pragma unroll
+      for (int qh = 0; qh < 2; ++qh) {
+        const int row0 = i * C::BR + 64 * qh;
+        if (row0 >= p.N) break;  // uniform over the warpgroup
+        if (qh == 1 || C::SEP) {
+          if (issuer) bulk_wait_group_read<0>();  // the previous reduce has read the slots
+          named_bar_sync(1, 128);
+        }
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          my_slot[c * 64] = __uint_as_float(v[2 * qh + (c >> 5)][c & 31]) * p.scale;
+        fence_async_smem();
+        named_bar_sync(1, 128);
+        if (issuer) {
+          tma_reduce_add_3d(&tmdQ, smem_u32(slots), 0, row0, head);
+          tma_reduce_add_3d(&tmdQ, smem_u32(slots + 64 * 64), 64, row0, head);
+          bulk_commit_group();
+        }
+      }
+      // the dS^T tile may be rewritten once the reduces have read their staging
+      if (!C::SEP && issuer) {
+        bulk_wait_group_read<0>();
+        mbar_arrive(BAR_DSFREE);
+      }
+    }
+    if (issuer) bulk_wait_group_all();
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fattn

@@ -15,6 +15,7 @@
 
 #include "../../include/fattn.h"
 #include "bwd.cuh"
+#include "bwd_q128.cuh"
 #include "fwd.cuh"
 
 namespace {
@@ -212,6 +213,11 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// d = 128 backward: 128-query steps (fa_bwd_kernel_q128); 0 selects the 64-query kernel.
+#ifndef FA_BWD_Q128
+#define FA_BWD_Q128 1
+#endif
+
 template <int D, bool CAUSAL>
 int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, cudaStream_t st) {
   using C = fattn::BwdCfg<D>;
@@ -230,12 +236,39 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fa_bwd preprocess launch");
-  auto kern = fattn::fa_bwd_kernel<D, CAUSAL>;
-  if ((rc = set_smem(kern, C::SMEM_BYTES))) return rc;
-  dim3 grid(unsigned(p.BH) * unsigned(p.nkb) * unsigned(C::NSL));
-  {
-    TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, p);
+  if (D == 128 && FA_BWD_Q128) {
+    // d = 128: 128-query steps (every GEMM of a step is 128 x 128 x 128)
+    using CQ = fattn::BwdQ128Cfg;
+    auto kq = fattn::fa_bwd_kernel_q128<CAUSAL>;
+    if ((rc = set_smem(kq, CQ::SMEM_BYTES))) return rc;
+    // setmaxnreg.inc draws on the registers the CTA was launched with: refuse a build whose
+    // launch allocation is below the kernel's register split
+    static int checked = 0;  // 0 unknown, 1 ok, 2 bad
+    if (checked == 0) {
+      cudaFuncAttributes fa_attr;
+      e = cudaFuncGetAttributes(&fa_attr, kq);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+      checked = (fa_attr.numRegs * CQ::THREADS >=
+                 CQ::CMP_REGS * 256 + CQ::DQ_REGS * 128 + CQ::CTRL_REGS * 128) ? 1 : 2;
+    }
+    if (checked == 2)
+      return fail(FA_ERR_UNSUPPORTED, "fa_bwd kernel built with too few launch registers for its "
+                                      "register split");
+    if ((rc = make_map(&mq, q, p.BH, p.N, D, CQ::BR))) return rc;
+    if ((rc = make_map(&mdo, p.dO, p.BH, p.N, D, CQ::BR))) return rc;
+    dim3 grid(unsigned(p.BH) * unsigned(p.nkb));
+    {
+      TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
+      kq<<<grid, CQ::THREADS, CQ::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, p);
+    }
+  } else {
+    auto kern = fattn::fa_bwd_kernel<D, CAUSAL>;
+    if ((rc = set_smem(kern, C::SMEM_BYTES))) return rc;
+    dim3 grid(unsigned(p.BH) * unsigned(p.nkb) * unsigned(C::NSL));
+    {
+      TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
+      kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, p);
+    }
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fa_bwd launch");
