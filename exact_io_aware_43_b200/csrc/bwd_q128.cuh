@@ -47,11 +47,6 @@
 #ifndef FA_BWDQ_DK_SS
 #define FA_BWDQ_DK_SS 1
 #endif
-// FA_BWDQ_PREFETCH: the producer asks L2 for the Q and dO tiles this many steps ahead of the
-// ones it loads into shared memory (0: no prefetch).
-#ifndef FA_BWDQ_PREFETCH
-#define FA_BWDQ_PREFETCH 0
-#endif
 
 namespace fattn {
 
@@ -156,7 +151,8 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
   constexpr int DS_ = C::DO_STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
-  const Waiter W{abort_flag, p.limit_ns};
+  // plain try_wait polling (no suspend hint) measured faster here than sleeping waits
+  const Waiter W{abort_flag, p.limit_ns, false};
 
   if (threadIdx.x == 0) {
     mbar_init(BAR_KV, 1);
@@ -207,16 +203,6 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       for (int t = 0; t < nit; ++t) {
         const int i = i_start + t;
         const int s = t & 1;
-        if (FA_BWDQ_PREFETCH > 0) {
-          // tiles t+1 .. t+PREFETCH are in flight to L2 after the first step; one more per step
-          for (int u = (t == 0 ? 1 : FA_BWDQ_PREFETCH); u <= FA_BWDQ_PREFETCH; ++u) {
-            if (t + u >= nit) break;
-            for (int kb = 0; kb < 2; ++kb) {
-              tma_prefetch_3d(&tmQ, kb * 64, (i + u) * C::BR, head);
-              tma_prefetch_3d(&tmdO, kb * 64, (i + u) * C::BR, head);
-            }
-          }
-        }
         // Q_i, L2_i and D_i into stage s once dK of step t-2 has released it
         if (!W.wait(BAR_QE(s), ((t >> 1) & 1) ^ 1, 31)) break;
         mbar_arrive_expect_tx(BAR_QF(s), C::TILE + 2 * C::BR * 4);
@@ -384,6 +370,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       tmem_ld32(tmem + lane_base + C::T_S + c0 + 32, sv[1]);
       tmem_wait_ld(sv[0]);
       tmem_wait_ld(sv[1]);
+      FA_TRACE_EV(15, t);
       // P^T = exp2(S^T s log2e - L2); zero for masked (causal key > query) and padded keys.
       // Only the diagonal block (i == j) and a ragged last key block need the test.
       uint32_t pk[32];
@@ -406,8 +393,10 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
         pk[2 * c4 + 1] = pack_bf16(pr[2], pr[3]);
       }
       // P^T over this thread's own S^T columns (the whole warpgroup has read them)
+      FA_TRACE_EV(16, t);
       tmem_st32(tmem + lane_base + C::T_S + 96 * h, pk);
       tmem_wait_st();
+      FA_TRACE_EV(17, t);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_PF);
@@ -420,6 +409,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       tmem_ld32(tmem + lane_base + C::T_DP + c0 + 32, sv[1]);
       tmem_wait_ld(sv[0]);
       tmem_wait_ld(sv[1]);
+      FA_TRACE_EV(18, t);
       uint32_t dsk[32];
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
@@ -439,6 +429,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       // dS^T into the shared tile (for dQ^T, and for dK when it reads shared memory) and, when dK
       // reads tensor memory, over this thread's own dP^T columns; with shared staging the tile
       // is free once the drain warps' reduce of the previous step has read its staging
+      FA_TRACE_EV(19, t);
       if (!FA_BWDQ_DK_SS) tmem_st32(tmem + lane_base + C::T_DP + 96 * h, dsk);
       if (!C::SEP && t > 0 && !(ok = W.wait_warp(BAR_DSFREE, (t - 1) & 1, 54))) {
         if (!FA_BWDQ_DK_SS) tmem_wait_st();
@@ -450,6 +441,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
         *reinterpret_cast<uint4*>(ds_row + ((c ^ (r & 7)) << 4)) = v;
       }
       fence_async_smem();
+      FA_TRACE_EV(21, t);
       if (!FA_BWDQ_DK_SS) tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -503,6 +495,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       const int i = i_start + t;
       // the four drain warps leave the loop together (they share named barriers below)
       if (!named_bar_and(1, 128, W.wait_warp(BAR_DQF, t & 1, 60))) break;
+      FA_TRACE_EV(60, t);
       tc_fence_after();
       uint32_t v[4][32];
 #pragma unroll
@@ -512,6 +505,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_DQE);
+      FA_TRACE_EV(61, t);
 #pragma unroll
       for (int qh = 0; qh < 2; ++qh) {
         const int row0 = i * C::BR + 64 * qh;
@@ -525,6 +519,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
           my_slot[c * 64] = __uint_as_float(v[2 * qh + (c >> 5)][c & 31]) * p.scale;
         fence_async_smem();
         named_bar_sync(1, 128);
+        FA_TRACE_EV(62 + qh, t);
         if (issuer) {
           tma_reduce_add_3d(&tmdQ, smem_u32(slots), 0, row0, head);
           tma_reduce_add_3d(&tmdQ, smem_u32(slots + 64 * 64), 64, row0, head);

@@ -128,15 +128,19 @@ __device__ __forceinline__ uint32_t mbar_try_wait_sleep(uint32_t bar, uint32_t p
 struct Waiter {
   volatile int* abort_flag;
   uint64_t limit_ns;
+  bool sleep = true;  // false: poll with plain try_wait between the abort / deadline checks
 
-  // After the first failed try_wait the thread sleeps in try_wait (up to 1 ms per call, woken
-  // when the phase completes); between calls it checks the abort flag and the deadline.  A
-  // busy spin measurably slowed both kernels by taking issue slots from the computing warps.
+  // After the first failed try_wait the thread waits in try_wait again -- with `sleep`, with a
+  // 1 ms suspend hint (woken when the phase completes), else with the hardware's own short
+  // suspend -- and between calls checks the abort flag and the deadline.  Which is faster
+  // depends on the kernel (it trades wake-up latency against issue slots taken from the
+  // computing warps), so each kernel picks one by measurement.
   __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, int site) const {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
-      if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+      if (sleep ? mbar_try_wait_sleep(bar, parity, 1000000u) : mbar_try_wait(bar, parity))
+        return true;
       if (*abort_flag) return false;
       if (global_ns() - t0 > limit_ns) {
         *abort_flag = 1;
@@ -177,14 +181,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
-}
-
-// Prefetch a 3-D tile into L2 (no shared-memory destination, no completion to wait for).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* m, int x, int y, int z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(x), "r"(y), "r"(z)
-               : "memory");
 }
 
 // Untiled bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
