@@ -44,16 +44,18 @@ def draw_bits(shape, seed: int, tensor: str, sigma: float = 1.0) -> np.ndarray:
 
 
 def make_inputs(B: int, H: int, N: int, d: int, seed: int = 0, sigma_qk: float = 1.0,
-                with_do: bool = True) -> dict:
-    """Q, K, V (and dO) as bf16 bit arrays of shape [B, H, N, d].
+                with_do: bool = True, kv_heads: int | None = None) -> dict:
+    """Q, K, V (and dO) as bf16 bit arrays: Q and dO [B, H, N, d], K and V [B, H_kv, N, d] with
+    H_kv = ``kv_heads`` (default H; a divisor of H for grouped-query attention).
 
     ``sigma_qk`` = 3 gives the peaky-softmax variant (Q, K ~ N(0, 3^2)); V and dO stay N(0, 1).
     """
     shape = (B, H, N, d)
+    kv_shape = (B, H if kv_heads is None else kv_heads, N, d)
     out = {
         "q": draw_bits(shape, seed, "q", sigma_qk),
-        "k": draw_bits(shape, seed, "k", sigma_qk),
-        "v": draw_bits(shape, seed, "v", 1.0),
+        "k": draw_bits(kv_shape, seed, "k", sigma_qk),
+        "v": draw_bits(kv_shape, seed, "v", 1.0),
     }
     if with_do:
         out["do"] = draw_bits(shape, seed, "do", 1.0)

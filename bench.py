@@ -64,12 +64,20 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--shape", default=None,
                     help="B,H,N,d,causal override (profiling runs on a smaller case)")
+    ap.add_argument("--kv-heads", type=int, default=None,
+                    help="key/value heads per batch (grouped-query attention; default: H)")
     args = ap.parse_args(argv)
+    global WORKLOAD_NAME
     if args.shape:
         B, H, N, d, c = (int(x) for x in args.shape.split(","))
         WORKLOAD.update(B=B, H=H, N=N, d=d, causal=bool(c))
-        global WORKLOAD_NAME
         WORKLOAD_NAME = f"shape override B={B} H={H} N={N} d={d} causal={bool(c)} (profiling)"
+    if args.kv_heads is not None and args.kv_heads != WORKLOAD["H"]:
+        if args.kv_heads < 1 or WORKLOAD["H"] % args.kv_heads:
+            ap.error("--kv-heads must divide H")
+        WORKLOAD["H_kv"] = args.kv_heads
+        WORKLOAD_NAME += (f", grouped-query attention: {WORKLOAD['H']} query heads on "
+                          f"{args.kv_heads} key/value heads")
     return args
 
 
@@ -272,7 +280,7 @@ def run_gpu(args):
     W = WORKLOAD
     B, H, N, d, causal = W["B"], W["H"], W["N"], W["d"], W["causal"]
     s = ai.default_scale(d)
-    x = ai.make_inputs(B, H, N, d, seed=rank_seed(rank))
+    x = ai.make_inputs(B, H, N, d, seed=rank_seed(rank), kv_heads=W.get("H_kv"))
     host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) for k, v in x.items()}
     q, k, v, do = (host[t].to(dev) for t in ("q", "k", "v", "do"))
     o = torch.empty_like(q)
@@ -349,7 +357,7 @@ def run_gpu(args):
     e2e = None
     if args.e2e_steps > 0:
         hin = {t: host[t].pin_memory() for t in ("q", "k", "v", "do")}
-        hout = [torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+        hout = [torch.empty(t.shape, dtype=torch.bfloat16).pin_memory() for t in (dq, dk, dv)]
         e_ev = []
         torch.cuda.synchronize()
         barrier(dev)

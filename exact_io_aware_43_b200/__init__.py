@@ -1,8 +1,9 @@
 """exact_io_aware_43_b200 -- exact, IO-aware attention on B200 (sm_100a).
 
 Thin Python binding over the C ABI of ``libfattn.so`` (include/fattn.h).  The functions
-``fa_fwd``, ``fa_bwd``, ``fa_bwd_workspace_size``, ``fa_last_error``, ``fa_device_status`` have
-the same names and arguments as the C entry points (pointers as Python ints, streams as raw
+``fa_fwd``, ``fa_bwd``, ``fa_fwd_gqa``, ``fa_bwd_gqa``, ``fa_bwd_workspace_size``,
+``fa_last_error``, ``fa_device_status`` (and the rest) have the same names and arguments as the
+C entry points (pointers as Python ints, streams as raw
 ``cudaStream_t`` handles).  ``forward``/``backward``/``attention`` are conveniences that take
 torch tensors, allocate the outputs with torch (device memory and streams are the only things
 torch provides here) and call the same entry points.  There is no other code path: if the
@@ -46,6 +47,10 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_workspace_size.restype = sz
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
     L.fa_bwd.restype = i
+    L.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
+    L.fa_fwd_gqa.restype = i
+    L.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, sz, vp]
+    L.fa_bwd_gqa.restype = i
     L.fa_last_error.argtypes = []
     L.fa_last_error.restype = ctypes.c_char_p
     L.fa_device_status.argtypes = [vp]
@@ -92,6 +97,16 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, workspace
            workspace_bytes, stream) -> int:
     return lib().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, int(causal), float(scale),
                         workspace, workspace_bytes, stream)
+
+
+def fa_fwd_gqa(q, k, v, o, lse, B, H, H_kv, N, d, causal, scale, stream) -> int:
+    return lib().fa_fwd_gqa(q, k, v, o, lse, B, H, H_kv, N, d, int(causal), float(scale), stream)
+
+
+def fa_bwd_gqa(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, causal, scale, workspace,
+               workspace_bytes, stream) -> int:
+    return lib().fa_bwd_gqa(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, int(causal),
+                            float(scale), workspace, workspace_bytes, stream)
 
 
 def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, stream) -> int:
@@ -146,19 +161,41 @@ def _default_scale(d):
     return float(np.float32(1.0 / np.sqrt(np.float64(d))))
 
 
+def _check_tensor(t, shape, dtype, name):
+    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape:
+        raise ValueError(f"{name} must be a contiguous {dtype} CUDA tensor of shape {shape}")
+
+
+def _kv_heads(q, k):
+    """H_kv of k ([B, H_kv, N, d]); H_kv must divide q's H (grouped-query attention)."""
+    B, H, N, d = _shape(q)
+    if k.dim() != 4 or k.shape[0] != B or k.shape[2] != N or k.shape[3] != d or \
+            k.shape[1] < 1 or H % k.shape[1] != 0:
+        raise ValueError("k, v must be [B, H_kv, N, d] with H_kv dividing q's H")
+    return int(k.shape[1])
+
+
 def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
-    """O, L = attention(q, k, v) for contiguous bf16 CUDA tensors [B, H, N, d]."""
+    """O, L = attention(q, k, v) for contiguous bf16 CUDA tensors: q [B, H, N, d] and k, v
+    [B, H_kv, N, d] (H_kv = H, or a divisor of H for grouped-query attention)."""
     import torch
     B, H, N, d = _shape(q)
-    for t in (q, k, v):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or \
-                tuple(t.shape) != (B, H, N, d):
-            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors of one shape")
+    Hkv = _kv_heads(q, k)
+    _check_tensor(q, (B, H, N, d), torch.bfloat16, "q")
+    _check_tensor(k, (B, Hkv, N, d), torch.bfloat16, "k")
+    _check_tensor(v, (B, Hkv, N, d), torch.bfloat16, "v")
     scale = _default_scale(d) if scale is None else float(scale)
     o = torch.empty_like(q) if out is None else out
     L = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    _check(fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
-                  B, H, N, d, causal, scale, _stream_handle(q)))
+    _check_tensor(o, (B, H, N, d), torch.bfloat16, "out")
+    _check_tensor(L, (B, H, N), torch.float32, "lse")
+    if Hkv == H:
+        rc = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
+                    B, H, N, d, causal, scale, _stream_handle(q))
+    else:
+        rc = fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
+                        B, H, Hkv, N, d, causal, scale, _stream_handle(q))
+    _check(rc)
     return o, L
 
 
@@ -167,6 +204,12 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
     """dQ, dK, dV for contiguous bf16 CUDA tensors; ``workspace`` (uint8 CUDA tensor) optional."""
     import torch
     B, H, N, d = _shape(q)
+    Hkv = _kv_heads(q, k)
+    for t, shp, name in ((q, (B, H, N, d), "q"), (k, (B, Hkv, N, d), "k"),
+                         (v, (B, Hkv, N, d), "v"), (o, (B, H, N, d), "o"),
+                         (do, (B, H, N, d), "do")):
+        _check_tensor(t, shp, torch.bfloat16, name)
+    _check_tensor(lse, (B, H, N), torch.float32, "lse")
     scale = _default_scale(d) if scale is None else float(scale)
     need = fa_bwd_workspace_size(B, H, N, d)
     if workspace is None:
@@ -174,10 +217,18 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     dq, dk, dv = grads
-    _check(fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                  do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                  B, H, N, d, causal, scale, workspace.data_ptr(), workspace.numel(),
-                  _stream_handle(q)))
+    for t, shp, name in ((dq, (B, H, N, d), "dq"), (dk, (B, Hkv, N, d), "dk"),
+                         (dv, (B, Hkv, N, d), "dv")):
+        _check_tensor(t, shp, torch.bfloat16, name)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+            do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
+    if Hkv == H:
+        rc = fa_bwd(*args, B, H, N, d, causal, scale, workspace.data_ptr(), workspace.numel(),
+                    _stream_handle(q))
+    else:
+        rc = fa_bwd_gqa(*args, B, H, Hkv, N, d, causal, scale, workspace.data_ptr(),
+                        workspace.numel(), _stream_handle(q))
+    _check(rc)
     return dq, dk, dv
 
 

@@ -56,13 +56,65 @@ struct BwdParams {
   float* dq_acc;   // [BH, N, D] fp32
   float* L2;       // [BH, Npad] fp32: lse * log2(e), +inf on padded rows
   float* Drow;     // [BH, Npad] fp32: rowsum(dO * O), 0 on padded rows
-  int BH;
+  int BH;          // batch * query heads (rows of dq_acc, L2, Drow)
   int N;
   int Npad;        // N rounded up to 128
   int nkb;         // key blocks of 128 per head
+  int H;           // query heads per batch
+  int Hkv;         // key/value heads per batch (H is a multiple of Hkv)
+  int G;           // query heads per key/value head, H / Hkv
+  int BHkv;        // batch * key/value heads (CTAs of the main kernels: BHkv x key blocks)
   float scale;
   float scale_log2;
   uint64_t limit_ns;
+};
+
+// Grouped heads in the main backward kernels.  A CTA owns key block j of key/value head kvh
+// (= b * Hkv + hk) and runs nit_h query-block steps for each of the G query heads b * H + hk * G
+// + g that share it, one head after the other; dK_j and dV_j accumulate over all of them in
+// tensor memory (the gradient of a shared K/V row is the sum over the heads that read it).
+struct BwdGroup {
+  int qh0;      // first query head of the group
+  int nit_h;    // query-block steps per query head
+  int i_start;  // first query block
+  __device__ __forceinline__ BwdGroup(const BwdParams& p, int kvh, int i0, int nqblk)
+      : qh0((kvh / p.Hkv) * p.H + (kvh % p.Hkv) * p.G), nit_h(nqblk - i0), i_start(i0) {}
+};
+// CTA -> (key block j, key/value head, d slice).  Heads are taken in bands of kBwdHeadBand; within
+// a band the key block is outermost, so the key blocks with the most query steps (causal: the
+// first ones) of the band's heads start first, while the query tiles in flight stay those of a
+// few heads (their reads are served from L2).
+#ifndef FA_BWD_HEAD_BAND
+#define FA_BWD_HEAD_BAND 4
+#endif
+constexpr int kBwdHeadBand = FA_BWD_HEAD_BAND;
+struct BwdUnit {
+  int j, kvh, slice;
+  __device__ __forceinline__ BwdUnit(int x, const BwdParams& p, int nsl) {
+    const int band_ctas = kBwdHeadBand * p.nkb * nsl;
+    const int band = x / band_ctas;
+    const int h0 = band * kBwdHeadBand;
+    const int nh = min(kBwdHeadBand, p.BHkv - h0);
+    const int r = x - band * band_ctas;
+    j = r / (nh * nsl);
+    const int rem = r - j * (nh * nsl);
+    kvh = h0 + rem / nsl;
+    slice = rem - (rem / nsl) * nsl;
+  }
+};
+
+// Walks the steps of a BwdGroup in order (no division per step): `i` and `head` describe the
+// current step; next() moves to the following one.
+struct BwdCursor {
+  int i, head, i_start, i_end;
+  __device__ __forceinline__ explicit BwdCursor(const BwdGroup& g)
+      : i(g.i_start), head(g.qh0), i_start(g.i_start), i_end(g.i_start + g.nit_h) {}
+  __device__ __forceinline__ void next() {
+    if (++i == i_end) {
+      i = i_start;
+      ++head;
+    }
+  }
 };
 
 // ------------------------------------------------------------------------------------------
@@ -196,16 +248,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const int lane = threadIdx.x & 31;
   FA_TRACE_DECL;
 
-  // ---- work unit: (head, key block j, d slice); key blocks with more queries first
-  const int per_head = p.nkb * C::NSL;
-  const int head = blockIdx.x / per_head;
-  const int rem = blockIdx.x % per_head;
-  const int j = rem / C::NSL;
-  const int slice = rem % C::NSL;
+  // ---- work unit: (key block j, key/value head, d slice) in the order of BwdUnit.  Steps run
+  // over the group's query heads, each over its query blocks (see BwdGroup).
+  const BwdUnit unit(blockIdx.x, p, C::NSL);
+  const int j = unit.j, kvh = unit.kvh, slice = unit.slice;
   const int k0 = j * C::BC;
   const int nqblk = (p.N + C::BR - 1) / C::BR;
-  const int i_start = CAUSAL ? (k0 / C::BR) : 0;
-  const int nit = nqblk - i_start;  // >= 1
+  const BwdGroup grp(p, kvh, CAUSAL ? (k0 / C::BR) : 0, nqblk);
+  const int nit = p.G * grp.nit_h;  // >= 1
 
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
   const uint32_t BAR_KV = bar(0);
@@ -258,12 +308,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tma_prefetch_desc(&tmdO);
       mbar_arrive_expect_tx(BAR_KV, 2 * C::KV_BYTES);
       for (int kb = 0; kb < C::KB; ++kb) {
-        tma_load_3d(sbase + C::OFF_K + kb * C::KV_BLK, &tmK, BAR_KV, kb * 64, k0, head);
-        tma_load_3d(sbase + C::OFF_V + kb * C::KV_BLK, &tmV, BAR_KV, kb * 64, k0, head);
+        tma_load_3d(sbase + C::OFF_K + kb * C::KV_BLK, &tmK, BAR_KV, kb * 64, k0, kvh);
+        tma_load_3d(sbase + C::OFF_V + kb * C::KV_BLK, &tmV, BAR_KV, kb * 64, k0, kvh);
       }
       int it = 0;
+      BwdCursor cur(grp);
       for (; it < nit; ++it) {
-        const int i = i_start + it;
+        const int i = cur.i, head = cur.head;
+        cur.next();
         const int s = it % C::STAGES;
         if (!W.wait(BAR_QE(s), ((it / C::STAGES) & 1) ^ 1, 31)) break;
         FA_TRACE_EV(20, it);
@@ -390,8 +442,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     uint8_t* ds_row = smem + C::OFF_DS + r * 128;
     bool ok = true;
+    BwdCursor cur(grp);
     for (int it = 0; it < nit; ++it) {
-      const int i = i_start + it;
+      const int i = cur.i;
+      cur.next();
       const int s = it % C::STAGES;
       const float* L2s = rows_smem + s * 2 * C::BR + c0;
       const float* Ds = rows_smem + s * 2 * C::BR + C::BR + c0;
@@ -501,7 +555,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       ok = W.wait_warp(BAR_DQF, (nit - 1) & 1, 55);
       if (ok) {
         tc_fence_after();
-        const size_t base = (size_t(head) * p.N + key) * D + slice * C::DO;
+        const size_t base = (size_t(kvh) * p.N + key) * D + slice * C::DO;
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
           if (C::SPLIT && which != h) continue;
@@ -545,8 +599,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     float* slots = reinterpret_cast<float*>(smem + C::OFF_DQS);
     if (issuer) tma_prefetch_desc(&tmdQ);
     int group = 0;
+    BwdCursor cur(grp);
     for (int it = 0; it < nit; ++it) {
-      const int i = i_start + it;
+      const int i = cur.i, head = cur.head;
+      cur.next();
       // the four drain warps leave the loop together (they share named barriers below)
       if (!named_bar_and(1, 128, W.wait_warp(BAR_DQF, it & 1, 60))) break;
       tc_fence_after();

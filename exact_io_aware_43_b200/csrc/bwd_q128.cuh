@@ -131,13 +131,14 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
   const int lane = threadIdx.x & 31;
   FA_TRACE_DECL;
 
-  // ---- work unit: (head, key block j); query blocks i from j (causal) or 0 to the last
-  const int head = blockIdx.x / p.nkb;
-  const int j = blockIdx.x % p.nkb;
+  // ---- work unit: (key block j, key/value head) in the order of BwdUnit; for each query head
+  // of the group (see BwdGroup), query blocks i from j (causal) or 0 to the last
+  const BwdUnit unit(blockIdx.x, p, 1);
+  const int j = unit.j, kvh = unit.kvh;
   const int k0 = j * C::BC;
   const int nqb = (p.N + C::BR - 1) / C::BR;
-  const int i_start = CAUSAL ? j : 0;
-  const int nit = nqb - i_start;  // >= 1
+  const BwdGroup grp(p, kvh, CAUSAL ? j : 0, nqb);
+  const int nit = p.G * grp.nit_h;  // >= 1
 
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
   const uint32_t BAR_KV = bar(0);
@@ -196,12 +197,14 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       tma_prefetch_desc(&tmdO);
       mbar_arrive_expect_tx(BAR_KV, 2 * C::TILE);
       for (int kb = 0; kb < 2; ++kb) {
-        tma_load_3d(sbase + C::OFF_K + kb * C::BLK, &tmK, BAR_KV, kb * 64, k0, head);
-        tma_load_3d(sbase + C::OFF_V + kb * C::BLK, &tmV, BAR_KV, kb * 64, k0, head);
+        tma_load_3d(sbase + C::OFF_K + kb * C::BLK, &tmK, BAR_KV, kb * 64, k0, kvh);
+        tma_load_3d(sbase + C::OFF_V + kb * C::BLK, &tmV, BAR_KV, kb * 64, k0, kvh);
       }
       int tq = 0, td = 0;  // Q / dO tiles issued
+      BwdCursor cur(grp);
       for (int t = 0; t < nit; ++t) {
-        const int i = i_start + t;
+        const int i = cur.i, head = cur.head;
+        cur.next();
         const int s = t & 1;
         // Q_i, L2_i and D_i into stage s once dK of step t-2 has released it
         if (!W.wait(BAR_QE(s), ((t >> 1) & 1) ^ 1, 31)) break;
@@ -356,8 +359,10 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     uint8_t* ds_row = smem + C::OFF_DS + h * C::BLK + r * 128;
     bool ok = true;
+    BwdCursor cur(grp);
     for (int t = 0; t < nit; ++t) {
-      const int i = i_start + t;
+      const int i = cur.i;
+      cur.next();
       const int s = t & 1;
       const float* L2s = rows_smem + s * 2 * C::BR + c0;
       const float* Ds = rows_smem + s * 2 * C::BR + C::BR + c0;
@@ -453,7 +458,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       ok = W.wait_warp(BAR_DKD, (nit - 1) & 1, 55);
       if (ok) {
         tc_fence_after();
-        const size_t base = (size_t(head) * p.N + key) * C::D;
+        const size_t base = (size_t(kvh) * p.N + key) * C::D;
         const uint32_t col = h == 0 ? C::T_DV : C::T_DK;
         const float mul = h == 0 ? 1.f : p.scale;
         __nv_bfloat16* dst = (h == 0 ? p.dv : p.dk) + base;
@@ -491,8 +496,10 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
     float* slots = reinterpret_cast<float*>(smem + C::OFF_STG);
     float* my_slot = slots + (drow >> 6) * (64 * 64) + (drow & 63);
     if (issuer) tma_prefetch_desc(&tmdQ);
+    BwdCursor cur(grp);
     for (int t = 0; t < nit; ++t) {
-      const int i = i_start + t;
+      const int i = cur.i, head = cur.head;
+      cur.next();
       // the four drain warps leave the loop together (they share named barriers below)
       if (!named_bar_and(1, 128, W.wait_warp(BAR_DQF, t & 1, 60))) break;
       FA_TRACE_EV(60, t);

@@ -125,6 +125,13 @@ uint64_t wait_limit_ns() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Grouped heads: H query heads share H_kv key/value heads, H / H_kv consecutive query heads each.
+int check_groups(int H, int H_kv) {
+  if (H_kv < 1 || H_kv > H || H % H_kv != 0)
+    return fail(FA_ERR_INVALID_ARG, "H_kv must divide H (got H=%d, H_kv=%d)", H, H_kv);
+  return FA_OK;
+}
+
 int check_common(int B, int H, int N, int d, float scale) {
   if (B < 1 || H < 1 || N < 1)
     return fail(FA_ERR_INVALID_ARG, "B, H and N must be >= 1 (got %d, %d, %d)", B, H, N);
@@ -224,8 +231,8 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
   int rc;
   CUtensorMap mq, mk, mv, mdo;
   if ((rc = make_map(&mq, q, p.BH, p.N, D, C::BR))) return rc;
-  if ((rc = make_map(&mk, k, p.BH, p.N, D, C::BC))) return rc;
-  if ((rc = make_map(&mv, v, p.BH, p.N, D, C::BC))) return rc;
+  if ((rc = make_map(&mk, k, p.BHkv, p.N, D, C::BC))) return rc;
+  if ((rc = make_map(&mv, v, p.BHkv, p.N, D, C::BC))) return rc;
   if ((rc = make_map(&mdo, p.dO, p.BH, p.N, D, C::BR))) return rc;
   CUtensorMap mdq;
   if ((rc = make_map_f32(&mdq, p.dq_acc, p.BH, p.N, D))) return rc;
@@ -256,7 +263,7 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
                                       "register split");
     if ((rc = make_map(&mq, q, p.BH, p.N, D, CQ::BR))) return rc;
     if ((rc = make_map(&mdo, p.dO, p.BH, p.N, D, CQ::BR))) return rc;
-    dim3 grid(unsigned(p.BH) * unsigned(p.nkb));
+    dim3 grid(unsigned(p.BHkv) * unsigned(p.nkb));
     {
       TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
       kq<<<grid, CQ::THREADS, CQ::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, p);
@@ -264,7 +271,7 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
   } else {
     auto kern = fattn::fa_bwd_kernel<D, CAUSAL>;
     if ((rc = set_smem(kern, C::SMEM_BYTES))) return rc;
-    dim3 grid(unsigned(p.BH) * unsigned(p.nkb) * unsigned(C::NSL));
+    dim3 grid(unsigned(p.BHkv) * unsigned(p.nkb) * unsigned(C::NSL));
     {
       TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
       kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, p);
@@ -283,8 +290,9 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
 }
 
 int bwd_dispatch(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                 const void* dO, void* dq, void* dk, void* dv, int BH, int N, int d, bool causal,
-                 float scale, void* workspace, cudaStream_t st) {
+                 const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int d,
+                 bool causal, float scale, void* workspace, cudaStream_t st) {
+  const int BH = B * H;
   fattn::BwdParams p{};
   p.o = static_cast<const __nv_bfloat16*>(o);
   p.dO = static_cast<const __nv_bfloat16*>(dO);
@@ -303,6 +311,10 @@ int bwd_dispatch(const void* q, const void* k, const void* v, const void* o, con
   p.N = N;
   p.Npad = int(npad);
   p.nkb = (N + 127) / 128;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.BHkv = B * Hkv;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.limit_ns = wait_limit_ns();
@@ -320,24 +332,27 @@ const char* fa_last_error(void) { return g_msg; }
 
 int fa_version(void) { return 100; }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
-           int d, int causal, float scale, void* stream) {
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int H_kv, int N, int d, int causal, float scale, void* stream) {
   g_msg[0] = 0;
   if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID_ARG, "null tensor pointer");
   int rc = check_common(B, H, N, d, scale);
   if (rc) return rc;
+  if ((rc = check_groups(H, H_kv))) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return fail(FA_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
   if ((rc = check_device())) return rc;
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
   if ((rc = make_map(&mq, q, BH, N, d, 128))) return rc;
-  if ((rc = make_map(&mk, k, BH, N, d, 128))) return rc;
-  if ((rc = make_map(&mv, v, BH, N, d, 128))) return rc;
+  if ((rc = make_map(&mk, k, B * H_kv, N, d, 128))) return rc;
+  if ((rc = make_map(&mv, v, B * H_kv, N, d, 128))) return rc;
   fattn::FwdParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.N = N;
+  p.H = H;
+  p.G = H / H_kv;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.limit_ns = wait_limit_ns();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -351,6 +366,11 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
                 : launch_fwd<256, false, 1>(mq, mk, mv, p, BH, st);
 }
 
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+           int d, int causal, float scale, void* stream) {
+  return fa_fwd_gqa(q, k, v, o, lse, B, H, H, N, d, causal, scale, stream);
+}
+
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128 && d != 256)) return 0;
   const size_t bh = size_t(B) * size_t(H);
@@ -360,14 +380,15 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return dq + 2 * rows;
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-           const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal,
-           float scale, void* workspace, size_t workspace_bytes, void* stream) {
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
+               int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
   g_msg[0] = 0;
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv)
     return fail(FA_ERR_INVALID_ARG, "null tensor pointer");
   int rc = check_common(B, H, N, d, scale);
   if (rc) return rc;
+  if ((rc = check_groups(H, H_kv))) return rc;
   for (const void* ptr : {q, k, v, o, static_cast<const void*>(lse), dO,
                           static_cast<const void*>(dq), static_cast<const void*>(dk),
                           static_cast<const void*>(dv)})
@@ -376,8 +397,15 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if (!workspace || !aligned16(workspace) || workspace_bytes < need)
     return fail(FA_ERR_WORKSPACE, "workspace must be 16-byte aligned and >= %zu bytes", need);
   if ((rc = check_device())) return rc;
-  return bwd_dispatch(q, k, v, o, lse, dO, dq, dk, dv, B * H, N, d, causal != 0, scale,
+  return bwd_dispatch(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, causal != 0, scale,
                       workspace, static_cast<cudaStream_t>(stream));
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal,
+           float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return fa_bwd_gqa(q, k, v, o, lse, dO, dq, dk, dv, B, H, H, N, d, causal, scale, workspace,
+                    workspace_bytes, stream);
 }
 
 int fa_timer_enable(int on) {
@@ -477,7 +505,7 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
   if ((rc = check_device())) return rc;
   void* ws = nullptr;
   if ((rc = noalloc_scratch(&ws))) return rc;
-  return bwd_dispatch(q, k, v, o, lse, dO, dq, dk, dv, B * H, N, d, causal != 0, scale, ws,
+  return bwd_dispatch(q, k, v, o, lse, dO, dq, dk, dv, B, H, H, N, d, causal != 0, scale, ws,
                       static_cast<cudaStream_t>(stream));
 }
 

@@ -53,7 +53,9 @@ struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
   int N;            // sequence length (queries = keys)
-  int BH;           // batch * heads
+  int BH;           // batch * query heads
+  int H;            // query heads per batch
+  int G;            // query heads per key/value head (grouped-query attention; 1 = one each)
   int nqb;          // query blocks (of NQT*128 rows) per head
   int units;        // BH * nqb
   float scale_log2; // scale * log2(e)
@@ -104,15 +106,17 @@ __device__ __forceinline__ int fwd_unit_of(int k, int c, int G, int units) {
   return u < units ? u : -1;
 }
 
-// Unit u -> (head, first query row, KV tiles per query tile).  Units are numbered query block
-// major, heaviest (latest) query blocks first when causal, heads inner.
+// Unit u -> (head, its key/value head, first query row, KV tiles per query tile).  Units are
+// numbered query block major, heaviest (latest) query blocks first when causal, heads inner, so
+// the query heads that share a key/value head run side by side and share its tiles in L2.
 template <int NQT, bool CAUSAL>
 struct FwdUnit {
-  int head, q0, J;
+  int head, kv_head, q0, J;
   int nkv[NQT];
   __device__ __forceinline__ FwdUnit(int u, const FwdParams& p) {
     const int qi = u / p.BH;
     head = u - qi * p.BH;
+    kv_head = (head / p.H) * (p.H / p.G) + (head % p.H) / p.G;
     const int qb = CAUSAL ? (p.nqb - 1 - qi) : qi;
     q0 = qb * NQT * 128;
     const int n_kv_total = (p.N + 127) / 128;
@@ -225,13 +229,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
             mbar_arrive_expect_tx(BAR_KF(s), C::KVTILE_BYTES);
             for (int kb = 0; kb < C::KB; ++kb)
               tma_load_3d(sbase + C::OFF_K + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmK,
-                          BAR_KF(s), kb * 64, j * C::BN, un.head);
+                          BAR_KF(s), kb * 64, j * C::BN, un.kv_head);
             if (!(ok = W.wait(BAR_VE(s), ph ^ 1, 2))) break;
             FA_TRACE_EV(21, j);
             mbar_arrive_expect_tx(BAR_VF(s), C::KVTILE_BYTES);
             for (int kb = 0; kb < C::KB; ++kb)
               tma_load_3d(sbase + C::OFF_V + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmV,
-                          BAR_VF(s), kb * 64, j * C::BN, un.head);
+                          BAR_VF(s), kb * 64, j * C::BN, un.kv_head);
           }
           if (!ok) break;
           kv_it += un.J;

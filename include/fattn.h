@@ -117,13 +117,36 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    const void* dO, void* dq, void* dk, void* dv,
                    int B, int H, int N, int d, int causal, float scale, void* stream);
 
+/*
+ * Grouped-query attention (GQA): H query heads share H_kv key/value heads.  H_kv = 1 is the
+ * multi-query attention (MQA) that systems-analysis.info "FlashAttention (PL)", section
+ * "FlashAttention-2 (2023)", lists among the second version's additions; H_kv between 1 and H
+ * generalises it.  Query head h reads key/value head h / (H / H_kv): consecutive groups
+ * of H / H_kv query heads share one.  The result is exactly that of fa_fwd / fa_bwd on K and V
+ * with each key/value head repeated H / H_kv times, without materialising the copies.
+ *   q, o, dO, dq : bfloat16 [B, H, N, d]        lse : float32 [B, H, N]
+ *   k, v, dk, dv : bfloat16 [B, H_kv, N, d]
+ * dk and dv hold the gradient summed over the H / H_kv query heads that read each key/value
+ * head.  H_kv must divide H (else FA_ERR_INVALID_ARG).  The workspace is the one
+ * fa_bwd_workspace_size(B, H, N, d) gives (it depends on the query heads only).  Every other
+ * convention -- alignment, ownership, streams, errors -- is that of fa_fwd / fa_bwd, which are
+ * these calls with H_kv = H.
+ */
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+               int B, int H, int H_kv, int N, int d, int causal, float scale, void* stream);
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dO, void* dq, void* dk, void* dv,
+               int B, int H, int H_kv, int N, int d, int causal, float scale,
+               void* workspace, size_t workspace_bytes, void* stream);
+
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 const char* fa_last_error(void);
 
 /*
  * fa_device_status -- synchronises `stream`, then reads and clears the device status word of
  * the current device.  Returns FA_OK, FA_ERR_TIMEOUT if a kernel abandoned a bounded wait since
- * the last call, or FA_ERR_CUDA if the synchronisation itself failed.
+ * the last call, FA_ERR_UNSUPPORTED if a kernel found its shared memory placed so that its tiles
+ * could not be aligned and did no work, or FA_ERR_CUDA if the synchronisation itself failed.
  */
 int fa_device_status(void* stream);
 

@@ -217,3 +217,42 @@ def attention_dq_rows(q, k, v, do, rows, causal: bool, scale: float):
     D = np.sum(do[rows] * O, axis=1)
     ds = p * (dp - D[:, None])
     return scale * (ds @ k)
+
+
+def _group_size(q, k):
+    H, Hkv = q.shape[1], k.shape[1]
+    if Hkv < 1 or H % Hkv:
+        raise ValueError("the key/value head count must divide the query head count")
+    return H // Hkv
+
+
+def attention_forward_gqa(q, k, v, causal: bool, scale: float):
+    """Grouped-query attention forward: q [B,H,N,d], k and v [B,H_kv,N,d] with H_kv dividing H.
+
+    [P2] section "FlashAttention-2 (2023)" lists multi-query attention (one key/value head for all
+    query heads) among the method's extensions; the grouped form lets query head h read key/value
+    head h // (H // H_kv), consecutive groups of query heads sharing one.  Written as the plain
+    definition: attention with each key/value head repeated for the query heads of its group.
+    Returns (O [B,H,N,d], L [B,H,N]).
+    """
+    G = _group_size(q, k)
+    k_rep = np.repeat(np.asarray(k, np.float64), G, axis=1)
+    v_rep = np.repeat(np.asarray(v, np.float64), G, axis=1)
+    return attention_forward(q, k_rep, v_rep, causal, scale)
+
+
+def attention_backward_gqa(q, k, v, o, lse, do, causal: bool, scale: float):
+    """Gradients of the grouped-query attention above.
+
+    A shared key/value row enters the loss once per query head of its group, so its gradient is
+    the sum of the per-head gradients: dK and dV of the repeated heads, summed over each group.
+    Returns (dQ [B,H,N,d], dK [B,H_kv,N,d], dV [B,H_kv,N,d]).
+    """
+    G = _group_size(q, k)
+    B, Hkv, N, d = k.shape
+    k_rep = np.repeat(np.asarray(k, np.float64), G, axis=1)
+    v_rep = np.repeat(np.asarray(v, np.float64), G, axis=1)
+    dq, dk_rep, dv_rep = attention_backward(q, k_rep, v_rep, o, lse, do, causal, scale)
+    dk = dk_rep.reshape(B, Hkv, G, N, d).sum(axis=2)
+    dv = dv_rep.reshape(B, Hkv, G, N, v.shape[-1]).sum(axis=2)
+    return dq, dk, dv

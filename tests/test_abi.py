@@ -103,3 +103,37 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(fa, "LIB_PATH", "/nonexistent/libfattn.so")
     with pytest.raises(fa.FattnError):
         fa.lib()
+
+
+def fwd_gqa(**kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=4, H_kv=2, N=128, d=64, causal=0, scale=0.125,
+             stream=None)
+    a.update(kw)
+    return fa.fa_fwd_gqa(**a)
+
+
+def bwd_gqa(**kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, dO=A, dq=A, dk=A, dv=A, B=1, H=4, H_kv=2, N=128, d=64,
+             causal=0, scale=0.125, workspace=A, workspace_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return fa.fa_bwd_gqa(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(H_kv=3), fa.FA_ERR_INVALID_ARG),     # does not divide H
+    (dict(H_kv=0), fa.FA_ERR_INVALID_ARG),
+    (dict(H_kv=-2), fa.FA_ERR_INVALID_ARG),
+    (dict(H_kv=8), fa.FA_ERR_INVALID_ARG),     # more key/value heads than query heads
+    (dict(k=None), fa.FA_ERR_INVALID_ARG),
+    (dict(d=48), fa.FA_ERR_UNSUPPORTED),
+    (dict(v=A + 8), fa.FA_ERR_MISALIGNED),
+])
+def test_gqa_rejects(kw, code):
+    assert fwd_gqa(**kw) == code
+    assert fa.fa_last_error() != ""
+    assert bwd_gqa(**kw) == code
+
+
+def test_gqa_bwd_rejects_small_workspace():
+    need = fa.fa_bwd_workspace_size(1, 4, 128, 64)
+    assert bwd_gqa(workspace_bytes=need - 16) == fa.FA_ERR_WORKSPACE
