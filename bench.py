@@ -66,6 +66,9 @@ def parse_args(argv=None):
                     help="B,H,N,d,causal override (profiling runs on a smaller case)")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="key/value heads per batch (grouped-query attention; default: H)")
+    ap.add_argument("--decode", default=None,
+                    help="B,H,H_kv,Nq,Nk,d[,splits]: time the split-key forward (decoding) instead "
+                         "of the headline step; reports HBM throughput")
     args = ap.parse_args(argv)
     global WORKLOAD_NAME
     if args.shape:
@@ -409,10 +412,103 @@ def run_gpu(args):
     return 0
 
 
+DECODE_DEFAULT = "16,32,8,1,8192,128"
+
+
+def run_decode(args):
+    """Split-key forward on a decoding shape: Nq queries at the end of an Nk-key cache (causal),
+    K/V shared by groups of query heads.  HBM bound: the algorithmic bytes are the K/V cache
+    plus Q, O and L; the roofline peak is the measured copy bandwidth."""
+    import torch
+    import exact_io_aware_43_b200 as fa
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    rank, world = dist_init("nccl")
+    parts = [int(x) for x in args.decode.split(",")]
+    B, H, Hkv, Nq, Nk, d = parts[:6]
+    s = ai.default_scale(d)
+    xq = ai.make_inputs(B, H, Nq, d, seed=rank_seed(rank), with_do=False)["q"]
+    xkv = ai.make_inputs(B, Hkv, Nk, d, seed=rank_seed(rank) + 1, with_do=False)
+    to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v = to_dev(xq), to_dev(xkv["k"]), to_dev(xkv["v"])
+    splits = parts[6] if len(parts) > 6 else fa.default_splits(B, H, Nq, Nk, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(16, fa.fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, splits)),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        fa.forward_splitkv(q, k, v, True, s, splits=splits, out=o, lse=lse, workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == 0, "a kernel reported a timeout during warm-up"
+    for kk in range(5):
+        fa.fa_timer_read(kk)
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(dev)
+    torch.cuda.synchronize()
+    fa.fa_timer_enable(True)
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    fa.fa_timer_enable(False)
+    barrier(dev)
+    clocks = sampler.stop()
+    status = fa.fa_device_status()
+    ms = reduce_max(sum(a.elapsed_time(b) for a, b in ev) / args.steps, dev)
+    kt = {kk: fa.fa_timer_read(kk) for kk in (fa.FA_KERNEL_FWD, fa.FA_KERNEL_FWD_MERGE)}
+    algo_bytes = (2 * B * Hkv * Nk * d * 2) + (2 * B * H * Nq * d * 2) + 4 * B * H * Nq
+    peaks, peak_src = load_peaks()
+    value = world * algo_bytes / (ms * 1e-3) / 1e9
+    n_f, t_f = kt[fa.FA_KERNEL_FWD]
+    fwd_ms = t_f / max(1, n_f)
+    roof = {"bound": "hbm", "achieved": algo_bytes / (fwd_ms * 1e-3) / 1e9,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": algo_bytes / (fwd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "peak_source": f"{peak_src} hbm_gbs", "kernel": "fa_fwd_kernel", "launches": n_f,
+            "avg_ms": fwd_ms, "traffic": None,
+            "algorithmic_bytes": algo_bytes}
+    if rank == 0:
+        line = {
+            "metric": "split-key decode attention, HBM GB/s (K/V cache + Q, O, L bytes per step)",
+            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"decode: B={B} H={H} H_kv={Hkv} Nq={Nq} Nk={Nk} d={d} causal, "
+                                   f"{splits} key ranges", "B": B, "H": H, "H_kv": Hkv,
+                       "Nq": Nq, "Nk": Nk, "d": d, "splits": splits,
+                       "l2": "flushed before every timed step (256 MiB write, outside the events)"},
+            "kernel_ms": {"fa_fwd_kernel": fwd_ms,
+                          "fa_fwd_merge_kernel": kt[fa.FA_KERNEL_FWD_MERGE][1] /
+                          max(1, kt[fa.FA_KERNEL_FWD_MERGE][0])},
+            "roofline": roof, "clocks": clocks,
+            "gpu_launches": n_f + kt[fa.FA_KERNEL_FWD_MERGE][0], "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.decode is not None:
+        return run_decode(args)
     return run_gpu(args)
 
 

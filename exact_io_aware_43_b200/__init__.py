@@ -51,6 +51,10 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_gqa.restype = i
     L.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, sz, vp]
     L.fa_bwd_gqa.restype = i
+    L.fa_fwd_splitkv_workspace_size.argtypes = [i, i, i, i, i, i]
+    L.fa_fwd_splitkv_workspace_size.restype = sz
+    L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, sz, vp]
+    L.fa_fwd_splitkv.restype = i
     L.fa_last_error.argtypes = []
     L.fa_last_error.restype = ctypes.c_char_p
     L.fa_device_status.argtypes = [vp]
@@ -109,6 +113,16 @@ def fa_bwd_gqa(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, causal, scale,
                             float(scale), workspace, workspace_bytes, stream)
 
 
+def fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, splits) -> int:
+    return lib().fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, splits)
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, B, H, H_kv, Nq, Nk, d, causal, scale, splits, workspace,
+                   workspace_bytes, stream) -> int:
+    return lib().fa_fwd_splitkv(q, k, v, o, lse, B, H, H_kv, Nq, Nk, d, int(causal), float(scale),
+                                int(splits), workspace, workspace_bytes, stream)
+
+
 def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, stream) -> int:
     """fa_bwd with the library's static scratch instead of a caller workspace (for callers that
     cannot allocate device memory; shapes up to FA_NOALLOC_SCRATCH_BYTES of workspace)."""
@@ -127,9 +141,10 @@ def fa_version() -> int:
     return lib().fa_version()
 
 
-FA_KERNEL_FWD, FA_KERNEL_BWD_PRE, FA_KERNEL_BWD_MAIN, FA_KERNEL_BWD_POST = range(4)
+FA_KERNEL_FWD, FA_KERNEL_BWD_PRE, FA_KERNEL_BWD_MAIN, FA_KERNEL_BWD_POST, FA_KERNEL_FWD_MERGE = range(5)
 KERNEL_NAMES = {FA_KERNEL_FWD: "fa_fwd_kernel", FA_KERNEL_BWD_PRE: "fa_bwd_pre_kernel",
-                FA_KERNEL_BWD_MAIN: "fa_bwd_kernel", FA_KERNEL_BWD_POST: "fa_bwd_post_kernel"}
+                FA_KERNEL_BWD_MAIN: "fa_bwd_kernel", FA_KERNEL_BWD_POST: "fa_bwd_post_kernel",
+                FA_KERNEL_FWD_MERGE: "fa_fwd_merge_kernel"}
 
 
 def fa_timer_enable(on: bool) -> int:
@@ -230,6 +245,44 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
                         workspace.numel(), _stream_handle(q))
     _check(rc)
     return dq, dk, dv
+
+
+def default_splits(B, H, Nq, Nk, device=None) -> int:
+    """A split count that gives the forward about two work units per SM (at most one range per
+    128-key tile): the split only pays when (query blocks x heads) alone leave SMs idle."""
+    import torch
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    units = B * H * ((Nq + 255) // 256)
+    tiles = (Nk + 127) // 128
+    return max(1, min(tiles, (2 * sms + units - 1) // units))
+
+
+def forward_splitkv(q, k, v, causal: bool = False, scale: float | None = None,
+                    splits: int | None = None, out=None, lse=None, workspace=None):
+    """O, L for q [B, H, Nq, d] against k, v [B, H_kv, Nk, d] (Nq and Nk may differ; causal is
+    aligned to the end of the keys) with the keys split into ``splits`` ranges and merged."""
+    import torch
+    B, H, Nq, d = _shape(q)
+    if k.dim() != 4 or k.shape[0] != B or k.shape[3] != d or k.shape[1] < 1 or H % k.shape[1]:
+        raise ValueError("k, v must be [B, H_kv, Nk, d] with H_kv dividing q's H")
+    Hkv, Nk = int(k.shape[1]), int(k.shape[2])
+    _check_tensor(q, (B, H, Nq, d), torch.bfloat16, "q")
+    _check_tensor(k, (B, Hkv, Nk, d), torch.bfloat16, "k")
+    _check_tensor(v, (B, Hkv, Nk, d), torch.bfloat16, "v")
+    scale = _default_scale(d) if scale is None else float(scale)
+    if splits is None:
+        splits = default_splits(B, H, Nq, Nk, q.device)
+    o = torch.empty_like(q) if out is None else out
+    L = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor(o, (B, H, Nq, d), torch.bfloat16, "out")
+    _check_tensor(L, (B, H, Nq), torch.float32, "lse")
+    need = fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
+                          B, H, Hkv, Nq, Nk, d, causal, scale, splits, workspace.data_ptr(),
+                          workspace.numel(), _stream_handle(q)))
+    return o, L
 
 
 def attention(q, k, v, causal: bool = False, scale: float | None = None):

@@ -16,6 +16,7 @@
 #include "../../include/fattn.h"
 #include "bwd.cuh"
 #include "bwd_q128.cuh"
+#include "merge.cuh"
 #include "fwd.cuh"
 
 namespace {
@@ -74,7 +75,7 @@ int make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_row
 struct KernelTimer {
   std::mutex mu;
   bool on = false;
-  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev[4];
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev[5];
 };
 KernelTimer g_timer;
 
@@ -188,26 +189,28 @@ template <int D, bool CAUSAL, int NQT>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                fattn::FwdParams p, int BH, cudaStream_t st) {
   using C = fattn::FwdCfg<D, NQT>;
-  auto kern = fattn::fa_fwd_kernel<D, CAUSAL, NQT>;
+  auto kern = p.o_part != nullptr ? fattn::fa_fwd_kernel<D, CAUSAL, NQT, true>
+                                  : fattn::fa_fwd_kernel<D, CAUSAL, NQT, false>;
   int rc = set_smem(kern, C::SMEM_BYTES);
   if (rc) return rc;
   if (C::REALLOC) {
     // setmaxnreg.inc can only draw on the registers the CTA was launched with; refuse to launch
     // a build whose per-thread launch allocation is below the split the kernel asks for.
-    static int checked = 0;  // 0 unknown, 1 ok, 2 bad
-    if (checked == 0) {
+    static int checked[2] = {0, 0};  // per kernel variant: 0 unknown, 1 ok, 2 bad
+    int& chk = checked[p.o_part != nullptr];
+    if (chk == 0) {
       cudaFuncAttributes fa_attr;
       cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-      checked = (fa_attr.numRegs * C::THREADS >= C::CTRL_REGS * 128 + C::SOFTMAX_REGS * 256) ? 1 : 2;
+      chk = (fa_attr.numRegs * C::THREADS >= C::CTRL_REGS * 128 + C::SOFTMAX_REGS * 256) ? 1 : 2;
     }
-    if (checked == 2)
+    if (chk == 2)
       return fail(FA_ERR_UNSUPPORTED, "fa_fwd kernel built with too few launch registers for its "
                                       "register split");
   }
-  p.nqb = (p.N + NQT * C::BM - 1) / (NQT * C::BM);
+  p.nqb = (p.Nq + NQT * C::BM - 1) / (NQT * C::BM);
   p.BH = BH;
-  p.units = BH * p.nqb;
+  p.units = BH * p.nqb * p.splits;
   // persistent: one CTA per SM (at most one unit each when there are fewer units than SMs)
   const int G = FA_FWD_PERSISTENT ? (p.units < sm_count() ? p.units : sm_count()) : p.units;
   dim3 grid(static_cast<unsigned>(G));
@@ -289,6 +292,55 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
   return FA_OK;
 }
 
+// KV tiles of 128 keys per split and the number of non-empty splits for a requested count.
+int split_chunk(int Nk, int splits) {
+  const int tiles = (Nk + 127) / 128;
+  const int s = splits < tiles ? splits : tiles;
+  return (tiles + s - 1) / s;
+}
+int effective_splits(int Nk, int splits) {
+  if (splits < 1 || Nk < 1) return 0;
+  const int tiles = (Nk + 127) / 128;
+  const int chunk = split_chunk(Nk, splits);
+  return (tiles + chunk - 1) / chunk;
+}
+
+// Forward on Nq queries and Nk keys per head (causal: bottom-right aligned, query i sees keys
+// j <= i + Nk - Nq) with the keys cut into `splits` ranges; with more than one, partial outputs
+// go to o_part / lse_part (see FwdParams) instead of o / lse.
+int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, float* o_part,
+               float* lse_part, int B, int H, int H_kv, int Nq, int Nk, int d, bool causal,
+               float scale, int splits, cudaStream_t st) {
+  int rc;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if ((rc = make_map(&mq, q, BH, Nq, d, 128))) return rc;
+  if ((rc = make_map(&mk, k, B * H_kv, Nk, d, 128))) return rc;
+  if ((rc = make_map(&mv, v, B * H_kv, Nk, d, 128))) return rc;
+  fattn::FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.o_part = splits > 1 ? o_part : nullptr;
+  p.lse_part = splits > 1 ? lse_part : nullptr;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.off = Nk - Nq;
+  p.H = H;
+  p.G = H / H_kv;
+  p.splits = splits;
+  p.kv_chunk = split_chunk(Nk, splits);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.limit_ns = wait_limit_ns();
+  if (d == 64)
+    return causal ? launch_fwd<64, true, 2>(mq, mk, mv, p, BH, st)
+                  : launch_fwd<64, false, 2>(mq, mk, mv, p, BH, st);
+  if (d == 128)
+    return causal ? launch_fwd<128, true, 2>(mq, mk, mv, p, BH, st)
+                  : launch_fwd<128, false, 2>(mq, mk, mv, p, BH, st);
+  return causal ? launch_fwd<256, true, 1>(mq, mk, mv, p, BH, st)
+                : launch_fwd<256, false, 1>(mq, mk, mv, p, BH, st);
+}
+
 int bwd_dispatch(const void* q, const void* k, const void* v, const void* o, const float* lse,
                  const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int d,
                  bool causal, float scale, void* workspace, cudaStream_t st) {
@@ -342,28 +394,64 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return fail(FA_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
   if ((rc = check_device())) return rc;
-  const int BH = B * H;
-  CUtensorMap mq, mk, mv;
-  if ((rc = make_map(&mq, q, BH, N, d, 128))) return rc;
-  if ((rc = make_map(&mk, k, B * H_kv, N, d, 128))) return rc;
-  if ((rc = make_map(&mv, v, B * H_kv, N, d, 128))) return rc;
-  fattn::FwdParams p{};
-  p.o = static_cast<__nv_bfloat16*>(o);
-  p.lse = lse;
-  p.N = N;
-  p.H = H;
-  p.G = H / H_kv;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.limit_ns = wait_limit_ns();
+  return fwd_launch(q, k, v, o, lse, nullptr, nullptr, B, H, H_kv, N, N, d, causal != 0, scale,
+                    1, static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int Nk, int d, int splits) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || splits < 1 || (d != 64 && d != 128 && d != 256))
+    return 0;
+  const int eff = effective_splits(Nk, splits);
+  if (eff <= 1) return 0;
+  const size_t rows = size_t(B) * size_t(H) * size_t(Nq);
+  return round_up(size_t(eff) * rows * size_t(d) * 4, 256) + round_up(size_t(eff) * rows * 4, 256);
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                   int H, int H_kv, int Nq, int Nk, int d, int causal, float scale, int splits,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  g_msg[0] = 0;
+  if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID_ARG, "null tensor pointer");
+  int rc = check_common(B, H, Nq, d, scale);
+  if (rc) return rc;
+  if ((rc = check_common(B, H, Nk, d, scale))) return rc;
+  if ((rc = check_groups(H, H_kv))) return rc;
+  if (causal && Nq > Nk)
+    return fail(FA_ERR_INVALID_ARG, "causal attention needs Nq <= Nk (got Nq=%d, Nk=%d)", Nq, Nk);
+  if (splits < 1) return fail(FA_ERR_INVALID_ARG, "splits must be >= 1 (got %d)", splits);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return fail(FA_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+  const int eff = effective_splits(Nk, splits);
+  const size_t need = fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, splits);
+  if (need && (!workspace || !aligned16(workspace) || workspace_bytes < need))
+    return fail(FA_ERR_WORKSPACE, "workspace must be 16-byte aligned and >= %zu bytes", need);
+  if ((rc = check_device())) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 64)
-    return causal ? launch_fwd<64, true, 2>(mq, mk, mv, p, BH, st)
-                  : launch_fwd<64, false, 2>(mq, mk, mv, p, BH, st);
-  if (d == 128)
-    return causal ? launch_fwd<128, true, 2>(mq, mk, mv, p, BH, st)
-                  : launch_fwd<128, false, 2>(mq, mk, mv, p, BH, st);
-  return causal ? launch_fwd<256, true, 1>(mq, mk, mv, p, BH, st)
-                : launch_fwd<256, false, 1>(mq, mk, mv, p, BH, st);
+  if (eff <= 1)
+    return fwd_launch(q, k, v, o, lse, nullptr, nullptr, B, H, H_kv, Nq, Nk, d, causal != 0,
+                      scale, 1, st);
+  const long long rows = (long long)B * H * Nq;
+  float* o_part = static_cast<float*>(workspace);
+  float* lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                             round_up(size_t(eff) * rows * size_t(d) * 4, 256));
+  if ((rc = fwd_launch(q, k, v, o, lse, o_part, lse_part, B, H, H_kv, Nq, Nk, d, causal != 0,
+                       scale, eff, st)))
+    return rc;
+  const long long want = (rows + 7) / 8;
+  const int blocks = int(want < sm_count() * 16ll ? want : sm_count() * 16ll);
+  {
+    TimedLaunch tl(FA_KERNEL_FWD_MERGE, st);
+    auto* ob = static_cast<__nv_bfloat16*>(o);
+    if (d == 64)
+      fattn::fa_fwd_merge_kernel<64><<<blocks, 256, 0, st>>>(o_part, lse_part, ob, lse, eff, rows);
+    else if (d == 128)
+      fattn::fa_fwd_merge_kernel<128><<<blocks, 256, 0, st>>>(o_part, lse_part, ob, lse, eff, rows);
+    else
+      fattn::fa_fwd_merge_kernel<256><<<blocks, 256, 0, st>>>(o_part, lse_part, ob, lse, eff, rows);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_splitkv merge launch");
+  return FA_OK;
 }
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
@@ -415,7 +503,7 @@ int fa_timer_enable(int on) {
 }
 
 int fa_timer_read(int kernel, int* launches, double* total_ms) {
-  if (kernel < 0 || kernel > 3 || !launches || !total_ms)
+  if (kernel < 0 || kernel > 4 || !launches || !total_ms)
     return fail(FA_ERR_INVALID_ARG, "fa_timer_read: bad kernel kind or null output");
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> evs;
   {

@@ -50,15 +50,21 @@
 namespace fattn {
 
 struct FwdParams {
-  __nv_bfloat16* o;
-  float* lse;
-  int N;            // sequence length (queries = keys)
-  int BH;           // batch * query heads
-  int H;            // query heads per batch
-  int G;            // query heads per key/value head (grouped-query attention; 1 = one each)
-  int nqb;          // query blocks (of NQT*128 rows) per head
-  int units;        // BH * nqb
-  float scale_log2; // scale * log2(e)
+  __nv_bfloat16* o;  // [BH, Nq, D] bf16 (one split) ...
+  float* lse;        // [BH, Nq]
+  float* o_part;     // ... or, with several splits, [splits, BH, Nq, D] fp32 partial outputs
+  float* lse_part;   //     and [splits, BH, Nq] their logsumexps (natural log, -inf if empty)
+  int Nq;            // queries per head
+  int Nk;            // keys per head
+  int off;           // causal alignment: query i sees keys j <= i + off (off = Nk - Nq)
+  int BH;            // batch * query heads
+  int H;             // query heads per batch
+  int G;             // query heads per key/value head (grouped-query attention; 1 = one each)
+  int nqb;           // query blocks (of NQT*128 rows) per head
+  int splits;        // key ranges per (head, query block); 1 = the whole key sequence
+  int kv_chunk;      // KV tiles of 128 keys per split
+  int units;         // BH * nqb * splits
+  float scale_log2;  // scale * log2(e)
   uint64_t limit_ns;
 };
 
@@ -106,33 +112,46 @@ __device__ __forceinline__ int fwd_unit_of(int k, int c, int G, int units) {
   return u < units ? u : -1;
 }
 
-// Unit u -> (head, its key/value head, first query row, KV tiles per query tile).  Units are
-// numbered query block major, heaviest (latest) query blocks first when causal, heads inner, so
-// the query heads that share a key/value head run side by side and share its tiles in L2.
+// Unit u -> (head, its key/value head, split, first query row, first KV tile, KV tiles per
+// query tile).  Units are numbered query block major (heaviest, i.e. latest, query blocks first
+// when causal), then split, heads inner, so the query heads that share a key/value head run side
+// by side and share its tiles in L2.  A split covers KV tiles [kt0, kt0 + kv_chunk); a query
+// tile takes those of them that hold at least one key it may see.
 template <int NQT, bool CAUSAL>
 struct FwdUnit {
-  int head, kv_head, q0, J;
+  int head, kv_head, split, q0, kt0, J;
   int nkv[NQT];
   __device__ __forceinline__ FwdUnit(int u, const FwdParams& p) {
-    const int qi = u / p.BH;
-    head = u - qi * p.BH;
+    const int per_qb = p.BH * p.splits;
+    const int qi = u / per_qb;
+    const int rem = u - qi * per_qb;
+    split = rem / p.BH;
+    head = rem - split * p.BH;
     kv_head = (head / p.H) * (p.H / p.G) + (head % p.H) / p.G;
     const int qb = CAUSAL ? (p.nqb - 1 - qi) : qi;
     q0 = qb * NQT * 128;
-    const int n_kv_total = (p.N + 127) / 128;
+    const int n_kv_total = (p.Nk + 127) / 128;
+    kt0 = split * p.kv_chunk;
+    const int kt1 = min(n_kv_total, kt0 + p.kv_chunk);
     J = 0;
 #pragma unroll
     for (int t = 0; t < NQT; ++t) {
       const int r0 = q0 + t * 128;
       int n = 0;
-      if (r0 < p.N) n = CAUSAL ? min(n_kv_total, (r0 + 127) / 128 + 1) : n_kv_total;
+      if (r0 < p.Nq) {
+        // last key any row of the tile may see, and the KV tile holding it
+        const int last = CAUSAL ? min(p.Nk - 1, min(r0 + 127, p.Nq - 1) + p.off) : p.Nk - 1;
+        n = max(0, min(kt1, last / 128 + 1) - kt0);
+      }
       nkv[t] = n;
       J = max(J, n);
     }
   }
 };
 
-template <int D, bool CAUSAL, int NQT>
+// SPLIT: partial outputs per key range (see FwdParams); only then can a row meet a range that
+// holds no key it may see, so only then are the empty-row guards compiled in.
+template <int D, bool CAUSAL, int NQT, bool SPLIT>
 __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -203,14 +222,15 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
         int kv_it = 0;   // KV tiles loaded so far (ring position)
-        int k = 0;
+        int kq = 0;      // units with work so far (the Q barriers' phase)
         bool ok = true;
-        for (;; ++k) {
+        for (int k = 0;; ++k) {
           const int u = fwd_unit_of(k, cta, G, p.units);
           if (u < 0) break;
           const Unit un(u, p);
+          if (un.J == 0) continue;  // a key range none of its queries may see (split mode)
           // Q of this unit replaces the previous unit's once its last S MMA has completed
-          if (k > 0 && !(ok = W.wait(BAR_QE, (k - 1) & 1, 3))) break;
+          if (kq > 0 && !(ok = W.wait(BAR_QE, (kq - 1) & 1, 3))) break;
           int q_tiles = 0;
           for (int t = 0; t < NQT; ++t) q_tiles += (un.nkv[t] > 0);
           mbar_arrive_expect_tx(BAR_Q, q_tiles * C::QTILE_BYTES);
@@ -229,20 +249,21 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
             mbar_arrive_expect_tx(BAR_KF(s), C::KVTILE_BYTES);
             for (int kb = 0; kb < C::KB; ++kb)
               tma_load_3d(sbase + C::OFF_K + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmK,
-                          BAR_KF(s), kb * 64, j * C::BN, un.kv_head);
+                          BAR_KF(s), kb * 64, (un.kt0 + j) * C::BN, un.kv_head);
             if (!(ok = W.wait(BAR_VE(s), ph ^ 1, 2))) break;
             FA_TRACE_EV(21, j);
             mbar_arrive_expect_tx(BAR_VF(s), C::KVTILE_BYTES);
             for (int kb = 0; kb < C::KB; ++kb)
               tma_load_3d(sbase + C::OFF_V + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmV,
-                          BAR_VF(s), kb * 64, j * C::BN, un.kv_head);
+                          BAR_VF(s), kb * 64, (un.kt0 + j) * C::BN, un.kv_head);
           }
           if (!ok) break;
           kv_it += un.J;
+          ++kq;
         }
         if (!ok) {
           // drain (bounded): every load issued so far lands before the CTA exits
-          W.drain(BAR_Q, k & 1);
+          W.drain(BAR_Q, kq & 1);
           for (int s = 0; s < C::STAGES; ++s) {
             W.drain(BAR_KF(s), 0);
             W.drain(BAR_KF(s), 1);
@@ -272,13 +293,15 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
 #pragma unroll
         for (int t = 0; t < NQT; ++t) tit[t] = tun[t] = 0;
         bool ok = true;
+        int kq = 0;  // units with work so far (the Q barriers' phase)
         for (int k = 0; ok; ++k) {
           const int u = fwd_unit_of(k, cta, G, p.units);
           if (u < 0) break;
           const Unit un(u, p);
           const int J = un.J;
+          if (J == 0) continue;  // skipped by the producer too
           const int s0 = kv_it % C::STAGES;
-          if (!(ok = W.wait(BAR_Q, k & 1, 10))) break;
+          if (!(ok = W.wait(BAR_Q, kq & 1, 10))) break;
           if (!(ok = W.wait(BAR_KF(s0), (kv_it / C::STAGES) & 1, 11))) break;
           for (int t = 0; t < NQT && ok; ++t) {
             if (un.nkv[t] == 0) continue;
@@ -337,6 +360,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
 #pragma unroll
           for (int t = 0; t < NQT; ++t) tun[t] += (un.nkv[t] > 0);
           kv_it += J;
+          ++kq;
         }
         // every MMA issued above has completed before the tensor memory is released
         tc_commit(BAR_DRAIN);
@@ -362,8 +386,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       if (u < 0) break;
       const Unit un(u, p);
       const int n = un.nkv[t];
-      if (n == 0) continue;
       const int row = un.q0 + t * C::BM + r;  // query index
+      if (n == 0) {
+        // split mode: this tile's queries see none of the range's keys; its partials weigh 0
+        if (SPLIT && row < p.Nq)
+          p.lse_part[(size_t(un.split) * p.BH + un.head) * p.Nq + row] = -INFINITY;
+        continue;
+      }
       float m = -INFINITY;
       float l = 0.f;   // sum of the fp32 exponentials (for L)
       float lr = 0.f;  // sum of the bf16-rounded exponentials (divides O)
@@ -378,9 +407,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_wait_ld(s[c]);
         FA_TRACE_EV(15, j);
-        // mask keys past N and, on diagonal tiles, keys after the query (causal)
-        const int key0 = j * C::BN;
-        const int lim = CAUSAL ? min(row, p.N - 1) - key0 : (p.N - 1) - key0;  // last valid col
+        // mask keys past Nk and, on diagonal tiles, keys after the query's position (causal)
+        const int key0 = (un.kt0 + j) * C::BN;
+        const int lim = CAUSAL ? min(row + p.off, p.Nk - 1) - key0 : (p.Nk - 1) - key0;
         if (lim < C::BN - 1) {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
@@ -410,12 +439,15 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         const float m_tile = mx * p.scale_log2;
         const float m_use = (j == 0 || m_tile > m + kRescale) ? fmaxf(m, m_tile) : m;
         const float alpha = (j == 0 || m_use == m) ? 1.f : ex2(m - m_use);
+        // a row that has seen no key yet (possible only when a split starts past its last
+        // visible key) keeps m = -inf; its exponentials are taken against 0 and come out 0
+        const float m_ref = (SPLIT && m_use == -INFINITY) ? 0.f : m_use;
         // exact fp32 sum (for L) and the sum of the bf16-rounded weights the PV MMA uses (for
         // O's normalisation: numerator and denominator then agree, so a row dominated by one
         // key reproduces that key's V), both accumulated in paired fp32
         uint64_t sum_x[2] = {0ull, 0ull}, sum_r[2] = {0ull, 0ull};
         const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
-        const uint64_t nm2 = f2pack(-m_use, -m_use);
+        const uint64_t nm2 = f2pack(-m_ref, -m_ref);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
@@ -494,8 +526,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       // next unit's first PV once its last chunk has been read.
       if (!(ok = W.wait_warp(BAR_OD(t), (tit - 1) & 1, 22))) break;
       tc_fence_after();
-      const float inv_l = 1.f / lr;
-      __nv_bfloat16* orow = p.o + (size_t(un.head) * p.N + row) * D;
+      // a row with no visible key in this split (split mode only) gets O = 0 and L = -inf
+      const float inv_l = (!SPLIT || lr > 0.f) ? 1.f / lr : 0.f;
+      constexpr bool part = SPLIT;
+      const size_t prow = (size_t(un.split) * p.BH + un.head) * p.Nq + row;
+      __nv_bfloat16* orow = p.o + (size_t(un.head) * p.Nq + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -506,18 +541,36 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(BAR_OF(t));
         }
+        if (part) {
+          if (row < p.Nq) {
+            float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l,
+                                   __uint_as_float(o[4 * e + 1]) * inv_l,
+                                   __uint_as_float(o[4 * e + 2]) * inv_l,
+                                   __uint_as_float(o[4 * e + 3]) * inv_l);
+          }
+          continue;
+        }
         uint4 pk[4];
         uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pw[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        if (row < p.N) {
+        if (row < p.Nq) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = pk[e];
         }
       }
-      if (row < p.N) p.lse[size_t(un.head) * p.N + row] = (m + lg2(l)) * 0.69314718055994531f;
+      if (row < p.Nq) {
+        const float L = (!SPLIT || l > 0.f) ? (m + lg2(l)) * 0.69314718055994531f : -INFINITY;
+        if (part)
+          p.lse_part[prow] = L;
+        else
+          p.lse[size_t(un.head) * p.Nq + row] = L;
+      }
     }
     tc_fence_before();
   }

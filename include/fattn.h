@@ -139,6 +139,31 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
                int B, int H, int H_kv, int N, int d, int causal, float scale,
                void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Split-key forward with a logsumexp merge (decoding and other shapes with few query blocks, or
+ * queries and keys of different lengths).  The keys of each head are cut into `splits` ranges
+ * of whole 128-key tiles that run as separate work units; each writes a partial output and
+ * logsumexp, and a merge kernel combines them exactly by the associativity of the online-softmax
+ * update (robocikowo.com "Flash Attention": O <- rescale(O_prev, m_old, m_new) + ...;
+ * chipfoundryservices.com glossary "Online Softmax Trick"):  L = ln sum_s exp(L_s),
+ * O = sum_s exp(L_s - L) O_s.  The result is that of the plain definition.
+ *   q, o : bfloat16 [B, H, Nq, d]     lse : float32 [B, H, Nq]
+ *   k, v : bfloat16 [B, H_kv, Nk, d]  (H_kv divides H, as for fa_fwd_gqa)
+ * causal != 0 aligns the queries with the END of the keys: query i sees keys j <= i + Nk - Nq
+ * (the last query sees every key, as a decoding step does); it needs Nq <= Nk.
+ * splits >= 1 is the requested number of ranges; it is reduced to the number of key tiles,
+ * ceil(Nk / 128), and to the ranges that stay non-empty.  With one range nothing is merged and
+ * no workspace is needed.  Otherwise workspace is a caller-owned device buffer, 16-byte
+ * aligned, of at least fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, splits) bytes (fp32
+ * partial outputs and logsumexps); its contents on entry are ignored.  Calls that share a
+ * workspace must not overlap on the GPU.  Errors as for fa_fwd, plus FA_ERR_INVALID_ARG for
+ * splits < 1 or causal with Nq > Nk, and FA_ERR_WORKSPACE for a missing or short workspace.
+ */
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int Nk, int d, int splits);
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int H, int H_kv, int Nq, int Nk, int d, int causal, float scale,
+                   int splits, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 const char* fa_last_error(void);
 
@@ -159,9 +184,11 @@ int fa_version(void);
  * events around itself on its launching stream (host-side objects only; no device memory).
  * fa_timer_read(kernel, &launches, &total_ms) waits for the recorded events of one kernel kind,
  * returns the number of launches and their summed device time, and forgets them.
- * Kernel kinds: FA_KERNEL_FWD, FA_KERNEL_BWD_PRE, FA_KERNEL_BWD_MAIN, FA_KERNEL_BWD_POST.
+ * Kernel kinds: FA_KERNEL_FWD, FA_KERNEL_BWD_PRE, FA_KERNEL_BWD_MAIN, FA_KERNEL_BWD_POST,
+ * FA_KERNEL_FWD_MERGE (the split-key merge of fa_fwd_splitkv).
  */
-enum { FA_KERNEL_FWD = 0, FA_KERNEL_BWD_PRE = 1, FA_KERNEL_BWD_MAIN = 2, FA_KERNEL_BWD_POST = 3 };
+enum { FA_KERNEL_FWD = 0, FA_KERNEL_BWD_PRE = 1, FA_KERNEL_BWD_MAIN = 2, FA_KERNEL_BWD_POST = 3,
+       FA_KERNEL_FWD_MERGE = 4 };
 int fa_timer_enable(int on);
 int fa_timer_read(int kernel, int* launches, double* total_ms);
 

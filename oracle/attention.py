@@ -256,3 +256,36 @@ def attention_backward_gqa(q, k, v, o, lse, do, causal: bool, scale: float):
     dk = dk_rep.reshape(B, Hkv, G, N, d).sum(axis=2)
     dv = dv_rep.reshape(B, Hkv, G, N, v.shape[-1]).sum(axis=2)
     return dq, dk, dv
+
+
+def attention_forward_rect(q, k, v, causal: bool, scale: float):
+    """Attention of Nq queries against Nk keys per head: q [B,H,Nq,d], k and v [B,H_kv,Nk,d]
+    (H_kv dividing H, query head h reading key/value head h // (H // H_kv)).
+
+    The plain definition ([P2] "Problematyka standardowego mechanizmu uwagi", [P3] first
+    paragraph) for rectangular score matrices.  Causal aligns the queries with the end of the
+    keys: query i sees keys j <= i + Nk - Nq (a decoding step's last query sees every key); it
+    needs Nq <= Nk so that every query sees at least one key.  Returns (O [B,H,Nq,d], L [B,H,Nq]).
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    G = _group_size(q, k)
+    B, H, Nq, _ = q.shape
+    Nk = k.shape[2]
+    if causal and Nq > Nk:
+        raise ValueError("causal attention needs Nq <= Nk")
+    O = np.empty((B, H, Nq, v.shape[-1]))
+    L = np.empty((B, H, Nq))
+    for b in range(B):
+        for h in range(H):
+            s = scale * (q[b, h] @ k[b, h // G].T)
+            if causal:
+                hidden = np.arange(Nk)[None, :] > (np.arange(Nq)[:, None] + (Nk - Nq))
+                s = np.where(hidden, -np.inf, s)
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            l = e.sum(axis=1, keepdims=True)
+            O[b, h] = (e / l) @ v[b, h // G]
+            L[b, h] = (m + np.log(l))[:, 0]
+    return O, L

@@ -137,3 +137,49 @@ def test_gqa_rejects(kw, code):
 def test_gqa_bwd_rejects_small_workspace():
     need = fa.fa_bwd_workspace_size(1, 4, 128, 64)
     assert bwd_gqa(workspace_bytes=need - 16) == fa.FA_ERR_WORKSPACE
+
+
+def fwd_split(**kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=4, H_kv=2, Nq=4, Nk=1000, d=128, causal=1,
+             scale=0.125, splits=4, workspace=A, workspace_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return fa.fa_fwd_splitkv(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(splits=0), fa.FA_ERR_INVALID_ARG),
+    (dict(splits=-3), fa.FA_ERR_INVALID_ARG),
+    (dict(Nq=2000), fa.FA_ERR_INVALID_ARG),          # causal with more queries than keys
+    (dict(Nq=0), fa.FA_ERR_INVALID_ARG),
+    (dict(Nk=0), fa.FA_ERR_INVALID_ARG),
+    (dict(H_kv=3), fa.FA_ERR_INVALID_ARG),
+    (dict(d=80), fa.FA_ERR_UNSUPPORTED),
+    (dict(k=A + 4), fa.FA_ERR_MISALIGNED),
+    (dict(workspace=None), fa.FA_ERR_WORKSPACE),
+    (dict(workspace_bytes=64), fa.FA_ERR_WORKSPACE),
+])
+def test_splitkv_rejects(kw, code):
+    assert fwd_split(**kw) == code
+    assert fa.fa_last_error() != ""
+
+
+def test_splitkv_workspace_size():
+    # Nk = 1000 -> 8 key tiles; 4 splits of 2 tiles: 4 fp32 partial rows of d plus 4 logsumexps
+    rows = 1 * 4 * 4
+    want = -(-4 * rows * 128 * 4 // 256) * 256 + -(-4 * rows * 4 // 256) * 256
+    assert fa.fa_fwd_splitkv_workspace_size(1, 4, 4, 1000, 128, 4) == want
+    # requests beyond the tile count are reduced to it; one range needs no workspace
+    assert fa.fa_fwd_splitkv_workspace_size(1, 4, 4, 1000, 128, 100) == \
+        fa.fa_fwd_splitkv_workspace_size(1, 4, 4, 1000, 128, 8)
+    assert fa.fa_fwd_splitkv_workspace_size(1, 4, 4, 100, 128, 4) == 0
+    assert fa.fa_fwd_splitkv_workspace_size(1, 4, 4, 1000, 128, 1) == 0
+    # 3 requested ranges over 8 tiles: chunks of 3 tiles -> 3 non-empty ranges
+    assert fa.fa_fwd_splitkv_workspace_size(1, 1, 1, 1000, 64, 3) == \
+        -(-3 * 64 * 4 // 256) * 256 + 256
+    assert fa.fa_fwd_splitkv_workspace_size(0, 4, 4, 1000, 128, 4) == 0
+
+
+def test_splitkv_one_range_needs_no_workspace():
+    # a single key tile: nothing to merge, so a null workspace is fine (fails later: no device)
+    rc = fwd_split(Nk=100, Nq=4, workspace=None, workspace_bytes=0)
+    assert rc not in (fa.FA_ERR_WORKSPACE, fa.FA_ERR_INVALID_ARG)
