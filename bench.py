@@ -433,7 +433,7 @@ def run_decode(args):
     xkv = ai.make_inputs(B, Hkv, Nk, d, seed=rank_seed(rank) + 1, with_do=False)
     to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
     q, k, v = to_dev(xq), to_dev(xkv["k"]), to_dev(xkv["v"])
-    splits = parts[6] if len(parts) > 6 else fa.default_splits(B, H, Nq, Nk, dev)
+    splits = parts[6] if len(parts) > 6 else fa.default_splits(B, H, Nq, Nk, dev, Hkv)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
     ws = torch.empty(max(16, fa.fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, splits)),

@@ -57,12 +57,15 @@ EncodeTiledFn encode_fn() {
 
 // Tiled map over a contiguous bf16 [BH, N, d] tensor: box = 64 columns (128 bytes, one swizzle
 // row) x `box_rows` rows x 1 head, 128-byte swizzle, zero fill past N.
-int make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
+// bf16 [BH, N, d] map, 128-byte swizzle, box 64 columns x box_rows rows x box_heads heads (the
+// box's rows land in shared memory head-major: row g * box_rows + i).
+int make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows,
+             int box_heads = 1) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
   cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(N) * cuuint64_t(d) * 2};
-  cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
+  cuuint32_t box[3] = {64, cuuint32_t(box_rows), cuuint32_t(box_heads)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -189,15 +192,16 @@ template <int D, bool CAUSAL, int NQT>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                fattn::FwdParams p, int BH, cudaStream_t st) {
   using C = fattn::FwdCfg<D, NQT>;
-  auto kern = p.o_part != nullptr ? fattn::fa_fwd_kernel<D, CAUSAL, NQT, true>
-                                  : fattn::fa_fwd_kernel<D, CAUSAL, NQT, false>;
+  const bool general = p.o_part != nullptr || p.pack > 1;
+  auto kern = general ? fattn::fa_fwd_kernel<D, CAUSAL, NQT, true>
+                      : fattn::fa_fwd_kernel<D, CAUSAL, NQT, false>;
   int rc = set_smem(kern, C::SMEM_BYTES);
   if (rc) return rc;
   if (C::REALLOC) {
     // setmaxnreg.inc can only draw on the registers the CTA was launched with; refuse to launch
     // a build whose per-thread launch allocation is below the split the kernel asks for.
     static int checked[2] = {0, 0};  // per kernel variant: 0 unknown, 1 ok, 2 bad
-    int& chk = checked[p.o_part != nullptr];
+    int& chk = checked[general ? 1 : 0];
     if (chk == 0) {
       cudaFuncAttributes fa_attr;
       cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
@@ -208,9 +212,14 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
       return fail(FA_ERR_UNSUPPORTED, "fa_fwd kernel built with too few launch registers for its "
                                       "register split");
   }
-  p.nqb = (p.Nq + NQT * C::BM - 1) / (NQT * C::BM);
   p.BH = BH;
-  p.units = BH * p.nqb * p.splits;
+  if (p.pack > 1) {
+    p.nqb = 1;
+    p.units = (BH / p.G) * p.splits;
+  } else {
+    p.nqb = (p.Nq + NQT * C::BM - 1) / (NQT * C::BM);
+    p.units = BH * p.nqb * p.splits;
+  }
   // persistent: one CTA per SM (at most one unit each when there are fewer units than SMs)
   const int G = FA_FWD_PERSISTENT ? (p.units < sm_count() ? p.units : sm_count()) : p.units;
   dim3 grid(static_cast<unsigned>(G));
@@ -310,11 +319,13 @@ int effective_splits(int Nk, int splits) {
 // go to o_part / lse_part (see FwdParams) instead of o / lse.
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, float* o_part,
                float* lse_part, int B, int H, int H_kv, int Nq, int Nk, int d, bool causal,
-               float scale, int splits, cudaStream_t st) {
+               float scale, int splits, bool pack, cudaStream_t st) {
   int rc;
   const int BH = B * H;
+  const int G = H / H_kv;
+  pack = pack && G > 1 && G * Nq <= 128;
   CUtensorMap mq, mk, mv;
-  if ((rc = make_map(&mq, q, BH, Nq, d, 128))) return rc;
+  if ((rc = pack ? make_map(&mq, q, BH, Nq, d, Nq, G) : make_map(&mq, q, BH, Nq, d, 128))) return rc;
   if ((rc = make_map(&mk, k, B * H_kv, Nk, d, 128))) return rc;
   if ((rc = make_map(&mv, v, B * H_kv, Nk, d, 128))) return rc;
   fattn::FwdParams p{};
@@ -329,6 +340,8 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
   p.G = H / H_kv;
   p.splits = splits;
   p.kv_chunk = split_chunk(Nk, splits);
+  p.pack = pack ? G : 0;
+  p.Hkv = H_kv;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.limit_ns = wait_limit_ns();
   if (d == 64)
@@ -395,7 +408,7 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
     return fail(FA_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
   if ((rc = check_device())) return rc;
   return fwd_launch(q, k, v, o, lse, nullptr, nullptr, B, H, H_kv, N, N, d, causal != 0, scale,
-                    1, static_cast<cudaStream_t>(stream));
+                    1, false, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int Nk, int d, int splits) {
@@ -429,13 +442,13 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (eff <= 1)
     return fwd_launch(q, k, v, o, lse, nullptr, nullptr, B, H, H_kv, Nq, Nk, d, causal != 0,
-                      scale, 1, st);
+                      scale, 1, true, st);
   const long long rows = (long long)B * H * Nq;
   float* o_part = static_cast<float*>(workspace);
   float* lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                              round_up(size_t(eff) * rows * size_t(d) * 4, 256));
   if ((rc = fwd_launch(q, k, v, o, lse, o_part, lse_part, B, H, H_kv, Nq, Nk, d, causal != 0,
-                       scale, eff, st)))
+                       scale, eff, true, st)))
     return rc;
   const long long want = (rows + 7) / 8;
   const int blocks = int(want < sm_count() * 16ll ? want : sm_count() * 16ll);

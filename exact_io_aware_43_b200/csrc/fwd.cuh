@@ -62,6 +62,9 @@ struct FwdParams {
   int G;             // query heads per key/value head (grouped-query attention; 1 = one each)
   int nqb;           // query blocks (of NQT*128 rows) per head
   int splits;        // key ranges per (head, query block); 1 = the whole key sequence
+  int pack;          // > 1: the pack = G query heads of a key/value head share one query tile
+                     // (rows g * Nq + i; needs G * Nq <= 128), one unit per (K/V head, range)
+  int Hkv;           // key/value heads per batch
   int kv_chunk;      // KV tiles of 128 keys per split
   int units;         // BH * nqb * splits
   float scale_log2;  // scale * log2(e)
@@ -122,6 +125,23 @@ struct FwdUnit {
   int head, kv_head, split, q0, kt0, J;
   int nkv[NQT];
   __device__ __forceinline__ FwdUnit(int u, const FwdParams& p) {
+    const int n_kv_total = (p.Nk + 127) / 128;
+    if (p.pack > 1) {
+      // packed query heads: unit = (range, K/V head); `head` is the group's first query head
+      const int bhkv = p.BH / p.G;
+      split = u / bhkv;
+      kv_head = u - split * bhkv;
+      head = (kv_head / p.Hkv) * p.H + (kv_head % p.Hkv) * p.G;
+      q0 = 0;
+      kt0 = split * p.kv_chunk;
+      const int kt1 = min(n_kv_total, kt0 + p.kv_chunk);
+      const int last = CAUSAL ? min(p.Nk - 1, p.Nq - 1 + p.off) : p.Nk - 1;
+      nkv[0] = max(0, min(kt1, last / 128 + 1) - kt0);
+#pragma unroll
+      for (int t = 1; t < NQT; ++t) nkv[t] = 0;
+      J = nkv[0];
+      return;
+    }
     const int per_qb = p.BH * p.splits;
     const int qi = u / per_qb;
     const int rem = u - qi * per_qb;
@@ -130,7 +150,6 @@ struct FwdUnit {
     kv_head = (head / p.H) * (p.H / p.G) + (head % p.H) / p.G;
     const int qb = CAUSAL ? (p.nqb - 1 - qi) : qi;
     q0 = qb * NQT * 128;
-    const int n_kv_total = (p.Nk + 127) / 128;
     kt0 = split * p.kv_chunk;
     const int kt1 = min(n_kv_total, kt0 + p.kv_chunk);
     J = 0;
@@ -149,8 +168,9 @@ struct FwdUnit {
   }
 };
 
-// SPLIT: partial outputs per key range (see FwdParams); only then can a row meet a range that
-// holds no key it may see, so only then are the empty-row guards compiled in.
+// SPLIT: the general variant -- partial outputs per key range and packed query heads (see
+// FwdParams).  Only with ranges can a row meet one that holds no key it may see, so only this
+// variant carries the empty-row guards; plain calls use the lean one.
 template <int D, bool CAUSAL, int NQT, bool SPLIT>
 __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -231,14 +251,21 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           if (un.J == 0) continue;  // a key range none of its queries may see (split mode)
           // Q of this unit replaces the previous unit's once its last S MMA has completed
           if (kq > 0 && !(ok = W.wait(BAR_QE, (kq - 1) & 1, 3))) break;
-          int q_tiles = 0;
-          for (int t = 0; t < NQT; ++t) q_tiles += (un.nkv[t] > 0);
-          mbar_arrive_expect_tx(BAR_Q, q_tiles * C::QTILE_BYTES);
-          for (int t = 0; t < NQT; ++t) {
-            if (un.nkv[t] == 0) continue;
+          if (SPLIT && p.pack > 1) {
+            // the group's G query heads as rows g * Nq + i of tile 0: one box of Nq x G rows
+            mbar_arrive_expect_tx(BAR_Q, C::KB * p.pack * p.Nq * 128);
             for (int kb = 0; kb < C::KB; ++kb)
-              tma_load_3d(sbase + C::OFF_Q + t * C::QTILE_BYTES + kb * (C::BM * 128), &tmQ, BAR_Q,
-                          kb * 64, un.q0 + t * C::BM, un.head);
+              tma_load_3d(sbase + C::OFF_Q + kb * (C::BM * 128), &tmQ, BAR_Q, kb * 64, 0, un.head);
+          } else {
+            int q_tiles = 0;
+            for (int t = 0; t < NQT; ++t) q_tiles += (un.nkv[t] > 0);
+            mbar_arrive_expect_tx(BAR_Q, q_tiles * C::QTILE_BYTES);
+            for (int t = 0; t < NQT; ++t) {
+              if (un.nkv[t] == 0) continue;
+              for (int kb = 0; kb < C::KB; ++kb)
+                tma_load_3d(sbase + C::OFF_Q + t * C::QTILE_BYTES + kb * (C::BM * 128), &tmQ, BAR_Q,
+                            kb * 64, un.q0 + t * C::BM, un.head);
+            }
           }
           for (int j = 0; j < un.J; ++j) {
             const int g = kv_it + j;
@@ -386,11 +413,15 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       if (u < 0) break;
       const Unit un(u, p);
       const int n = un.nkv[t];
-      const int row = un.q0 + t * C::BM + r;  // query index
+      // this thread's query: index `row` of head `qh` (packed: tile row g * Nq + i)
+      const bool packed = SPLIT && p.pack > 1;
+      const int row = packed ? r % p.Nq : un.q0 + t * C::BM + r;
+      const int qh = packed ? un.head + r / p.Nq : un.head;
+      const bool valid = packed ? (t == 0 && r < p.pack * p.Nq) : row < p.Nq;
       if (n == 0) {
         // split mode: this tile's queries see none of the range's keys; its partials weigh 0
-        if (SPLIT && row < p.Nq)
-          p.lse_part[(size_t(un.split) * p.BH + un.head) * p.Nq + row] = -INFINITY;
+        if (SPLIT && valid && p.lse_part != nullptr)
+          p.lse_part[(size_t(un.split) * p.BH + qh) * p.Nq + row] = -INFINITY;
         continue;
       }
       float m = -INFINITY;
@@ -528,9 +559,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       tc_fence_after();
       // a row with no visible key in this split (split mode only) gets O = 0 and L = -inf
       const float inv_l = (!SPLIT || lr > 0.f) ? 1.f / lr : 0.f;
-      constexpr bool part = SPLIT;
-      const size_t prow = (size_t(un.split) * p.BH + un.head) * p.Nq + row;
-      __nv_bfloat16* orow = p.o + (size_t(un.head) * p.Nq + row) * D;
+      const bool part = SPLIT && p.o_part != nullptr;
+      const size_t prow = (size_t(un.split) * p.BH + qh) * p.Nq + row;
+      __nv_bfloat16* orow = p.o + (size_t(qh) * p.Nq + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -542,7 +573,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           if (lane == 0) mbar_arrive(BAR_OF(t));
         }
         if (part) {
-          if (row < p.Nq) {
+          if (valid) {
             float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D + 32 * c);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -558,18 +589,18 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pw[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        if (row < p.Nq) {
+        if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = pk[e];
         }
       }
-      if (row < p.Nq) {
+      if (valid) {
         const float L = (!SPLIT || l > 0.f) ? (m + lg2(l)) * 0.69314718055994531f : -INFINITY;
         if (part)
           p.lse_part[prow] = L;
         else
-          p.lse[size_t(un.head) * p.Nq + row] = L;
+          p.lse[size_t(qh) * p.Nq + row] = L;
       }
     }
     tc_fence_before();

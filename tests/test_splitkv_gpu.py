@@ -46,6 +46,20 @@ def test_decode_one_query(d, causal, splits):
     check(2, 4, 4, 1, 1000, d, causal, splits, seed=d + splits)
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("splits", [1, 3, 8])
+def test_decode_grouped_heads_packed(d, causal, splits):
+    """G = 4 query heads per key/value head, one query each: the group shares one query tile."""
+    check(2, 8, 2, 1, 1000, d, causal, splits, seed=40 + d + splits)
+
+
+@pytest.mark.parametrize("H,Hkv,Nq", [(16, 1, 8), (16, 1, 9), (6, 2, 5)])
+def test_packing_limits(H, Hkv, Nq):
+    """MQA with G * Nq = 128 rows exactly, one row over the limit (unpacked), and G = 3."""
+    check(1, H, Hkv, Nq, 777, 128, True, 4, seed=H + Nq)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_few_queries_grouped_heads(causal):
     check(1, 8, 2, 16, 4096, 128, causal, 8, seed=3)
