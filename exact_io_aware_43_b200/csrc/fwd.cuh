@@ -120,13 +120,13 @@ __device__ __forceinline__ int fwd_unit_of(int k, int c, int G, int units) {
 // when causal), then split, heads inner, so the query heads that share a key/value head run side
 // by side and share its tiles in L2.  A split covers KV tiles [kt0, kt0 + kv_chunk); a query
 // tile takes those of them that hold at least one key it may see.
-template <int NQT, bool CAUSAL>
+template <int NQT, bool CAUSAL, bool GENERAL>
 struct FwdUnit {
   int head, kv_head, split, q0, kt0, J;
   int nkv[NQT];
   __device__ __forceinline__ FwdUnit(int u, const FwdParams& p) {
     const int n_kv_total = (p.Nk + 127) / 128;
-    if (p.pack > 1) {
+    if (GENERAL && p.pack > 1) {
       // packed query heads: unit = (range, K/V head); `head` is the group's first query head
       const int bhkv = p.BH / p.G;
       split = u / bhkv;
@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D, NQT>;
-  using Unit = FwdUnit<NQT, CAUSAL>;
+  using Unit = FwdUnit<NQT, CAUSAL, SPLIT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
