@@ -62,6 +62,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="fattn", choices=["fattn", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-chunks", type=int, default=16,
+                    help="head chunks of fa_fwd_bwd_host in the end-to-end leg")
     ap.add_argument("--shape", default=None,
                     help="B,H,N,d,causal override (profiling runs on a smaller case)")
     ap.add_argument("--kv-heads", type=int, default=None,
@@ -356,24 +358,38 @@ def run_gpu(args):
     shares = {fa.KERNEL_NAMES[kk]: ktimes[kk][1] / max(1e-9, sum(t for _, t in ktimes.values()))
               for kk in range(4)}
 
-    # end to end through the public API: pinned host inputs -> device -> fwd+bwd -> host grads
+    # end to end through the public API: pinned host inputs -> device -> fwd+bwd -> host
+    # gradients, by fa_fwd_bwd_host (copies of one head chunk overlap the kernels of another);
+    # grouped heads have no host entry point and keep the serial copy -> step -> copy path
     e2e = None
     if args.e2e_steps > 0:
         hin = {t: host[t].pin_memory() for t in ("q", "k", "v", "do")}
         hout = [torch.empty(t.shape, dtype=torch.bfloat16).pin_memory() for t in (dq, dk, dv)]
+        grouped = W.get("H_kv", H) != H
+        chunks = max(1, min(args.e2e_chunks, B * H))
+        if not grouped:
+            hbuf = torch.empty(fa.fa_fwd_bwd_host_device_bytes(B, H, N, d, chunks),
+                               dtype=torch.uint8, device=dev)
+        st = torch.cuda.current_stream()
         e_ev = []
         torch.cuda.synchronize()
         barrier(dev)
         for i in range(args.e2e_steps + 2):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            q.copy_(hin["q"], non_blocking=True)
-            k.copy_(hin["k"], non_blocking=True)
-            v.copy_(hin["v"], non_blocking=True)
-            do.copy_(hin["do"], non_blocking=True)
-            step()
-            for hsrc, dsrc in zip(hout, (dq, dk, dv)):
-                hsrc.copy_(dsrc, non_blocking=True)
+            if grouped:
+                for t, dst in (("q", q), ("k", k), ("v", v), ("do", do)):
+                    dst.copy_(hin[t], non_blocking=True)
+                step()
+                for hsrc, dsrc in zip(hout, (dq, dk, dv)):
+                    hsrc.copy_(dsrc, non_blocking=True)
+            else:
+                rc = fa.fa_fwd_bwd_host(hin["q"].data_ptr(), hin["k"].data_ptr(),
+                                        hin["v"].data_ptr(), hin["do"].data_ptr(), None, None,
+                                        hout[0].data_ptr(), hout[1].data_ptr(),
+                                        hout[2].data_ptr(), B, H, N, d, causal, s, chunks,
+                                        hbuf.data_ptr(), hbuf.numel(), st.cuda_stream)
+                assert rc == 0, fa.fa_last_error()
             b.record()
             if i >= 2:
                 e_ev.append((a, b))
@@ -382,7 +398,9 @@ def run_gpu(args):
         h2d = sum(t.numel() * t.element_size() for t in hin.values())
         d2h = sum(t.numel() * t.element_size() for t in hout)
         e2e = {"value": world * (ff + fb) / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+               "api": "serial copies around fa_fwd_gqa / fa_bwd_gqa" if grouped else
+                      f"fa_fwd_bwd_host, {chunks} head chunks"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

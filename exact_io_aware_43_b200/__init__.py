@@ -55,6 +55,10 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_splitkv_workspace_size.restype = sz
     L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, sz, vp]
     L.fa_fwd_splitkv.restype = i
+    L.fa_fwd_bwd_host_device_bytes.argtypes = [i, i, i, i, i]
+    L.fa_fwd_bwd_host_device_bytes.restype = sz
+    L.fa_fwd_bwd_host.argtypes = [vp] * 9 + [i, i, i, i, i, f, i, vp, sz, vp]
+    L.fa_fwd_bwd_host.restype = i
     L.fa_last_error.argtypes = []
     L.fa_last_error.restype = ctypes.c_char_p
     L.fa_device_status.argtypes = [vp]
@@ -121,6 +125,16 @@ def fa_fwd_splitkv(q, k, v, o, lse, B, H, H_kv, Nq, Nk, d, causal, scale, splits
                    workspace_bytes, stream) -> int:
     return lib().fa_fwd_splitkv(q, k, v, o, lse, B, H, H_kv, Nq, Nk, d, int(causal), float(scale),
                                 int(splits), workspace, workspace_bytes, stream)
+
+
+def fa_fwd_bwd_host_device_bytes(B, H, N, d, chunks) -> int:
+    return lib().fa_fwd_bwd_host_device_bytes(B, H, N, d, chunks)
+
+
+def fa_fwd_bwd_host(q, k, v, dO, o, lse, dq, dk, dv, B, H, N, d, causal, scale, chunks,
+                    device_buffer, device_bytes, stream) -> int:
+    return lib().fa_fwd_bwd_host(q, k, v, dO, o, lse, dq, dk, dv, B, H, N, d, int(causal),
+                                 float(scale), int(chunks), device_buffer, device_bytes, stream)
 
 
 def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, stream) -> int:
@@ -291,6 +305,36 @@ def forward_splitkv(q, k, v, causal: bool = False, scale: float | None = None,
                           B, H, Hkv, Nq, Nk, d, causal, scale, splits, workspace.data_ptr(),
                           workspace.numel(), _stream_handle(q)))
     return o, L
+
+
+def forward_backward_host(q, k, v, do, causal: bool = False, scale: float | None = None,
+                          chunks: int = 4, grads=None, out=None, lse=None, device_buffer=None,
+                          stream=None):
+    """fa_fwd_bwd_host on CPU tensors (pinned for overlapped copies): returns (dq, dk, dv) as
+    CPU tensors; ``out`` / ``lse`` (CPU tensors) also receive O and L when given.  The call
+    synchronises the stream before returning."""
+    import torch
+    B, H, N, d = _shape(q)
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (do, "do")):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous() or \
+                tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{name} must be a contiguous bf16 CPU tensor of shape {(B, H, N, d)}")
+    scale = _default_scale(d) if scale is None else float(scale)
+    if grads is None:
+        grads = tuple(torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
+                      for _ in range(3))
+    need = fa_fwd_bwd_host_device_bytes(B, H, N, d, chunks)
+    if device_buffer is None:
+        device_buffer = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+    st = torch.cuda.current_stream() if stream is None else stream
+    _check(fa_fwd_bwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(),
+                           out.data_ptr() if out is not None else None,
+                           lse.data_ptr() if lse is not None else None,
+                           grads[0].data_ptr(), grads[1].data_ptr(), grads[2].data_ptr(),
+                           B, H, N, d, causal, scale, chunks, device_buffer.data_ptr(),
+                           device_buffer.numel(), st.cuda_stream))
+    st.synchronize()
+    return grads
 
 
 def attention(q, k, v, causal: bool = False, scale: float | None = None):

@@ -610,6 +610,151 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
                       static_cast<cudaStream_t>(stream));
 }
 
+// ------------------------------------------------------------------------------------------
+// fa_fwd_bwd_host: forward + backward from host buffers, copies overlapped with the kernels.
+// Heads are independent, so the B*H heads are cut into chunks of consecutive heads: chunk c's
+// inputs go up on one copy stream while chunk c-1 runs on the caller's stream and chunk c-2's
+// gradients come down on another copy stream (host->device and device->host use separate copy
+// engines).  Streams and events are host-side objects created once per device and reused.
+// ------------------------------------------------------------------------------------------
+namespace {
+
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  std::vector<cudaEvent_t> ev;  // 3 per chunk + 1
+};
+
+int host_pipe(int dev, int nev, HostPipe** out) {
+  static std::mutex mu;
+  static HostPipe pipes[128];
+  if (dev < 0 || dev >= 128) return fail(FA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> g(mu);
+  HostPipe& hp = pipes[dev];
+  cudaError_t e;
+  if (!hp.in) {
+    if ((e = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "cudaStreamCreateWithFlags");
+    if ((e = cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "cudaStreamCreateWithFlags");
+  }
+  while (int(hp.ev.size()) < nev) {
+    cudaEvent_t x;
+    if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_fail(e, "cudaEventCreateWithFlags");
+    hp.ev.push_back(x);
+  }
+  *out = &hp;
+  return FA_OK;
+}
+
+struct HostLayout {
+  size_t q, k, v, dO, o, lse, dq, dk, dv, ws, total;
+};
+
+HostLayout host_layout(int B, int H, int N, int d, int chunks) {
+  HostLayout L{};
+  const size_t bh = size_t(B) * size_t(H);
+  const size_t t = round_up(bh * size_t(N) * size_t(d) * 2, 256);
+  const int hc = int((bh + size_t(chunks) - 1) / size_t(chunks));
+  size_t off = 0;
+  for (size_t* f : {&L.q, &L.k, &L.v, &L.dO, &L.o, &L.dq, &L.dk, &L.dv}) {
+    *f = off;
+    off += t;
+  }
+  L.lse = off;
+  off += round_up(bh * size_t(N) * 4, 256);
+  L.ws = off;
+  off += round_up(fa_bwd_workspace_size(1, hc, N, d), 256);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" size_t fa_fwd_bwd_host_device_bytes(int B, int H, int N, int d, int chunks) {
+  if (B < 1 || H < 1 || N < 1 || chunks < 1 || (long long)chunks > (long long)B * H ||
+      (d != 64 && d != 128 && d != 256))
+    return 0;
+  return host_layout(B, H, N, d, chunks).total;
+}
+
+extern "C" int fa_fwd_bwd_host(const void* q, const void* k, const void* v, const void* dO,
+                               void* o, float* lse, void* dq, void* dk, void* dv, int B, int H,
+                               int N, int d, int causal, float scale, int chunks,
+                               void* device_buffer, size_t device_bytes, void* stream) {
+  g_msg[0] = 0;
+  if (!q || !k || !v || !dO || !dq || !dk || !dv)
+    return fail(FA_ERR_INVALID_ARG, "null tensor pointer");
+  int rc = check_common(B, H, N, d, scale);
+  if (rc) return rc;
+  if (chunks < 1 || (long long)chunks > (long long)B * H)
+    return fail(FA_ERR_INVALID_ARG, "chunks must be in [1, B*H] (got %d)", chunks);
+  const HostLayout L = host_layout(B, H, N, d, chunks);
+  if (!device_buffer || (reinterpret_cast<uintptr_t>(device_buffer) & 255u) ||
+      device_bytes < L.total)
+    return fail(FA_ERR_WORKSPACE, "device buffer must be 256-byte aligned and >= %zu bytes",
+                L.total);
+  if ((rc = check_device())) return rc;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  HostPipe* hp = nullptr;
+  if ((rc = host_pipe(dev, 3 * chunks + 1, &hp))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(device_buffer);
+  const long long bh = (long long)B * H;
+  const size_t head_elems = size_t(N) * size_t(d);
+  const size_t ws_bytes = round_up(fa_bwd_workspace_size(1, int((bh + chunks - 1) / chunks), N, d), 256);
+  // everything starts after the work already queued on the caller's stream
+  if ((e = cudaEventRecord(hp->ev[0], st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((e = cudaStreamWaitEvent(hp->in, hp->ev[0], 0)) != cudaSuccess)
+    return cuda_fail(e, "cudaStreamWaitEvent");
+  for (int c = 0; c < chunks; ++c) {
+    const long long h0 = bh * c / chunks, h1 = bh * (c + 1) / chunks;
+    const int hc = int(h1 - h0);
+    const size_t eoff = size_t(h0) * head_elems * 2;  // byte offset of the chunk's first head
+    const size_t ebytes = size_t(hc) * head_elems * 2;
+    cudaEvent_t ev_in = hp->ev[1 + 3 * c], ev_comp = hp->ev[2 + 3 * c], ev_out = hp->ev[3 + 3 * c];
+    const void* src[4] = {q, k, v, dO};
+    const size_t dst_off[4] = {L.q, L.k, L.v, L.dO};
+    for (int t = 0; t < 4; ++t)
+      if ((e = cudaMemcpyAsync(base + dst_off[t] + eoff, static_cast<const uint8_t*>(src[t]) + eoff,
+                               ebytes, cudaMemcpyHostToDevice, hp->in)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemcpyAsync (to device)");
+    if ((e = cudaEventRecord(ev_in, hp->in)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if ((e = cudaStreamWaitEvent(st, ev_in, 0)) != cudaSuccess)
+      return cuda_fail(e, "cudaStreamWaitEvent");
+    uint8_t* q_dev = base + L.q + eoff;
+    float* lse_c = reinterpret_cast<float*>(base + L.lse) + size_t(h0) * N;
+    if ((rc = fa_fwd(q_dev, base + L.k + eoff, base + L.v + eoff, base + L.o + eoff, lse_c, 1, hc,
+                     N, d, causal, scale, st)))
+      return rc;
+    if ((rc = fa_bwd(q_dev, base + L.k + eoff, base + L.v + eoff, base + L.o + eoff, lse_c,
+                     base + L.dO + eoff, base + L.dq + eoff, base + L.dk + eoff,
+                     base + L.dv + eoff, 1, hc, N, d, causal, scale, base + L.ws, ws_bytes, st)))
+      return rc;
+    if ((e = cudaEventRecord(ev_comp, st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if ((e = cudaStreamWaitEvent(hp->out, ev_comp, 0)) != cudaSuccess)
+      return cuda_fail(e, "cudaStreamWaitEvent");
+    void* dsts[5] = {dq, dk, dv, o, nullptr};
+    const size_t srco[4] = {L.dq, L.dk, L.dv, L.o};
+    for (int t = 0; t < 4; ++t) {
+      if (!dsts[t]) continue;  // o is optional
+      if ((e = cudaMemcpyAsync(static_cast<uint8_t*>(dsts[t]) + eoff, base + srco[t] + eoff, ebytes,
+                               cudaMemcpyDeviceToHost, hp->out)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemcpyAsync (to host)");
+    }
+    if (lse && (e = cudaMemcpyAsync(lse + size_t(h0) * N, lse_c, size_t(hc) * N * 4,
+                                    cudaMemcpyDeviceToHost, hp->out)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemcpyAsync (to host)");
+    if ((e = cudaEventRecord(ev_out, hp->out)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  }
+  // the caller's stream completes after the last copy to the host
+  if ((e = cudaStreamWaitEvent(st, hp->ev[3 * chunks], 0)) != cudaSuccess)
+    return cuda_fail(e, "cudaStreamWaitEvent");
+  return FA_OK;
+}
+
 #ifdef FA_TRACE
 // Trace build only: copy out (all per-warp slots) and clear the pipeline trace.
 extern "C" int fa_trace_read(unsigned long long* host, int max_records) {

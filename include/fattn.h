@@ -164,6 +164,32 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
                    int B, int H, int H_kv, int Nq, int Nk, int d, int causal, float scale,
                    int splits, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * fa_fwd_bwd_host -- forward and backward from HOST buffers, for callers whose tensors live in
+ * host memory.  The B*H heads are independent, so they are cut into `chunks` groups of
+ * consecutive heads: while group c runs fa_fwd + fa_bwd on `stream`, group c+1's inputs are
+ * copied to the device and group c-1's results back, on two copy streams of the library's own
+ * (host-side objects created once per device), so the PCIe transfers overlap the kernels.
+ *   q, k, v, dO      : host bfloat16 [B, H, N, d] inputs (pinned, e.g. cudaHostAlloc'd, for the
+ *                      copies to run asynchronously; pageable memory works but serialises them)
+ *   dq, dk, dv       : host bfloat16 [B, H, N, d] outputs; o (bf16) and lse (fp32 [B, H, N]) are
+ *                      optional outputs (NULL: not copied back)
+ *   device_buffer    : caller-owned device memory, 256-byte aligned, of at least
+ *                      fa_fwd_bwd_host_device_bytes(B, H, N, d, chunks) bytes (device copies of
+ *                      every tensor plus one group's backward workspace); contents unspecified
+ *   chunks           : 1 .. B*H (1: no overlap)
+ * The work starts after what is already queued on `stream` and the host outputs are complete
+ * when `stream` is; synchronise `stream` before reading them.  One head per key/value head only
+ * (no grouped heads).  Calls on one device must not overlap (they share the copy streams and
+ * events).  Errors as for fa_fwd / fa_bwd, FA_ERR_INVALID_ARG for chunks outside 1..B*H, and
+ * FA_ERR_WORKSPACE for a missing, misaligned or short device buffer.
+ */
+size_t fa_fwd_bwd_host_device_bytes(int B, int H, int N, int d, int chunks);
+int fa_fwd_bwd_host(const void* q, const void* k, const void* v, const void* dO,
+                    void* o, float* lse, void* dq, void* dk, void* dv,
+                    int B, int H, int N, int d, int causal, float scale, int chunks,
+                    void* device_buffer, size_t device_bytes, void* stream);
+
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 const char* fa_last_error(void);
 

@@ -183,3 +183,38 @@ def test_splitkv_one_range_needs_no_workspace():
     # a single key tile: nothing to merge, so a null workspace is fine (fails later: no device)
     rc = fwd_split(Nk=100, Nq=4, workspace=None, workspace_bytes=0)
     assert rc not in (fa.FA_ERR_WORKSPACE, fa.FA_ERR_INVALID_ARG)
+
+
+def host_call(**kw):
+    a = dict(q=A, k=A, v=A, dO=A, o=None, lse=None, dq=A, dk=A, dv=A, B=2, H=3, N=256, d=128,
+             causal=1, scale=0.125, chunks=2, device_buffer=1 << 30, device_bytes=1 << 40,
+             stream=None)
+    a.update(kw)
+    return fa.fa_fwd_bwd_host(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(chunks=0), fa.FA_ERR_INVALID_ARG),
+    (dict(chunks=7), fa.FA_ERR_INVALID_ARG),        # more chunks than B*H heads
+    (dict(q=None), fa.FA_ERR_INVALID_ARG),
+    (dict(dv=None), fa.FA_ERR_INVALID_ARG),
+    (dict(d=72), fa.FA_ERR_UNSUPPORTED),
+    (dict(device_buffer=None), fa.FA_ERR_WORKSPACE),
+    (dict(device_buffer=(1 << 30) + 128), fa.FA_ERR_WORKSPACE),
+    (dict(device_bytes=4096), fa.FA_ERR_WORKSPACE),
+])
+def test_host_pipeline_rejects(kw, code):
+    assert host_call(**kw) == code
+    assert fa.fa_last_error() != ""
+
+
+def test_host_pipeline_device_bytes():
+    B, H, N, d = 2, 16, 8192, 128
+    t = B * H * N * d * 2
+    one = fa.fa_fwd_bwd_host_device_bytes(B, H, N, d, 1)
+    four = fa.fa_fwd_bwd_host_device_bytes(B, H, N, d, 4)
+    # eight full-size tensors and L, plus one chunk's backward workspace
+    assert one == 8 * t + B * H * N * 4 + fa.fa_bwd_workspace_size(B, H, N, d)
+    assert four == 8 * t + B * H * N * 4 + fa.fa_bwd_workspace_size(1, 8, N, d)
+    assert fa.fa_fwd_bwd_host_device_bytes(B, H, N, d, 0) == 0
+    assert fa.fa_fwd_bwd_host_device_bytes(B, H, N, d, 33) == 0
