@@ -291,7 +291,8 @@ def run_gpu(args):
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    ws = torch.empty(fa.fa_bwd_gqa_workspace_size(B, H, W.get("H_kv", H), N, d), dtype=torch.uint8,
+                     device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def step():

@@ -47,6 +47,8 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_workspace_size.restype = sz
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
     L.fa_bwd.restype = i
+    L.fa_bwd_gqa_workspace_size.argtypes = [i, i, i, i, i]
+    L.fa_bwd_gqa_workspace_size.restype = sz
     L.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
     L.fa_fwd_gqa.restype = i
     L.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, sz, vp]
@@ -105,6 +107,10 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, workspace
            workspace_bytes, stream) -> int:
     return lib().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, int(causal), float(scale),
                         workspace, workspace_bytes, stream)
+
+
+def fa_bwd_gqa_workspace_size(B, H, H_kv, N, d) -> int:
+    return lib().fa_bwd_gqa_workspace_size(B, H, H_kv, N, d)
 
 
 def fa_fwd_gqa(q, k, v, o, lse, B, H, H_kv, N, d, causal, scale, stream) -> int:
@@ -240,7 +246,7 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
         _check_tensor(t, shp, torch.bfloat16, name)
     _check_tensor(lse, (B, H, N), torch.float32, "lse")
     scale = _default_scale(d) if scale is None else float(scale)
-    need = fa_bwd_workspace_size(B, H, N, d)
+    need = fa_bwd_gqa_workspace_size(B, H, Hkv, N, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if grads is None:

@@ -64,22 +64,53 @@ struct BwdParams {
   int Hkv;         // key/value heads per batch (H is a multiple of Hkv)
   int G;           // query heads per key/value head, H / Hkv
   int BHkv;        // batch * key/value heads (CTAs of the main kernels: BHkv x key blocks)
+  int gsplit;      // CTAs that share one (key block, key/value head), each taking gq query heads
+  int gq;          //   of the group; with gsplit > 1 they add their dK, dV into dk_acc, dv_acc
+  float* dk_acc;   // [BHkv, N, D] fp32 (scaled dK), used when gsplit > 1
+  float* dv_acc;   // [BHkv, N, D] fp32
   float scale;
   float scale_log2;
   uint64_t limit_ns;
 };
 
 // Grouped heads in the main backward kernels.  A CTA owns key block j of key/value head kvh
-// (= b * Hkv + hk) and runs nit_h query-block steps for each of the G query heads b * H + hk * G
-// + g that share it, one head after the other; dK_j and dV_j accumulate over all of them in
-// tensor memory (the gradient of a shared K/V row is the sum over the heads that read it).
+// (= b * Hkv + hk) and runs nit_h query-block steps for each of its query heads b * H + hk * G +
+// g, one head after the other; dK_j and dV_j accumulate over them in tensor memory (the gradient
+// of a shared K/V row is the sum over the heads that read it).  When (key blocks x K/V heads)
+// alone would leave SMs idle, the G heads are dealt out gq at a time to gsplit CTAs, which add
+// their sums into fp32 accumulators at the end.
 struct BwdGroup {
-  int qh0;      // first query head of the group
+  int qh0;      // first query head of this CTA
+  int nheads;   // query heads of this CTA
   int nit_h;    // query-block steps per query head
   int i_start;  // first query block
-  __device__ __forceinline__ BwdGroup(const BwdParams& p, int kvh, int i0, int nqblk)
-      : qh0((kvh / p.Hkv) * p.H + (kvh % p.Hkv) * p.G), nit_h(nqblk - i0), i_start(i0) {}
+  __device__ __forceinline__ BwdGroup(const BwdParams& p, int kvh, int gs, int i0, int nqblk)
+      : qh0((kvh / p.Hkv) * p.H + (kvh % p.Hkv) * p.G + gs * p.gq),
+        nheads(min(p.gq, p.G - gs * p.gq)), nit_h(nqblk - i0), i_start(i0) {}
 };
+
+// One 32-column chunk of a dK or dV row leaving tensor memory: bf16 straight to the output, or,
+// when the group's query heads are split over CTAs, an fp32 reduce-add into the accumulator.
+__device__ __forceinline__ void bwd_store_chunk(const uint32_t (&v)[32], float mul, bool row_ok,
+                                                __nv_bfloat16* dst, float* acc) {
+  if (!row_ok) return;
+  if (acc != nullptr) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      red_add_v4_f32(acc + 4 * e, __uint_as_float(v[4 * e]) * mul,
+                     __uint_as_float(v[4 * e + 1]) * mul, __uint_as_float(v[4 * e + 2]) * mul,
+                     __uint_as_float(v[4 * e + 3]) * mul);
+    return;
+  }
+  uint4 pkd[4];
+  uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
+#pragma unroll
+  for (int e = 0; e < 16; ++e)
+    pw[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) d4[e] = pkd[e];
+}
 // CTA -> (key block j, key/value head, d slice).  Heads are taken in bands of kBwdHeadBand; within
 // a band the key block is outermost, so the key blocks with the most query steps (causal: the
 // first ones) of the band's heads start first, while the query tiles in flight stay those of a
@@ -89,17 +120,20 @@ struct BwdGroup {
 #endif
 constexpr int kBwdHeadBand = FA_BWD_HEAD_BAND;
 struct BwdUnit {
-  int j, kvh, slice;
+  int j, kvh, gs, slice;
   __device__ __forceinline__ BwdUnit(int x, const BwdParams& p, int nsl) {
-    const int band_ctas = kBwdHeadBand * p.nkb * nsl;
+    const int per_head = nsl * p.gsplit;  // CTAs per (key block, K/V head)
+    const int band_ctas = kBwdHeadBand * p.nkb * per_head;
     const int band = x / band_ctas;
     const int h0 = band * kBwdHeadBand;
     const int nh = min(kBwdHeadBand, p.BHkv - h0);
     const int r = x - band * band_ctas;
-    j = r / (nh * nsl);
-    const int rem = r - j * (nh * nsl);
-    kvh = h0 + rem / nsl;
-    slice = rem - (rem / nsl) * nsl;
+    j = r / (nh * per_head);
+    const int rem = r - j * (nh * per_head);
+    kvh = h0 + rem / per_head;
+    const int rem2 = rem - (rem / per_head) * per_head;
+    gs = rem2 / nsl;
+    slice = rem2 - gs * nsl;
   }
 };
 
@@ -159,10 +193,20 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
       p.L2[r] = (q < p.N) ? p.lse[size_t(head) * p.N + q] * 1.4426950408889634f : INFINITY;
     }
   }
-  // zero the dQ accumulator (its size is a multiple of 4 floats: D >= 64)
+  // zero the dQ accumulator (its size is a multiple of 4 floats: D >= 64), and the dK, dV
+  // accumulators when a group's query heads are split over CTAs
   const long long n4 = (long long)p.BH * p.N * D / 4;
   float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
   for (long long i = tid; i < n4; i += nthreads) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (p.gsplit > 1) {
+    const long long m4 = (long long)p.BHkv * p.N * D / 4;
+    float4* k4 = reinterpret_cast<float4*>(p.dk_acc);
+    float4* v4 = reinterpret_cast<float4*>(p.dv_acc);
+    for (long long i = tid; i < m4; i += nthreads) {
+      k4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      v4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -254,8 +298,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const int j = unit.j, kvh = unit.kvh, slice = unit.slice;
   const int k0 = j * C::BC;
   const int nqblk = (p.N + C::BR - 1) / C::BR;
-  const BwdGroup grp(p, kvh, CAUSAL ? (k0 / C::BR) : 0, nqblk);
-  const int nit = p.G * grp.nit_h;  // >= 1
+  const BwdGroup grp(p, kvh, unit.gs, CAUSAL ? (k0 / C::BR) : 0, nqblk);
+  const int nit = grp.nheads * grp.nit_h;  // >= 1
 
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
   const uint32_t BAR_KV = bar(0);
@@ -562,21 +606,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           const uint32_t col = which == 0 ? C::T_DV : C::T_DK;
           const float mul = which == 0 ? 1.f : p.scale;
           __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + base;
+          float* acc = p.gsplit > 1 ? (which == 0 ? p.dv_acc : p.dk_acc) + base : nullptr;
 #pragma unroll
           for (int c = 0; c < C::DO / 32; ++c) {
             uint32_t v[32];
             tmem_ld32(tmem + lane_base + col + 32 * c, v);
             tmem_wait_ld(v);
-            uint4 pkd[4];
-            uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              pw[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
-            if (key_ok) {
-              uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) d4[e] = pkd[e];
-            }
+            bwd_store_chunk(v, mul, key_ok, dst + 32 * c, acc ? acc + 32 * c : nullptr);
           }
         }
       }

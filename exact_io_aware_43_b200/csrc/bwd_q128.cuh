@@ -137,8 +137,8 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
   const int j = unit.j, kvh = unit.kvh;
   const int k0 = j * C::BC;
   const int nqb = (p.N + C::BR - 1) / C::BR;
-  const BwdGroup grp(p, kvh, CAUSAL ? j : 0, nqb);
-  const int nit = p.G * grp.nit_h;  // >= 1
+  const BwdGroup grp(p, kvh, unit.gs, CAUSAL ? j : 0, nqb);
+  const int nit = grp.nheads * grp.nit_h;  // >= 1
 
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
   const uint32_t BAR_KV = bar(0);
@@ -462,21 +462,13 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
         const uint32_t col = h == 0 ? C::T_DV : C::T_DK;
         const float mul = h == 0 ? 1.f : p.scale;
         __nv_bfloat16* dst = (h == 0 ? p.dv : p.dk) + base;
+        float* acc = p.gsplit > 1 ? (h == 0 ? p.dv_acc : p.dk_acc) + base : nullptr;
 #pragma unroll
         for (int c = 0; c < C::D / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(tmem + lane_base + col + 32 * c, v);
           tmem_wait_ld(v);
-          uint4 pkd[4];
-          uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pw[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
-          if (key_ok) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) d4[e] = pkd[e];
-          }
+          bwd_store_chunk(v, mul, key_ok, dst + 32 * c, acc ? acc + 32 * c : nullptr);
         }
       }
     }

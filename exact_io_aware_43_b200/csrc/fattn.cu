@@ -275,7 +275,7 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
                                       "register split");
     if ((rc = make_map(&mq, q, p.BH, p.N, D, CQ::BR))) return rc;
     if ((rc = make_map(&mdo, p.dO, p.BH, p.N, D, CQ::BR))) return rc;
-    dim3 grid(unsigned(p.BHkv) * unsigned(p.nkb));
+    dim3 grid(unsigned(p.BHkv) * unsigned(p.nkb) * unsigned(p.gsplit));
     {
       TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
       kq<<<grid, CQ::THREADS, CQ::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, p);
@@ -283,7 +283,7 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
   } else {
     auto kern = fattn::fa_bwd_kernel<D, CAUSAL>;
     if ((rc = set_smem(kern, C::SMEM_BYTES))) return rc;
-    dim3 grid(unsigned(p.BHkv) * unsigned(p.nkb) * unsigned(C::NSL));
+    dim3 grid(unsigned(p.BHkv) * unsigned(p.nkb) * unsigned(C::NSL) * unsigned(p.gsplit));
     {
       TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
       kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, p);
@@ -295,6 +295,12 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
   {
     TimedLaunch tl(FA_KERNEL_BWD_POST, st);
     fattn::fa_bwd_post_kernel<<<grid_ew, 256, 0, st>>>(p.dq_acc, p.dq, n8);
+    if (p.gsplit > 1) {
+      // the group's dK, dV sums were reduced in fp32
+      const long long m8 = (long long)p.BHkv * p.N * D / 8;
+      fattn::fa_bwd_post_kernel<<<grid_ew, 256, 0, st>>>(p.dk_acc, p.dk, m8);
+      fattn::fa_bwd_post_kernel<<<grid_ew, 256, 0, st>>>(p.dv_acc, p.dv, m8);
+    }
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fa_bwd postprocess launch");
@@ -380,6 +386,32 @@ int bwd_dispatch(const void* q, const void* k, const void* v, const void* o, con
   p.Hkv = Hkv;
   p.G = H / Hkv;
   p.BHkv = B * Hkv;
+  // grouped heads: when (key blocks x K/V heads) would leave SMs idle, deal each group's query
+  // heads out to several CTAs, which reduce their dK, dV sums in fp32 (the workspace of
+  // fa_bwd_gqa_workspace_size holds the two accumulators after the row vectors)
+  p.gsplit = 1;
+  p.gq = p.G;
+  static const int gsplit_cap = [] {  // FA_BWD_GSPLIT caps the split (1: off), for comparisons
+    const char* e = getenv("FA_BWD_GSPLIT");
+    const int x = e ? atoi(e) : 0;
+    return x > 0 ? x : 1 << 30;
+  }();
+  if (p.G > 1 && gsplit_cap > 1) {
+    const long long ctas = (long long)p.BHkv * p.nkb * (d == 256 ? 2 : 1);
+    const long long target = 2ll * sm_count();
+    if (ctas < target) {
+      const int want = int((target + ctas - 1) / ctas);
+      int gs = want < p.G ? want : p.G;
+      if (gs > gsplit_cap) gs = gsplit_cap;
+      p.gq = (p.G + gs - 1) / gs;
+      p.gsplit = (p.G + p.gq - 1) / p.gq;
+    }
+  }
+  if (p.gsplit > 1) {
+    const size_t kv_bytes = round_up(size_t(p.BHkv) * size_t(N) * size_t(d) * 4, 256);
+    p.dk_acc = reinterpret_cast<float*>(ws + dq_bytes + 2 * row_bytes);
+    p.dv_acc = reinterpret_cast<float*>(ws + dq_bytes + 2 * row_bytes + kv_bytes);
+  }
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.limit_ns = wait_limit_ns();
@@ -481,6 +513,13 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return dq + 2 * rows;
 }
 
+size_t fa_bwd_gqa_workspace_size(int B, int H, int H_kv, int N, int d) {
+  const size_t base = fa_bwd_workspace_size(B, H, N, d);
+  if (!base || H_kv < 1 || H_kv > H || H % H_kv) return 0;
+  if (H_kv == H) return base;
+  return base + 2 * round_up(size_t(B) * size_t(H_kv) * size_t(N) * size_t(d) * 4, 256);
+}
+
 int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
                const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
                int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
@@ -494,7 +533,7 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
                           static_cast<const void*>(dq), static_cast<const void*>(dk),
                           static_cast<const void*>(dv)})
     if (!aligned16(ptr)) return fail(FA_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
-  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  const size_t need = fa_bwd_gqa_workspace_size(B, H, H_kv, N, d);
   if (!workspace || !aligned16(workspace) || workspace_bytes < need)
     return fail(FA_ERR_WORKSPACE, "workspace must be 16-byte aligned and >= %zu bytes", need);
   if ((rc = check_device())) return rc;

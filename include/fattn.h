@@ -127,11 +127,15 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
  *   q, o, dO, dq : bfloat16 [B, H, N, d]        lse : float32 [B, H, N]
  *   k, v, dk, dv : bfloat16 [B, H_kv, N, d]
  * dk and dv hold the gradient summed over the H / H_kv query heads that read each key/value
- * head.  H_kv must divide H (else FA_ERR_INVALID_ARG).  The workspace is the one
- * fa_bwd_workspace_size(B, H, N, d) gives (it depends on the query heads only).  Every other
- * convention -- alignment, ownership, streams, errors -- is that of fa_fwd / fa_bwd, which are
- * these calls with H_kv = H.
+ * head.  H_kv must divide H (else FA_ERR_INVALID_ARG).  The backward's workspace is
+ * fa_bwd_gqa_workspace_size(B, H, H_kv, N, d) bytes: fa_bwd_workspace_size's, plus, when H_kv < H,
+ * two fp32 [B, H_kv, N, d] accumulators.  They are used when there are too few (key block,
+ * key/value head) pairs to fill the GPU: a group's query heads are then dealt out to several
+ * CTAs whose dK, dV sums meet in fp32 (so dk and dv are not bitwise reproducible run to run in
+ * that case).  Every other convention -- alignment, ownership, streams, errors -- is that of
+ * fa_fwd / fa_bwd, which are these calls with H_kv = H.
  */
+size_t fa_bwd_gqa_workspace_size(int B, int H, int H_kv, int N, int d);
 int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
                int B, int H, int H_kv, int N, int d, int causal, float scale, void* stream);
 int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,

@@ -135,8 +135,19 @@ def test_gqa_rejects(kw, code):
 
 
 def test_gqa_bwd_rejects_small_workspace():
-    need = fa.fa_bwd_workspace_size(1, 4, 128, 64)
+    need = fa.fa_bwd_gqa_workspace_size(1, 4, 2, 128, 64)
     assert bwd_gqa(workspace_bytes=need - 16) == fa.FA_ERR_WORKSPACE
+    # the plain backward's workspace lacks the two fp32 dK, dV accumulators
+    assert bwd_gqa(workspace_bytes=fa.fa_bwd_workspace_size(1, 4, 128, 64)) == fa.FA_ERR_WORKSPACE
+
+
+def test_gqa_workspace_size():
+    base = fa.fa_bwd_workspace_size(2, 8, 1000, 128)
+    assert fa.fa_bwd_gqa_workspace_size(2, 8, 8, 1000, 128) == base
+    acc = -(-2 * 2 * 1000 * 128 * 4 // 256) * 256
+    assert fa.fa_bwd_gqa_workspace_size(2, 8, 2, 1000, 128) == base + 2 * acc
+    assert fa.fa_bwd_gqa_workspace_size(2, 8, 3, 1000, 128) == 0
+    assert fa.fa_bwd_gqa_workspace_size(2, 8, 0, 1000, 128) == 0
 
 
 def fwd_split(**kw):
