@@ -46,6 +46,12 @@
 #ifndef FA_FWD_MAX3
 #define FA_FWD_MAX3 0
 #endif
+// FA_FWD_ONES_SUM: at d = 64 (where tensor memory has room) the PV MMA also multiplies P~ by a
+// block of ones appended to V, so 16 extra O columns carry the sum of the bf16-rounded weights --
+// rescaled with O, and no longer summed by the softmax threads.
+#ifndef FA_FWD_ONES_SUM
+#define FA_FWD_ONES_SUM 1
+#endif
 
 namespace fattn {
 
@@ -91,22 +97,26 @@ struct FwdCfg {
   static constexpr int SOFTMAX_REGS = 200;
   static_assert(!REALLOC || CTRL_REGS * 128 + SOFTMAX_REGS * 256 <= LAUNCH_REGS * THREADS,
                 "register split exceeds the launch allocation");
+  // ones-column row sums (FA_FWD_ONES_SUM): O_t gets EXTRA more columns, V a ones block
+  static constexpr int EXTRA = (D == 64 && FA_FWD_ONES_SUM) ? 16 : 0;
+  static constexpr int OCOLS = D + EXTRA;
   static constexpr int TMEM_S = 0;               // S_t at column t*BN (P_t aliases its first BN/2)
-  static constexpr int TMEM_O = NQT * BN;        // O_t at TMEM_O + t*D
+  static constexpr int TMEM_O = NQT * BN;        // O_t at TMEM_O + t*OCOLS
   static constexpr int TMEM_COLS = 512;
-  static_assert(NQT * (BN + D) <= TMEM_COLS, "tensor memory budget");
+  static_assert(NQT * (BN + OCOLS) <= TMEM_COLS, "tensor memory budget");
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQT * QTILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KVTILE_BYTES;
-  static constexpr int OFF_BAR = OFF_V + STAGES * KVTILE_BYTES;
+  static constexpr int OFF_ONES = OFF_V + STAGES * KVTILE_BYTES;  // [BN keys][64] bf16 ones
+  static constexpr int OFF_BAR = OFF_ONES + (EXTRA ? BN * 128 : 0);
   // barriers: q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT],
   //           p_full[NQT], o_done[NQT], o_free[NQT], drain
   static constexpr int NBAR = 2 + 4 * STAGES + 4 * NQT + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem address + abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);   // Q, K both K-major
-  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);   // P (tmem), V MN-major
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, OCOLS, 0, 1);  // P (tmem), V MN-major
 };
 
 // The k-th unit of CTA c among G CTAs (zig-zag over rounds of G units), or -1 when none is left.
@@ -226,6 +236,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
     tc_fence_before();
+  }
+  if constexpr (C::EXTRA > 0) {
+    // the ones block V is extended with (every bf16 of it 1.0, so its swizzle does not matter)
+    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + C::OFF_ONES);
+    for (int i = threadIdx.x; i < C::BN * 128 / 4; i += C::THREADS) ones[i] = 0x3F803F80u;
+    fence_async_smem();
   }
   __syncthreads();
   tc_fence_after();
@@ -360,8 +376,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
               for (int kk = 0; kk < C::BN / 16; ++kk) {
                 // P~ is packed bf16: 16 keys = 8 columns; V rows (keys) are 128 B apart, so a
                 // 16-key slice is 2048 B further on; 64-wide d blocks are BN*128 B apart.
-                mma_ts(tmem + C::TMEM_O + t * D, tmem + C::TMEM_S + t * C::BN + kk * 8,
-                       sdesc_sw128(v_addr + kk * 2048, C::BN * 128, 1024), C::IDESC_PV,
+                // with EXTRA, the second 64-wide N block of B is the ones tile, LBO bytes on
+                mma_ts(tmem + C::TMEM_O + t * C::OCOLS, tmem + C::TMEM_S + t * C::BN + kk * 8,
+                       sdesc_sw128(v_addr + kk * 2048,
+                                   C::EXTRA ? uint32_t(C::OFF_ONES - C::OFF_V - s * C::KVTILE_BYTES)
+                                            : uint32_t(C::BN * 128),
+                                   1024),
+                       C::IDESC_PV,
                        (j > 0 || kk > 0) ? 1u : 0u);
               }
               tc_commit(BAR_OD(t));
@@ -401,7 +422,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     const int r = threadIdx.x & 127;          // row within the tile == TMEM lane
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + C::TMEM_S + t * C::BN;
-    const uint32_t tO = tmem + lane_base + C::TMEM_O + t * D;
+    const uint32_t tO = tmem + lane_base + C::TMEM_O + t * C::OCOLS;
     // m: reference max (log2 units of the scaled scores) that the exponentials and l are taken
     // against.  It only moves when a row's max grows by more than kRescale (2^8 in value): the
     // result is the same exact softmax, P~ stays <= 256, and O is rescaled far less often.
@@ -499,10 +520,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
             pk[e] = pack_bf16(p0, p1);
             sum_x[e & 1] = fadd2(sum_x[e & 1], f2pack(p0, p1));
 #if FA_FWD_RSUM == 1
-            sum_r[e & 1] = fadd2(sum_r[e & 1], f2pack(__uint_as_float(pk[e] << 16),
-                                                     __uint_as_float(pk[e] & 0xffff0000u)));
+            if (C::EXTRA == 0)
+              sum_r[e & 1] = fadd2(sum_r[e & 1], f2pack(__uint_as_float(pk[e] << 16),
+                                                       __uint_as_float(pk[e] & 0xffff0000u)));
 #elif FA_FWD_RSUM == 2
-            {
+            if (C::EXTRA == 0) {
               float r0, r1;
               f2unpack(sum_r[e & 1], r0, r1);
               add_bf16pair_f32(pk[e], r0, r1);
@@ -528,7 +550,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           f2unpack(fadd2(sum_x[0], sum_x[1]), a0, a1);
           f2unpack(fadd2(sum_r[0], sum_r[1]), b0, b1);
           l = l * alpha + (a0 + a1);
-          lr = (FA_FWD_RSUM == 0) ? l : lr * alpha + (b0 + b1);
+          if (C::EXTRA == 0) lr = (FA_FWD_RSUM == 0) ? l : lr * alpha + (b0 + b1);
         }
         m = m_use;
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -545,6 +567,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
             tmem_st32(tO + 32 * c, o);
           }
+          if constexpr (C::EXTRA > 0) {  // the row sums of the rounded weights, with O
+            uint32_t o[16];
+            tmem_ld16(tO + D, o);
+            tmem_wait_ld16(o);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(tO + D, o);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -558,6 +588,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       if (!(ok = W.wait_warp(BAR_OD(t), (tit - 1) & 1, 22))) break;
       tc_fence_after();
       // a row with no visible key in this split (split mode only) gets O = 0 and L = -inf
+      if constexpr (C::EXTRA > 0) {  // the MMA's row sum of the rounded weights
+        uint32_t o[16];
+        tmem_ld16(tO + D, o);
+        tmem_wait_ld16(o);
+        lr = __uint_as_float(o[0]);
+      }
       const float inv_l = (!SPLIT || lr > 0.f) ? 1.f / lr : 0.f;
       const bool part = SPLIT && p.o_part != nullptr;
       const size_t prow = (size_t(un.split) * p.BH + qh) * p.Nq + row;
