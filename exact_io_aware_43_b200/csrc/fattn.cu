@@ -4,7 +4,6 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -201,16 +200,15 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   if (C::REALLOC) {
     // setmaxnreg.inc can only draw on the registers the CTA was launched with; refuse to launch
     // a build whose per-thread launch allocation is below the split the kernel asks for.
-    static std::atomic<int> checked[2] = {{0}, {0}};  // per variant: 0 unknown, 1 ok, 2 bad
-    std::atomic<int>& chk = checked[general ? 1 : 0];
-    if (chk.load() == 0) {
+    static int checked[2] = {0, 0};  // per kernel variant: 0 unknown, 1 ok, 2 bad
+    int& chk = checked[general ? 1 : 0];
+    if (chk == 0) {
       cudaFuncAttributes fa_attr;
       cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-      chk.store((fa_attr.numRegs * C::THREADS >= C::CTRL_REGS * 128 + C::SOFTMAX_REGS * 256) ? 1
-                                                                                              : 2);
+      chk = (fa_attr.numRegs * C::THREADS >= C::CTRL_REGS * 128 + C::SOFTMAX_REGS * 256) ? 1 : 2;
     }
-    if (chk.load() == 2)
+    if (chk == 2)
       return fail(FA_ERR_UNSUPPORTED, "fa_fwd kernel built with too few launch registers for its "
                                       "register split");
   }
@@ -264,8 +262,8 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
     if ((rc = set_smem(kq, CQ::SMEM_BYTES))) return rc;
     // setmaxnreg.inc draws on the registers the CTA was launched with: refuse a build whose
     // launch allocation is below the kernel's register split
-    static std::atomic<int> checked{0};  // 0 unknown, 1 ok, 2 bad
-    if (checked.load() == 0) {
+    static int checked = 0;  // 0 unknown, 1 ok, 2 bad
+    if (checked == 0) {
       cudaFuncAttributes fa_attr;
       e = cudaFuncGetAttributes(&fa_attr, kq);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
