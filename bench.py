@@ -265,13 +265,25 @@ def kernel_traffic(kernel_name: str):
         return None
     if not rec:
         return None
-    src = hashlib.sha256()
-    for fn in sorted(os.listdir(os.path.join(ROOT, "exact_io_aware_43_b200", "csrc"))):
-        with open(os.path.join(ROOT, "exact_io_aware_43_b200", "csrc", fn), "rb") as f:
-            src.update(f.read())
-    if rec.get("csrc_sha256") != src.hexdigest():
+    if rec.get("csrc_sha256") != csrc_code_hash():
         return None
     return rec.get("bytes_per_launch")
+
+
+def csrc_code_hash() -> str:
+    """sha256 of the CUDA sources with comments removed and whitespace collapsed: a traffic
+    record stays valid across comment edits and goes stale with any change to the code."""
+    import re
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "exact_io_aware_43_b200", "csrc")
+    for fn in sorted(os.listdir(d)):
+        with open(os.path.join(d, fn), encoding="utf-8") as f:
+            txt = f.read()
+        txt = re.sub(r"/\*.*?\*/", " ", txt, flags=re.S)
+        txt = re.sub(r"//[^\n]*", " ", txt)
+        txt = " ".join(txt.split())
+        h.update(fn.encode() + b"\0" + txt.encode() + b"\0")
+    return h.hexdigest()
 
 
 def run_gpu(args):
