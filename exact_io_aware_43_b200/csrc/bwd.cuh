@@ -1,11 +1,14 @@
 // bwd.cuh -- attention backward for sm_100a, by recomputation (robocikowo.com "Flash Attention":
 // the backward recomputes the attention matrix from the saved O and L instead of storing it).
 //
-// Three kernels on the caller's stream:
+// Three kernels on the caller's stream (the main kernel for d = 128 is fa_bwd_kernel_q128, in
+// bwd_q128.cuh, with 128-query steps; this file's fa_bwd_kernel serves d = 64 and d = 256):
 //   fa_bwd_pre_kernel   D_i = sum_c dO_ic O_ic, L2_i = L_i log2(e) (padded rows: +inf, 0),
-//                       and zeroes the fp32 dQ accumulator.                         (HBM bound)
-//   fa_bwd_kernel       one CTA per (head, block of 128 keys [, 128-wide slice of d]): K_j, V_j
-//                       stay in shared memory while the CTA loops over 64-query blocks i:
+//                       and zeroes the fp32 dQ accumulator (and the dK, dV accumulators when
+//                       a group's query heads are split over CTAs).                  (HBM bound)
+//   fa_bwd_kernel       one CTA per (block of 128 keys, key/value head [, 128-wide slice of d]
+//                       [, share of the group's query heads]): K_j, V_j stay in shared memory
+//                       while the CTA loops over 64-query blocks i of each of its query heads:
 //                         S^T  = K_j Q_i^T               tcgen05.mma -> TMEM (keys on lanes)
 //                         P^T  = exp2(S^T s log2e - L2_i)   recomputed from L
 //                         dV  += P^T dO_i                A = P^T (bf16, TMEM)
@@ -14,12 +17,13 @@
 //                         dK  += dS^T Q_i                A = dS^T (bf16, TMEM)
 //                         dQ_i^T += K_j^T dS^T           -> fp32 reduction into the accumulator
 //                       dK is scaled by s in the epilogue, dQ when it is reduced.
-//   fa_bwd_post_kernel  dq = bf16(dQ accumulator).
+//   fa_bwd_post_kernel  dq = bf16(dQ accumulator) (and dk, dv from their accumulators).
 // No N x N buffer exists: the score and probability tiles live in tensor memory.
 //
-// Warp roles of fa_bwd_kernel: warps 0-3 compute P and dS (thread = key row = TMEM lane),
-// warps 4-7 drain dQ^T from tensor memory into the accumulator, warp 8 issues TMA loads,
-// warp 9 allocates tensor memory and issues the MMAs.
+// Warp roles of fa_bwd_kernel (FA_BWD_SPLIT, the default): warps 0-7 compute P and dS, two
+// warpgroups of 32 query columns each (thread = key row = TMEM lane); warps 8-11 drain dQ^T from
+// tensor memory into the accumulator; warp 12 issues TMA loads; warp 13 allocates tensor memory
+// and issues the MMAs.  With FA_BWD_SPLIT=0: one P/dS warpgroup, drain warps 4-7, warps 8, 9.
 #pragma once
 
 #include "sm100.cuh"

@@ -1,6 +1,8 @@
 // fattn.cu -- host side of libfattn: argument checks, TMA descriptors, launches (C ABI in
-// include/fattn.h).  Every step of the attention computation runs in the kernels of fwd.cuh and
-// bwd.cuh; this file only validates, encodes descriptors and launches.
+// include/fattn.h).  Every step of the attention computation runs in the kernels of fwd.cuh,
+// bwd.cuh, bwd_q128.cuh and merge.cuh; this file validates, encodes descriptors, picks the
+// schedule (units, key ranges, head groups) and launches, and for fa_fwd_bwd_host orders the
+// copies of head chunks around the kernels on its copy streams.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

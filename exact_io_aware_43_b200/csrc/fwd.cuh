@@ -1,7 +1,8 @@
 // fwd.cuh -- fused attention forward for sm_100a.
 //
-// A work unit is NQT query tiles of 128 rows of one (batch, head).  For each unit the CTA streams
-// every K_j, V_j tile of 128 keys through a shared-memory ring (chipfoundryservices.com glossary
+// A work unit is NQT query tiles of 128 rows of one (batch, head) -- or, in the general variant,
+// a range of the keys for them, or the packed query heads of one key/value head (see FwdUnit).
+// For each unit the CTA streams its K_j, V_j tiles of 128 keys through a shared-memory ring (chipfoundryservices.com glossary
 // "Flash Attention", "Tiling Algorithm" steps 1-2; robocikowo.com "Flash Attention": a Q block
 // is loaded once, then the loop runs over the K, V blocks).  Per KV tile and query tile:
 //   S   = Q_t K_j^T                  tcgen05.mma, bf16 x bf16 -> fp32 in tensor memory (step 3)
