@@ -107,3 +107,17 @@ MUTANTS = [
 @pytest.mark.parametrize("name,fwd", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_rect_planted_mistake_is_caught(name, fwd):
     assert any(p(fwd) for p in PINS), f"planted mistake {name} passed every pin"
+
+
+def test_rect_agrees_with_grouped_oracle_on_square_shapes():
+    """Where both apply (Nq = Nk, grouped heads) the rectangular and the grouped oracle -- pinned
+    separately -- must give the same result."""
+    from oracle import attention_forward_gqa
+    for (H, Hkv, N, d, seed) in ((4, 2, 7, 3, 70), (6, 1, 5, 4, 71), (3, 3, 9, 2, 72)):
+        q = rand((2, H, N, d), seed)
+        k = rand((2, Hkv, N, d), seed + 1)
+        v = rand((2, Hkv, N, d), seed + 2)
+        for causal in (False, True):
+            O1, L1 = attention_forward_rect(q, k, v, causal, 0.7)
+            O2, L2 = attention_forward_gqa(q, k, v, causal, 0.7)
+            assert np.allclose(O1, O2, atol=1e-12) and np.allclose(L1, L2, atol=1e-12)
