@@ -58,3 +58,22 @@ def test_flop_count_matches_metric_definition():
     assert ff == 4 * 2 * 16 * 8192 ** 2 * 128 / 2
     assert fb == 2.5 * ff
     assert bench.flops(1, 1, 10, 64, False)[0] == 4 * 100 * 64
+
+
+def test_reference_arm_under_two_ranks():
+    """`bench.py --impl reference` under torchrun: rank 0 times the oracle and prints one JSON
+    line with impl == "reference"; the other rank exits 0 without work."""
+    import json
+    import subprocess
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr=127.0.0.1", f"--master-port={port}",
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "1",
+           "--warmup", "0"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["value"] > 0
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
