@@ -18,6 +18,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB_DIR = os.path.join(HERE, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libfattn.so")
+# Test-only variant: the forward's producer leaves one K/V tile unissued (FA_TEST_STARVE) and the
+# waits are bounded at 1 ms, so a test can watch a bounded wait run out and the kernel report
+# FA_ERR_TIMEOUT without any fault or hang.  The product path never loads it.
+STARVE_PATH = os.path.join(LIB_DIR, "libfattn_starve.so")
+STARVE_DEFINES = ["-DFA_TEST_STARVE", "-DFA_DEFAULT_WAIT_LIMIT_NS=1000000ull"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 NVCC_FLAGS = [
@@ -41,19 +46,16 @@ def sources():
                   glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB_PATH):
+def up_to_date(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return False
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB_PATH
-    os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB_PATH + ".tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, "-o", tmp, os.path.join(CSRC, "fattn.cu")]
+def _compile(out: str, defines, verbose: bool) -> None:
+    tmp = out + ".tmp"
+    cmd = [nvcc(), *NVCC_FLAGS, *defines, "-o", tmp, os.path.join(CSRC, "fattn.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
@@ -62,9 +64,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
     if verbose:
         print(r.stdout + r.stderr)
-    os.replace(tmp, LIB_PATH)
+    os.replace(tmp, out)
+
+
+def build(force: bool = False, verbose: bool = False, starve: bool = True) -> str:
+    """Build libfattn.so (and, unless starve=False, the test-only libfattn_starve.so)."""
+    os.makedirs(LIB_DIR, exist_ok=True)
+    if force or not up_to_date(LIB_PATH):
+        _compile(LIB_PATH, [], verbose)
+    if starve and (force or not up_to_date(STARVE_PATH)):
+        _compile(STARVE_PATH, STARVE_DEFINES, False)
     return LIB_PATH
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                starve="--no-starve" not in sys.argv))

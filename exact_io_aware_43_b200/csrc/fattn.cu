@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -120,11 +121,17 @@ int make_map_f32(CUtensorMap* m, void* base, int BH, int N, int d) {
   return FA_OK;
 }
 
+// Default bound of every wait inside the kernels: 2 s, far above any legitimate wait.  The test
+// build that starves a wait on purpose compiles in a 1 ms default instead.
+#ifndef FA_DEFAULT_WAIT_LIMIT_NS
+#define FA_DEFAULT_WAIT_LIMIT_NS 2000000000ull
+#endif
+
 uint64_t wait_limit_ns() {
   static uint64_t v = [] {
     const char* e = getenv("FA_WAIT_LIMIT_NS");
     uint64_t x = e ? strtoull(e, nullptr, 10) : 0;
-    return x ? x : uint64_t(2000000000ull);  // 2 s: far above any legitimate wait
+    return x ? x : uint64_t(FA_DEFAULT_WAIT_LIMIT_NS);
   }();
   return v;
 }
@@ -202,13 +209,16 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   if (C::REALLOC) {
     // setmaxnreg.inc can only draw on the registers the CTA was launched with; refuse to launch
     // a build whose per-thread launch allocation is below the split the kernel asks for.
-    static int checked[2] = {0, 0};  // per kernel variant: 0 unknown, 1 ok, 2 bad
-    int& chk = checked[general ? 1 : 0];
+    // per kernel variant: 0 unknown, 1 ok, 2 bad; threads that race here compute the same value
+    static std::atomic<int> checked[2] = {{0}, {0}};
+    std::atomic<int>& chk_slot = checked[general ? 1 : 0];
+    int chk = chk_slot.load(std::memory_order_relaxed);
     if (chk == 0) {
       cudaFuncAttributes fa_attr;
       cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
       chk = (fa_attr.numRegs * C::THREADS >= C::CTRL_REGS * 128 + C::SOFTMAX_REGS * 256) ? 1 : 2;
+      chk_slot.store(chk, std::memory_order_relaxed);
     }
     if (chk == 2)
       return fail(FA_ERR_UNSUPPORTED, "fa_fwd kernel built with too few launch registers for its "
@@ -264,15 +274,17 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
     if ((rc = set_smem(kq, CQ::SMEM_BYTES))) return rc;
     // setmaxnreg.inc draws on the registers the CTA was launched with: refuse a build whose
     // launch allocation is below the kernel's register split
-    static int checked = 0;  // 0 unknown, 1 ok, 2 bad
-    if (checked == 0) {
+    static std::atomic<int> checked{0};  // 0 unknown, 1 ok, 2 bad
+    int chk = checked.load(std::memory_order_relaxed);
+    if (chk == 0) {
       cudaFuncAttributes fa_attr;
       e = cudaFuncGetAttributes(&fa_attr, kq);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-      checked = (fa_attr.numRegs * CQ::THREADS >=
-                 CQ::CMP_REGS * 256 + CQ::DQ_REGS * 128 + CQ::CTRL_REGS * 128) ? 1 : 2;
+      chk = (fa_attr.numRegs * CQ::THREADS >=
+             CQ::CMP_REGS * 256 + CQ::DQ_REGS * 128 + CQ::CTRL_REGS * 128) ? 1 : 2;
+      checked.store(chk, std::memory_order_relaxed);
     }
-    if (checked == 2)
+    if (chk == 2)
       return fail(FA_ERR_UNSUPPORTED, "fa_bwd kernel built with too few launch registers for its "
                                       "register split");
     if ((rc = make_map(&mq, q, p.BH, p.N, D, CQ::BR))) return rc;

@@ -29,15 +29,11 @@
 #include "sm100.cuh"
 
 // Tuning knobs (compile time), each chosen by measurement on the long-context workload.
-// FA_FWD_POLY_EVERY: one pair of exponentials in N goes through the FMA-pipe polynomial instead of
-// MUFU (0: none).  FA_FWD_RSUM: how O's normaliser is formed -- 0: the fp32 sum (also used for
+// FA_FWD_RSUM: how O's normaliser is formed -- 0: the fp32 sum (also used for
 // L); 1: sum of the bf16-rounded weights via integer unpack; 2: the same sum with mixed
 // bf16 + fp32 adds.  FA_FWD_RESCALE: the reference max moves (and O is rescaled) only when a row's
 // max grows by more than this many log2 units (0: on every increase).  FA_FWD_MAX3: three-input
 // max for the row maximum.
-#ifndef FA_FWD_POLY_EVERY
-#define FA_FWD_POLY_EVERY 0
-#endif
 #ifndef FA_FWD_RSUM
 #define FA_FWD_RSUM 2
 #endif
@@ -260,6 +256,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         tma_prefetch_desc(&tmV);
         int kv_it = 0;   // KV tiles loaded so far (ring position)
         int kq = 0;      // units with work so far (the Q barriers' phase)
+        int q_n = 0;     // Q loads issued, and K / V loads issued per ring stage: each issued load
+        int k_n[C::STAGES], v_n[C::STAGES];  // is one phase of its full barrier (drain below)
+#pragma unroll
+        for (int s = 0; s < C::STAGES; ++s) k_n[s] = v_n[s] = 0;
         bool ok = true;
         for (int k = 0;; ++k) {
           const int u = fwd_unit_of(k, cta, G, p.units);
@@ -273,6 +273,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
             mbar_arrive_expect_tx(BAR_Q, C::KB * p.pack * p.Nq * 128);
             for (int kb = 0; kb < C::KB; ++kb)
               tma_load_3d(sbase + C::OFF_Q + kb * (C::BM * 128), &tmQ, BAR_Q, kb * 64, 0, un.head);
+            ++q_n;
           } else {
             int q_tiles = 0;
             for (int t = 0; t < NQT; ++t) q_tiles += (un.nkv[t] > 0);
@@ -283,36 +284,51 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
                 tma_load_3d(sbase + C::OFF_Q + t * C::QTILE_BYTES + kb * (C::BM * 128), &tmQ, BAR_Q,
                             kb * 64, un.q0 + t * C::BM, un.head);
             }
+            ++q_n;
           }
           for (int j = 0; j < un.J; ++j) {
             const int g = kv_it + j;
             const int s = g % C::STAGES;
             const uint32_t ph = (g / C::STAGES) & 1;
+#ifdef FA_TEST_STARVE
+            // Test build only (libfattn_starve.so): CTA 0 never issues the second K/V tile of its
+            // first unit, so the MMA warp's bounded wait for it runs out and the kernel must
+            // report FA_ERR_TIMEOUT and tear down cleanly.  Nothing is left in flight: the loads
+            // issued so far are drained below like after any other abort.
+            if (cta == 0 && k == 0 && j == 1) {
+              ok = false;
+              break;
+            }
+#endif
             if (!(ok = W.wait(BAR_KE(s), ph ^ 1, 1))) break;
             FA_TRACE_EV(20, j);
             mbar_arrive_expect_tx(BAR_KF(s), C::KVTILE_BYTES);
             for (int kb = 0; kb < C::KB; ++kb)
               tma_load_3d(sbase + C::OFF_K + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmK,
                           BAR_KF(s), kb * 64, (un.kt0 + j) * C::BN, un.kv_head);
+            ++k_n[s];
             if (!(ok = W.wait(BAR_VE(s), ph ^ 1, 2))) break;
             FA_TRACE_EV(21, j);
             mbar_arrive_expect_tx(BAR_VF(s), C::KVTILE_BYTES);
             for (int kb = 0; kb < C::KB; ++kb)
               tma_load_3d(sbase + C::OFF_V + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmV,
                           BAR_VF(s), kb * 64, (un.kt0 + j) * C::BN, un.kv_head);
+            ++v_n[s];
           }
           if (!ok) break;
           kv_it += un.J;
           ++kq;
         }
         if (!ok) {
-          // drain (bounded): every load issued so far lands before the CTA exits
-          W.drain(BAR_Q, kq & 1);
+          // drain (bounded): every load issued so far lands before the CTA exits.  A barrier has
+          // at most its last phase outstanding (a load is issued only after the previous one on
+          // the same buffer was consumed), so waiting for the phase of its last issued load is
+          // enough; a barrier with no load issued is skipped.
+          if (q_n > 0) W.drain(BAR_Q, (q_n - 1) & 1);
+#pragma unroll
           for (int s = 0; s < C::STAGES; ++s) {
-            W.drain(BAR_KF(s), 0);
-            W.drain(BAR_KF(s), 1);
-            W.drain(BAR_VF(s), 0);
-            W.drain(BAR_VF(s), 1);
+            if (k_n[s] > 0) W.drain(BAR_KF(s), (k_n[s] - 1) & 1);
+            if (v_n[s] > 0) W.drain(BAR_VF(s), (v_n[s] - 1) & 1);
           }
         }
       }
@@ -510,14 +526,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
             f2unpack(ffma2(f2pack(__uint_as_float(s[c][2 * e]), __uint_as_float(s[c][2 * e + 1])),
                            sc2, nm2),
                      x0, x1);
-            // one pair in FA_FWD_POLY_EVERY goes through the FMA-pipe polynomial, the rest MUFU
-            if (FA_FWD_POLY_EVERY > 0 &&
-                (e % (FA_FWD_POLY_EVERY > 0 ? FA_FWD_POLY_EVERY : 1)) == FA_FWD_POLY_EVERY - 1) {
-              ex2_poly2(x0, x1, p0, p1);
-            } else {
-              p0 = ex2(x0);
-              p1 = ex2(x1);
-            }
+            p0 = ex2(x0);
+            p1 = ex2(x1);
             pk[e] = pack_bf16(p0, p1);
             sum_x[e & 1] = fadd2(sum_x[e & 1], f2pack(p0, p1));
 #if FA_FWD_RSUM == 1

@@ -149,11 +149,15 @@ struct Waiter {
       }
     }
   }
-  // Teardown wait: ignores the abort flag (used to drain copies/MMAs already in flight).
+  // Teardown wait: ignores the abort flag (used to drain copies/MMAs already in flight).  It has
+  // its own limit, far above any copy or MMA latency and independent of limit_ns, so a CTA that
+  // gave up early (even with a very short limit_ns) still lets its issued work land before it
+  // exits; the limit only keeps a wait for work that was never issued from running forever.
+  static constexpr uint64_t kDrainLimitNs = 4000000000ull;  // 4 s
   __device__ __forceinline__ bool drain(uint32_t bar, uint32_t parity) const {
     const uint64_t t0 = global_ns();
     while (!mbar_try_wait(bar, parity)) {
-      if (global_ns() - t0 > limit_ns) return false;
+      if (global_ns() - t0 > kDrainLimitNs) return false;
     }
     return true;
   }
@@ -409,26 +413,6 @@ __device__ __forceinline__ float lg2(float x) {
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// 2^x on the FMA/ALU pipes, for the share of exponentials taken off the MUFU unit.
-// Range reduction x = n + f with n = round(x) obtained by the 1.5*2^23 shifter trick (exact for
-// |x| < 2^22), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients are our own
-// minimax fit of the relative error on [-1/2, 1/2] (linear-programming fit on 4001 points;
-// max relative error 7.5e-5, far below the bf16 rounding applied to P afterwards); 2^n is
-// applied by adding n to the exponent field.  Inputs below -126 return 0 (masked scores are
-// -inf).  Valid for x <= 127.
-__device__ __forceinline__ float ex2_poly(float x) {
-  const float kShift = 12582912.0f;  // 1.5 * 2^23
-  const float xc = fmaxf(x, -126.0f);
-  const float t = xc + kShift;
-  const float n = t - kShift;
-  const float f = xc - n;
-  float p = fmaf(f, 0.0551716685295105f, 0.2426111251115799f);
-  p = fmaf(p, f, 0.6932609677314758f);
-  p = fmaf(p, f, 0.9999280571937561f);
-  const uint32_t bits = __float_as_uint(p) + (__float_as_uint(t) << 23);
-  return x < -126.0f ? 0.f : __uint_as_float(bits);
-}
-
 // Paired fp32 arithmetic (sm_100 f32x2 instructions: two lanes of fp32 per instruction).
 __device__ __forceinline__ uint64_t f2pack(float a, float b) {
   uint64_t r;
@@ -447,50 +431,6 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
-}
-
-// Cheaper pair form for inputs already known to be >= -126 (callers clamp): no select, and
-// the exponent is inserted with one integer multiply-add per value.
-__device__ __forceinline__ void ex2_poly2_clamped(float x0, float x1, float& p0, float& p1) {
-  const float kShift = 12582912.0f;  // 1.5 * 2^23
-  const uint64_t xc = f2pack(x0, x1);
-  const uint64_t t = fadd2(xc, f2pack(kShift, kShift));
-  const uint64_t nn = fadd2(t, f2pack(-kShift, -kShift));
-  float n0, n1;
-  f2unpack(nn, n0, n1);
-  const uint64_t f = fadd2(xc, f2pack(-n0, -n1));
-  uint64_t q = ffma2(f, f2pack(0.0551716685295105f, 0.0551716685295105f),
-                     f2pack(0.2426111251115799f, 0.2426111251115799f));
-  q = ffma2(q, f, f2pack(0.6932609677314758f, 0.6932609677314758f));
-  q = ffma2(q, f, f2pack(0.9999280571937561f, 0.9999280571937561f));
-  float q0, q1, t0, t1;
-  f2unpack(q, q0, q1);
-  f2unpack(t, t0, t1);
-  p0 = __uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(q0));
-  p1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(q1));
-}
-
-// ex2_poly on a pair, with the range reduction and polynomial in paired fp32 instructions.
-__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& p0, float& p1) {
-  const float kShift = 12582912.0f;  // 1.5 * 2^23
-  const float a0 = fmaxf(x0, -126.0f), a1 = fmaxf(x1, -126.0f);
-  const uint64_t xc = f2pack(a0, a1);
-  const uint64_t t = fadd2(xc, f2pack(kShift, kShift));
-  const uint64_t nn = fadd2(t, f2pack(-kShift, -kShift));
-  float n0, n1;
-  f2unpack(nn, n0, n1);
-  const uint64_t f = fadd2(xc, f2pack(-n0, -n1));
-  uint64_t q = ffma2(f, f2pack(0.0551716685295105f, 0.0551716685295105f),
-                     f2pack(0.2426111251115799f, 0.2426111251115799f));
-  q = ffma2(q, f, f2pack(0.6932609677314758f, 0.6932609677314758f));
-  q = ffma2(q, f, f2pack(0.9999280571937561f, 0.9999280571937561f));
-  float q0, q1, t0, t1;
-  f2unpack(q, q0, q1);
-  f2unpack(t, t0, t1);
-  const float r0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  const float r1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-  p0 = x0 < -126.0f ? 0.f : r0;
-  p1 = x1 < -126.0f ? 0.f : r1;
 }
 
 // acc0 += lo(bf16 pair), acc1 += hi(bf16 pair), with mixed-precision fp32 + bf16 adds.

@@ -107,6 +107,10 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
  *
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress,
  * with that device current) and caches it; make that first call before any stream capture.
+ * The cached address belongs to the device's primary context, which the CUDA runtime keeps for
+ * the life of the process: a caller that resets the device (cudaDeviceReset) or drives the
+ * library from another context on the same device invalidates it, and must not call this
+ * entry point afterwards.
  * All calls on a device share the one array, which keeps whatever the last call left in it
  * (the kernels clear what must start at zero).  Calls that overlap on the GPU -- on different
  * streams, or from different host threads -- race on the array and corrupt each other's

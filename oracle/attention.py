@@ -28,6 +28,8 @@ exactly).  Arrays are [B, H, N, d]; L and D are [B, H, N].
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 
@@ -83,14 +85,43 @@ def attention_probs(q, k, causal: bool, scale: float):
     return P
 
 
-def attention_forward_online(q, k, v, causal: bool, scale: float, block_r: int, block_c: int):
-    """The tiled forward with the online-softmax recurrence, in the pages' order.
+def _block_summary(s_blk, v_blk):
+    """Softmax statistics of one block of keys for a block of query rows: the row max m, the sum
+    of exponentials l = sum_j exp(s_j - m) and the unnormalised output u = sum_j exp(s_j - m) v_j.
 
-    [P3] "Tiling Algorithm": (1) split Q into B_r x d blocks and K, V into B_c x d blocks;
-    (2) for each Q block iterate over all K, V blocks; (3) S_ij = Q_i K_j^T (scaled);
-    (4) track the running row max m and row sum l; (5) update O_i, rescaling the previous partial
-    result by exp(m_old - m_new) and adding exp(S_ij - m_new) V_j ([P1] update rule);
-    (6) after the last block divide O_i by l.  L_i = m_i + ln l_i is kept for the backward ([P1]).
+    A row whose scores in this block are all -inf (every key masked) has no maximum; it gets
+    m = -inf, l = 0 and u = 0, the identity of the combination below.
+    """
+    m = s_blk.max(axis=1)
+    seen = np.isfinite(m)
+    e = np.exp(s_blk - np.where(seen, m, 0.0)[:, None])
+    return m, e.sum(axis=1), e @ v_blk
+
+
+def _combine(a, b):
+    """Merge the statistics of two disjoint key sets ([P1] rescale(O_prev, m_old, m_new); [P3]
+    "Online Softmax Trick"): move both onto the larger maximum and add.  The operation is
+    associative and commutative, so any grouping of the key blocks gives the same softmax."""
+    (m1, l1, u1), (m2, l2, u2) = a, b
+    m = np.maximum(m1, m2)
+    ref = np.where(np.isfinite(m), m, 0.0)
+    w1 = np.where(np.isfinite(m1), np.exp(m1 - ref), 0.0)
+    w2 = np.where(np.isfinite(m2), np.exp(m2 - ref), 0.0)
+    return m, w1 * l1 + w2 * l2, w1[:, None] * u1 + w2[:, None] * u2
+
+
+def attention_forward_online(q, k, v, causal: bool, scale: float, block_r: int, block_c: int,
+                             tree: bool = False):
+    """The blockwise forward: the softmax of a row is assembled from per-block statistics.
+
+    The keys are cut into blocks of ``block_c`` and the queries into blocks of ``block_r``
+    ([P3] "Tiling Algorithm"; [P1]: a Q block against every K, V block).  For each (query block,
+    key block) pair the scores exist only for that pair; their summary (row max m, exponential
+    sum l, unnormalised output u, see ``_block_summary``) is folded into the running summary by
+    ``_combine`` ([P1] rescale rule; [P2] "Obliczanie Softmax w trybie online": the two running
+    values).  Left to right (``tree=False``) this is the running recurrence; ``tree=True`` merges
+    the block summaries pairwise instead, which associativity says must give the same result.
+    Finally O = u / l and L = m + ln l ([P1]: L is kept for the backward).
     Masked entries are -inf and contribute exp(-inf) = 0.
     """
     q = np.asarray(q, np.float64)
@@ -104,27 +135,27 @@ def attention_forward_online(q, k, v, causal: bool, scale: float, block_r: int, 
         for h in range(H):
             for r0 in range(0, N, block_r):
                 r1 = min(N, r0 + block_r)
-                qi = q[b, h, r0:r1]
-                m = np.full(r1 - r0, -np.inf)
-                l = np.zeros(r1 - r0)
-                acc = np.zeros((r1 - r0, v.shape[-1]))
+                parts = []
                 for c0 in range(0, Nk, block_c):
                     c1 = min(Nk, c0 + block_c)
-                    s = scale * (qi @ k[b, h, c0:c1].T)
+                    s = scale * (q[b, h, r0:r1] @ k[b, h, c0:c1].T)
                     if causal:
-                        rows = np.arange(r0, r1)[:, None]
-                        cols = np.arange(c0, c1)[None, :]
-                        s = np.where(cols > rows, -np.inf, s)
-                    m_new = np.maximum(m, s.max(axis=1))
-                    # a row whose keys so far are all masked keeps m = -inf; nothing to add yet
-                    safe = np.isfinite(m_new)
-                    m_ref = np.where(safe, m_new, 0.0)
-                    p = np.exp(s - m_ref[:, None])
-                    alpha = np.where(safe, np.exp(m - m_ref), 1.0)
-                    acc = alpha[:, None] * acc + p @ v[b, h, c0:c1]
-                    l = alpha * l + p.sum(axis=1)
-                    m = m_new
-                O[b, h, r0:r1] = acc / l[:, None]
+                        hidden = np.arange(c0, c1)[None, :] > np.arange(r0, r1)[:, None]
+                        s = np.where(hidden, -np.inf, s)
+                    parts.append(_block_summary(s, v[b, h, c0:c1]))
+                if tree:
+                    while len(parts) > 1:
+                        nxt = [_combine(parts[i], parts[i + 1])
+                               for i in range(0, len(parts) - 1, 2)]
+                        if len(parts) % 2:
+                            nxt.append(parts[-1])
+                        parts = nxt
+                    m, l, u = parts[0]
+                else:
+                    m, l, u = parts[0]
+                    for part in parts[1:]:
+                        m, l, u = _combine((m, l, u), part)
+                O[b, h, r0:r1] = u / l[:, None]
                 L[b, h, r0:r1] = m + np.log(l)
     return O, L
 
@@ -162,24 +193,6 @@ def attention_backward(q, k, v, o, lse, do, causal: bool, scale: float):
     return dq, dk, dv
 
 
-def attention_head_subset(q, k, v, do, causal: bool, scale: float, heads):
-    """Forward + backward on a subset of (b, h) heads only (heads are independent).
-
-    Used where the full workload is too large for the oracle: the returned arrays hold complete
-    results for the listed heads.  Returns dict head -> (O, L, dQ, dK, dV), each one head's slice.
-    """
-    out = {}
-    for (b, h) in heads:
-        sl = (slice(b, b + 1), slice(h, h + 1))
-        O, L = attention_forward(q[sl], k[sl], v[sl], causal, scale)
-        res = [O[0, 0], L[0, 0]]
-        if do is not None:
-            dq, dk, dv = attention_backward(q[sl], k[sl], v[sl], O, L, do[sl], causal, scale)
-            res += [dq[0, 0], dk[0, 0], dv[0, 0]]
-        out[(b, h)] = tuple(res)
-    return out
-
-
 def attention_rows(q, k, v, rows, causal: bool, scale: float):
     """Forward outputs of selected query rows of ONE head (q, k, v: [N, d] arrays).
 
@@ -191,13 +204,16 @@ def attention_rows(q, k, v, rows, causal: bool, scale: float):
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
     rows = np.asarray(rows)
-    s = scale * (q[rows] @ k.T)
+    # causal: keys after the last requested row are hidden from every one of them (they would
+    # contribute exp(-inf) = 0), so they are left out of the products
+    nk = min(k.shape[0], int(rows.max()) + 1) if causal else k.shape[0]
+    s = scale * (q[rows] @ k[:nk].T)
     if causal:
-        s = np.where(np.arange(k.shape[0])[None, :] > rows[:, None], -np.inf, s)
+        s = np.where(np.arange(nk)[None, :] > rows[:, None], -np.inf, s)
     m = s.max(axis=1, keepdims=True)
     e = np.exp(s - m)
     l = e.sum(axis=1, keepdims=True)
-    return (e / l) @ v, (m + np.log(l))[:, 0]
+    return (e / l) @ v[:nk], (m + np.log(l))[:, 0]
 
 
 def attention_dq_rows(q, k, v, do, rows, causal: bool, scale: float):
@@ -217,6 +233,63 @@ def attention_dq_rows(q, k, v, do, rows, causal: bool, scale: float):
     D = np.sum(do[rows] * O, axis=1)
     ds = p * (dp - D[:, None])
     return scale * (ds @ k)
+
+
+def attention_row_stats(q, k, v, do, causal: bool, scale: float, block: int = 256):
+    """L_i and D_i = dO_i . O_i for EVERY query row of ONE head (q, k, v, do: [N, d] arrays).
+
+    Each row needs its own scores against all keys only ([P2], [P3] formula), so the rows are
+    taken ``block`` at a time and no N x N array is ever formed.  Returns (L [N], D [N]).
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    do = np.asarray(do, np.float64)
+    N = q.shape[0]
+    L = np.empty(N)
+    D = np.empty(N)
+
+    def one_block(r0):
+        rows = np.arange(r0, min(N, r0 + block))
+        O, L[rows] = attention_rows(q, k, v, rows, causal, scale)
+        D[rows] = np.sum(do[rows] * O, axis=1)
+
+    # the blocks are independent; numpy releases the interpreter lock inside its array
+    # operations, so one thread per core (each with a single-threaded BLAS) keeps the host's cores
+    # busy on long heads
+    from concurrent.futures import ThreadPoolExecutor
+
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1), \
+            ThreadPoolExecutor(max_workers=len(os.sched_getaffinity(0))) as ex:
+        list(ex.map(one_block, range(0, N, block)))
+    return L, D
+
+
+def attention_dkdv_key_rows(q, k, v, do, keys, causal: bool, scale: float, stats=None):
+    """dK and dV of selected KEY rows of ONE head (q, k, v, do: [N, d] arrays).
+
+    Key j's gradients are column sums over the query rows that see it:
+      dV_j = sum_i P_ij dO_i,  dK_j = scale * sum_i P_ij (dP_ij - D_i) q_i,
+    with P_ij = exp(scale q_i . k_j - L_i) recomputed from the logsumexp ([P1]: the backward
+    recomputes P from L), dP_ij = dO_i . v_j and D_i = dO_i . O_i.  L and D of all rows come from
+    ``attention_row_stats`` (pass them as ``stats`` to reuse them).  Returns (dK [len(keys), d],
+    dV [len(keys), d]).
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    do = np.asarray(do, np.float64)
+    keys = np.asarray(keys)
+    L, D = attention_row_stats(q, k, v, do, causal, scale) if stats is None else stats
+    s = scale * (q @ k[keys].T)                                   # [N, len(keys)]
+    p = np.exp(s - L[:, None])
+    if causal:
+        p = np.where(keys[None, :] > np.arange(q.shape[0])[:, None], 0.0, p)
+    dv = p.T @ do
+    dp = do @ v[keys].T
+    ds = p * (dp - D[:, None])
+    return scale * (ds.T @ q), dv
 
 
 def _group_size(q, k):

@@ -19,6 +19,17 @@ def test_exports_every_declared_symbol():
         assert hasattr(L, n), n
 
 
+def test_starve_test_build_exports_the_same_symbols():
+    """The test-only build used by the bounded-wait test loads and exports the same entry points
+    (it differs from the product library by one left-out copy in the forward)."""
+    import ctypes
+
+    from exact_io_aware_43_b200.build import STARVE_PATH
+    L = ctypes.CDLL(STARVE_PATH)
+    for n in fa.header_functions():
+        assert hasattr(L, n), n
+
+
 def test_version():
     assert fa.fa_version() >= 100
 

@@ -15,8 +15,9 @@ import pytest
 import torch
 
 import attn_inputs as ai
-from oracle import (attention_backward, attention_forward, attention_forward_online,
-                    attention_probs)
+from oracle import (attention_backward, attention_dkdv_key_rows, attention_forward,
+                    attention_forward_online, attention_probs, attention_row_stats)
+from oracle.attention import _block_summary
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -39,7 +40,10 @@ def _arr(rows):
     return np.array([[_ev(c) for c in r] if isinstance(r, list) else _ev(r) for r in rows])
 
 
-@pytest.mark.parametrize("name", ["tiny_noncausal_n2_d1.json", "tiny_causal_n2_d1.json"])
+GOLDEN_CASES = ["tiny_noncausal_n2_d1.json", "tiny_causal_n2_d1.json", "tiny_scaled_n2_d1.json"]
+
+
+@pytest.mark.parametrize("name", GOLDEN_CASES)
 def test_golden_hand_worked(name):
     g = json.load(open(os.path.join(GOLDEN, name)))
     q, k, v, do = (_arr(g[t])[None, None] for t in ("q", "k", "v", "do"))
@@ -50,6 +54,27 @@ def test_golden_hand_worked(name):
     np.testing.assert_allclose(dq[0, 0], _arr(g["dQ"]), rtol=0, atol=1e-13)
     np.testing.assert_allclose(dk[0, 0], _arr(g["dK"]), rtol=0, atol=1e-13)
     np.testing.assert_allclose(dv[0, 0], _arr(g["dV"]), rtol=0, atol=1e-13)
+
+
+def _golden_probs_error(name, probs):
+    g = json.load(open(os.path.join(GOLDEN, name)))
+    q, k = (_arr(g[t])[None, None] for t in ("q", "k"))
+    P = probs(q, k, g["causal"], g["scale"])
+    return float(np.abs(P[0, 0] - _arr(g["P"])).max())
+
+
+@pytest.mark.parametrize("name", GOLDEN_CASES)
+def test_golden_probabilities(name):
+    """attention_probs against the hand-worked P of each golden case."""
+    assert _golden_probs_error(name, attention_probs) <= 1e-15
+
+
+def test_golden_probabilities_catch_a_scale_slip():
+    """A probability helper that drops (or doubles) the scale fails the scaled golden case."""
+    dropped = lambda q, k, c, s: attention_probs(q, k, c, 1.0)
+    doubled = lambda q, k, c, s: attention_probs(q, k, c, 2.0 * s)
+    for bad in (dropped, doubled):
+        assert _golden_probs_error("tiny_scaled_n2_d1.json", bad) > 1e-3
 
 
 def test_golden_naive_score_bytes():
@@ -67,9 +92,11 @@ def pin_online_equals_two_pass(fwd, online):
     for causal in (False, True):
         O2, L2 = fwd(q, k, v, causal, 0.35)
         for (br, bc) in ((1, 1), (7, 7), (16, 5), (64, 64), (37, 1), (5, 37)):
-            O1, L1 = online(q, k, v, causal, 0.35, br, bc)
-            if not (np.allclose(O1, O2, atol=1e-12, rtol=0) and np.allclose(L1, L2, atol=1e-12)):
-                return f"online != two-pass at causal={causal} Br={br} Bc={bc}"
+            for tree in (False, True):
+                O1, L1 = online(q, k, v, causal, 0.35, br, bc, tree)
+                if not (np.allclose(O1, O2, atol=1e-12, rtol=0) and
+                        np.allclose(L1, L2, atol=1e-12)):
+                    return f"online != two-pass at causal={causal} Br={br} Bc={bc} tree={tree}"
     return None
 
 
@@ -338,8 +365,8 @@ def _mut_fwd_causal_off_by_one(q, k, v, causal, scale):
     return O, L
 
 
-def _mut_online_no_rescale(q, k, v, causal, scale, br, bc):
-    # drops the exp(m_old - m_new) factor on the running output
+def _mut_online_no_rescale(q, k, v, causal, scale, br, bc, tree=False):
+    # merges block summaries without moving the running output onto the new maximum
     q = np.asarray(q, np.float64)
     B, H, N, d = q.shape
     O = np.empty((B, H, N, v.shape[-1]))
@@ -350,21 +377,22 @@ def _mut_online_no_rescale(q, k, v, causal, scale, br, bc):
                 r1 = min(N, r0 + br)
                 m = np.full(r1 - r0, -np.inf)
                 l = np.zeros(r1 - r0)
-                acc = np.zeros((r1 - r0, v.shape[-1]))
+                u = np.zeros((r1 - r0, v.shape[-1]))
                 for c0 in range(0, N, bc):
                     c1 = min(N, c0 + bc)
                     s = scale * q[b, h, r0:r1] @ k[b, h, c0:c1].T
                     if causal:
                         s = np.where(np.arange(c0, c1)[None] > np.arange(r0, r1)[:, None],
                                      -np.inf, s)
-                    mn = np.maximum(m, s.max(1))
-                    mr = np.where(np.isfinite(mn), mn, 0)
-                    p = np.exp(s - mr[:, None])
-                    al = np.where(np.isfinite(mn), np.exp(m - mr), 1.0)
-                    acc = acc + p @ v[b, h, c0:c1]
-                    l = al * l + p.sum(1)
+                    m2, l2, u2 = _block_summary(s, v[b, h, c0:c1])
+                    mn = np.maximum(m, m2)
+                    ref = np.where(np.isfinite(mn), mn, 0.0)
+                    w1 = np.where(np.isfinite(m), np.exp(m - ref), 0.0)
+                    w2 = np.where(np.isfinite(m2), np.exp(m2 - ref), 0.0)
+                    l = w1 * l + w2 * l2
+                    u = u + w2[:, None] * u2  # the slip: u is not multiplied by w1
                     m = mn
-                O[b, h, r0:r1] = acc / l[:, None]
+                O[b, h, r0:r1] = u / l[:, None]
                 L[b, h, r0:r1] = m + np.log(l)
     return O, L
 
@@ -444,3 +472,74 @@ def test_rows_closed_forms():
     assert np.allclose(O, np.stack([v[:r + 1].mean(0) for r in rows]), atol=1e-14)
     dq = orc.attention_dq_rows(rand((N, 4), 87), k, v, do, np.array([0]), True, 0.5)
     assert np.allclose(dq, 0.0, atol=1e-15)
+
+
+# --------------------------------------------------------------------------------------------
+# key-row gradients (used where a head is too long for the full N x N oracle)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_stats_match_full_oracle(causal):
+    q, k, v, do = (rand((1, 1, 70, 8), s) for s in (90, 91, 92, 93))
+    O, L = attention_forward(q, k, v, causal, 0.3)
+    Lr, Dr = attention_row_stats(q[0, 0], k[0, 0], v[0, 0], do[0, 0], causal, 0.3, block=16)
+    assert np.allclose(Lr, L[0, 0], atol=1e-13)
+    assert np.allclose(Dr, np.sum(do[0, 0] * O[0, 0], axis=1), atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_rows_match_full_backward_and_autograd(causal):
+    """dK, dV of sampled key rows equal those rows of the full analytic backward and of torch
+    float64 autograd; with every key selected they are the whole gradient."""
+    N, d = 53, 8
+    q, k, v, do = (rand((1, 1, N, d), s) for s in (94, 95, 96, 97))
+    O, L = attention_forward(q, k, v, causal, 0.45)
+    _, dk, dv = attention_backward(q, k, v, O, L, do, causal, 0.45)
+    tq, tk, tv = (torch.from_numpy(a).requires_grad_() for a in (q, k, v))
+    torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal,
+                                                     scale=0.45).backward(torch.from_numpy(do))
+    for keys in (np.array([0, 1, 17, 51, 52]), np.arange(N)):
+        dk_r, dv_r = attention_dkdv_key_rows(q[0, 0], k[0, 0], v[0, 0], do[0, 0], keys, causal,
+                                             0.45)
+        assert np.allclose(dk_r, dk[0, 0, keys], atol=1e-12)
+        assert np.allclose(dv_r, dv[0, 0, keys], atol=1e-12)
+        assert np.allclose(dk_r, tk.grad.numpy()[0, 0, keys], atol=1e-12)
+        assert np.allclose(dv_r, tv.grad.numpy()[0, 0, keys], atol=1e-12)
+
+
+def test_key_rows_invariants_and_closed_forms():
+    """Over all keys, sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i; causal: the last key is seen
+    only by the last query, so dV_{N-1} = P_{N-1,N-1} dO_{N-1}; with Q = 0 that weight is 1/N."""
+    N, d = 40, 4
+    q, k, v, do = (rand((N, d), s) for s in (98, 99, 100, 101))
+    keys = np.arange(N)
+    for causal in (False, True):
+        dk, dv = attention_dkdv_key_rows(q, k, v, do, keys, causal, 0.5)
+        assert np.allclose(dk.sum(axis=0), 0.0, atol=1e-12)
+        assert np.allclose(dv.sum(axis=0), do.sum(axis=0), atol=1e-12)
+    _, dv_last = attention_dkdv_key_rows(np.zeros((N, d)), k, v, do, np.array([N - 1]), True, 0.5)
+    assert np.allclose(dv_last[0], do[N - 1] / N, atol=1e-15)
+
+
+@pytest.mark.parametrize("slip", ["no_D", "key_mask_transposed", "unscaled_dk"])
+def test_key_rows_planted_mistakes_fail(slip):
+    """Broken copies of the key-row function disagree with torch float64 autograd."""
+    N, d = 23, 4
+    q, k, v, do = (rand((N, d), s) for s in (102, 103, 104, 105))
+    keys = np.array([0, 5, 22])
+    tq, tk, tv = (torch.from_numpy(a[None, None]).requires_grad_() for a in (q, k, v))
+    torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True,
+                                                     scale=0.6).backward(
+        torch.from_numpy(do[None, None]))
+    L, D = attention_row_stats(q, k, v, do, True, 0.6)
+    if slip == "no_D":
+        dk, dv = attention_dkdv_key_rows(q, k, v, do, keys, True, 0.6, stats=(L, 0 * D))
+    elif slip == "key_mask_transposed":
+        dk, dv = attention_dkdv_key_rows(q[::-1], k, v, do[::-1], keys, True, 0.6,
+                                         stats=(L[::-1], D[::-1]))
+    else:
+        dk, dv = attention_dkdv_key_rows(q, k, v, do, keys, True, 0.6)
+        dk = dk / 0.6
+    ok = (np.allclose(dk, tk.grad.numpy()[0, 0, keys], atol=1e-9) and
+          np.allclose(dv, tv.grad.numpy()[0, 0, keys], atol=1e-9))
+    assert not ok
