@@ -62,6 +62,59 @@ def make_inputs(B: int, H: int, N: int, d: int, seed: int = 0, sigma_qk: float =
     return out
 
 
+# ------------------------------------------------------------------------------------ e4m3 codes
+E4M3_MAX = 448.0
+
+
+def e4m3_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Widen e4m3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no infinities,
+    S.1111.111 is NaN) exactly to float64."""
+    b = np.asarray(bits).astype(np.int64)
+    e = (b >> 3) & 0xF
+    m = b & 7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return np.where(b & 0x80, -mag, mag)
+
+
+def f64_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """Round values to e4m3 codes: round to nearest, ties to even, magnitudes above 448 saturate
+    to 448.  Normal numbers (>= 2^-6) have 3 mantissa bits; below 2^-6 the spacing is 2^-9."""
+    x = np.asarray(x, np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    _, ex = np.frexp(a)                      # a = f * 2^ex, f in [0.5, 1): binade 2^(ex-1)
+    binade = np.maximum(ex - 1, -6)          # subnormals share the 2^-6 binade's spacing
+    quantum = np.exp2((binade - 3).astype(np.float64))
+    r = np.minimum(np.round(a / quantum) * quantum, E4M3_MAX)  # numpy rounds halves to even
+    _, er = np.frexp(r)
+    normal = r >= 2.0 ** -6
+    exp_field = np.where(normal, er - 1 + 7, 0)
+    man = np.where(normal, r / np.exp2((er - 1).astype(np.float64)) * 8.0 - 8.0, r * 2.0 ** 9)
+    code = (exp_field.astype(np.int64) << 3) | man.astype(np.int64)
+    return (code | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
+
+
+def draw_e4m3(shape, seed: int, tensor: str, sigma: float = 1.0):
+    """One seeded tensor as e4m3 codes with a per-tensor scale: the same N(0, sigma^2) float32
+    draw as ``draw_bits``, divided (in float64) by scale = float32(max|x| / 448) and rounded to
+    e4m3, so the codes use the whole e4m3 range.  Returns (codes uint8, scale); the tensor the
+    codes stand for is scale * e4m3_bits_to_f64(codes)."""
+    rng = np.random.default_rng([int(seed), TENSOR_IDS[tensor]])
+    x = rng.standard_normal(size=tuple(shape), dtype=np.float32)
+    if sigma != 1.0:
+        x = (x * np.float32(sigma)).astype(np.float32)
+    scale = float(np.float32(np.abs(x).max() / E4M3_MAX)) if x.size else 1.0
+    return f64_to_e4m3_bits(x.astype(np.float64) / scale), scale
+
+
+def make_inputs_fp8(B: int, H: int, N: int, d: int, seed: int = 0, sigma_qk: float = 1.0) -> dict:
+    """Q, K, V [B, H, N, d] as e4m3 codes with one scale per tensor: {"q": (codes, scale), ...}.
+    ``sigma_qk`` = 3 gives the peaky-softmax variant, as for ``make_inputs``."""
+    shape = (B, H, N, d)
+    return {"q": draw_e4m3(shape, seed, "q", sigma_qk), "k": draw_e4m3(shape, seed, "k", sigma_qk),
+            "v": draw_e4m3(shape, seed, "v", 1.0)}
+
+
 def default_scale(d: int) -> float:
     """The scale the workloads use, 1/sqrt(d), as a float32 value."""
     return float(np.float32(1.0 / np.sqrt(np.float64(d))))

@@ -68,6 +68,8 @@ def parse_args(argv=None):
                     help="B,H,N,d,causal override (profiling runs on a smaller case)")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="key/value heads per batch (grouped-query attention; default: H)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the FP8 (e4m3) forward on the workload instead of the bf16 step")
     ap.add_argument("--decode", default=None,
                     help="B,H,H_kv,Nq,Nk,d[,splits]: time the split-key forward (decoding) instead "
                          "of the headline step; reports HBM throughput")
@@ -534,12 +536,120 @@ def run_decode(args):
     return 0
 
 
+def run_fp8(args):
+    """FP8 (e4m3) forward on the workload's shape: per-tensor scaled e4m3 Q, K, V resident on the
+    device, bf16 O and fp32 L out.  Tensor-bound like the bf16 forward; the roofline peak is the
+    measured dense bf16 rate times the nominal fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s = 2)."""
+    import torch
+    import exact_io_aware_43_b200 as fa
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    rank, world = dist_init("nccl")
+    W = WORKLOAD
+    B, H, N, d, causal = W["B"], W["H"], W["N"], W["d"], W["causal"]
+    s = ai.default_scale(d)
+    x = ai.make_inputs_fp8(B, H, N, d, seed=rank_seed(rank))
+    host = {t: torch.from_numpy(c) for t, (c, _) in x.items()}
+    sc = {t: sc_ for t, (_, sc_) in x.items()}
+    q, k, v = (host[t].to(dev) for t in ("q", "k", "v"))
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        fa.forward_fp8(q, k, v, sc["q"], sc["k"], sc["v"], causal, s, out=o, lse=lse)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == 0, "a kernel reported a timeout during warm-up"
+    fa.fa_timer_read(fa.FA_KERNEL_FWD)
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(dev)
+    torch.cuda.synchronize()
+    fa.fa_timer_enable(True)
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    fa.fa_timer_enable(False)
+    barrier(dev)
+    clocks = sampler.stop()
+    status = fa.fa_device_status()
+    ms = reduce_max(sum(a.elapsed_time(b) for a, b in ev) / args.steps, dev)
+    n_f, t_f = fa.fa_timer_read(fa.FA_KERNEL_FWD)
+    ff, _ = flops(B, H, N, d, causal)
+    peaks, peak_src = load_peaks()
+    peak = 2.0 * peaks["bf16_tflops"]
+    kern_ms = t_f / max(1, n_f)
+    achieved = ff / (kern_ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak,
+            "peak_source": f"{peak_src} bf16_tflops (burst) x 2, the nominal fp8/bf16 ratio",
+            "frac_of_bf16_peak": achieved / peaks["bf16_tflops"], "kernel": "fa_fwd_fp8_kernel",
+            "launches": n_f, "avg_ms": kern_ms, "traffic": None}
+    # end to end through the public API: e4m3 codes from pinned host memory, O and L back
+    e2e = None
+    if args.e2e_steps > 0:
+        hin = {t: host[t].pin_memory() for t in ("q", "k", "v")}
+        ho = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+        hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        e_ev = []
+        torch.cuda.synchronize()
+        for i in range(args.e2e_steps + 2):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for t, dst in (("q", q), ("k", k), ("v", v)):
+                dst.copy_(hin[t], non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+            b.record()
+            if i >= 2:
+                e_ev.append((a, b))
+        torch.cuda.synchronize()
+        e_ms = reduce_max(sum(a.elapsed_time(b) for a, b in e_ev) / len(e_ev), dev)
+        e2e = {"value": world * ff / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(t.numel() for t in hin.values()),
+               "d2h_bytes_per_step": ho.numel() * 2 + hl.numel() * 4, "ms_per_step": e_ms,
+               "api": "serial copies around fa_fwd_fp8"}
+    if rank == 0:
+        line = {
+            "metric": "attention fwd TFLOP/s fp8 (e4m3 Q, K, V, per-tensor scales) at N=8K d=128 "
+                      "causal; % of B200 FP8 peak",
+            "value": world * ff / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+            "data": "synthetic",
+            "config": {"workload": f"FP8 forward, B={B} H={H} N={N} d={d} causal={causal}",
+                       **WORKLOAD, "scale": s, "flops_per_step_per_gpu": ff,
+                       "l2": "flushed before every timed step (256 MiB write, outside the events)"},
+            "roofline": roof, "e2e": e2e, "clocks": clocks, "gpu_launches": n_f,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
     if args.decode is not None:
         return run_decode(args)
+    if args.fp8:
+        return run_fp8(args)
     return run_gpu(args)
 
 

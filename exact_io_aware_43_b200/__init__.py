@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
     L.fa_device_status.restype = i
     L.fa_version.argtypes = []
     L.fa_version.restype = i
+    L.fa_fwd_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, i, f, vp]
+    L.fa_fwd_fp8.restype = i
     L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
     L.fa_bwd_noalloc.restype = i
     L.fa_timer_enable.argtypes = [i]
@@ -107,6 +109,12 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, workspace
            workspace_bytes, stream) -> int:
     return lib().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, int(causal), float(scale),
                         workspace, workspace_bytes, stream)
+
+
+def fa_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, d, causal, scale,
+               stream) -> int:
+    return lib().fa_fwd_fp8(q8, k8, v8, float(q_scale), float(k_scale), float(v_scale), o, lse,
+                            B, H, N, d, int(causal), float(scale), stream)
 
 
 def fa_bwd_gqa_workspace_size(B, H, H_kv, N, d) -> int:
@@ -265,6 +273,27 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
                         workspace.numel(), _stream_handle(q))
     _check(rc)
     return dq, dk, dv
+
+
+def forward_fp8(q8, k8, v8, q_scale: float, k_scale: float, v_scale: float,
+                causal: bool = False, scale: float | None = None, out=None, lse=None):
+    """O, L = attention(q_scale*Q8, k_scale*K8, v_scale*V8) for e4m3 code tensors q8, k8, v8
+    (contiguous CUDA tensors of dtype uint8 or float8_e4m3fn, [B, H, N, d]); O is bf16, L fp32."""
+    import torch
+    B, H, N, d = _shape(q8)
+    for t, name in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn) or not t.is_cuda or \
+                not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{name} must be a contiguous uint8/float8_e4m3fn CUDA tensor of "
+                             f"shape {(B, H, N, d)}")
+    scale = _default_scale(d) if scale is None else float(scale)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device) if out is None else out
+    L = torch.empty((B, H, N), dtype=torch.float32, device=q8.device) if lse is None else lse
+    _check_tensor(o, (B, H, N, d), torch.bfloat16, "out")
+    _check_tensor(L, (B, H, N), torch.float32, "lse")
+    _check(fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), q_scale, k_scale, v_scale,
+                      o.data_ptr(), L.data_ptr(), B, H, N, d, causal, scale, _stream_handle(q8)))
+    return o, L
 
 
 def default_splits(B, H, Nq, Nk, device=None, H_kv=None) -> int:

@@ -60,6 +60,8 @@ struct BwdParams {
   float* dq_acc;   // [BH, N, D] fp32
   float* L2;       // [BH, Npad] fp32: lse * log2(e), +inf on padded rows
   float* Drow;     // [BH, Npad] fp32: rowsum(dO * O), 0 on padded rows
+  uint8_t* aug;    // d = 128 only: per 128-query block, 4 KB of MMA operand holding -L/s and -D
+                   // as three bf16 terms each (see fa_bwd_pre_kernel); nullptr otherwise
   int BH;          // batch * query heads (rows of dq_acc, L2, Drow)
   int N;
   int Npad;        // N rounded up to 128
@@ -158,6 +160,18 @@ struct BwdCursor {
 // ------------------------------------------------------------------------------------------
 // preprocess: D, L2, zero dQ accumulator
 // ------------------------------------------------------------------------------------------
+// x as three bf16 terms hi + mid + lo (each the rounding of what the previous ones left; about
+// 24 significant bits together) in the first three of eight bf16 slots, the rest zero.
+__device__ __forceinline__ uint4 split3_bf16(float x) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(hi);
+  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(mid);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+  return make_uint4(uint32_t(__bfloat16_as_ushort(hi)) | (uint32_t(__bfloat16_as_ushort(mid)) << 16),
+                    uint32_t(__bfloat16_as_ushort(lo)), 0u, 0u);
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
   constexpr int G = D / 8;  // lanes per row, 8 bf16 (16 bytes) each
@@ -195,6 +209,19 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
     if (in && sub == 0) {
       p.Drow[r] = acc;
       p.L2[r] = (q < p.N) ? p.lse[size_t(head) * p.N + q] * 1.4426950408889634f : INFINITY;
+      if (p.aug != nullptr) {
+        // the 128-query kernel's B operand for its ninth K step: row q of the block gets
+        // [-L/s as hi, mid, lo, 0 x 5] in the first 8-element K half and [-D likewise] in the
+        // second, each half a run of 8-row x 16-byte core matrices (rows 16 B apart, 8-row
+        // groups 128 B apart, the two halves 2 KB apart).  A padded row gets a huge finite
+        // -L/s (never inf: the other step multiplies it by zero), so its P is 0.
+        const float xl = (q < p.N) ? -p.lse[size_t(head) * p.N + q] / p.scale : -0x1p100f;
+        const int blk = q >> 7, rr = q & 127;
+        uint8_t* tile = p.aug + (size_t(head) * (p.Npad >> 7) + blk) * 4096 +
+                        (rr >> 3) * 128 + (rr & 7) * 16;
+        *reinterpret_cast<uint4*>(tile) = split3_bf16(xl);
+        *reinterpret_cast<uint4*>(tile + 2048) = split3_bf16(-acc);
+      }
     }
   }
   // zero the dQ accumulator (its size is a multiple of 4 floats: D >= 64), and the dK, dV

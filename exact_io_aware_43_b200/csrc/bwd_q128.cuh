@@ -13,6 +13,13 @@
 //   R2 [128,256)  dP^T = V_j dO_i^T (fp32); once the dS^T warps have read it, dQ_i^T =
 //                 K_j^T dS^T (fp32, d on lanes, 128 query columns).
 //   [256,384) dV accumulator, [384,512) dK accumulator.
+// The row statistics enter through the tensor core instead of shared-memory loads: each S^T
+// and dP^T group gets a ninth K = 16 step whose A operand is a constant ones block and whose B
+// operand holds, per query, -L/s and -D split into three bf16 terms each (hi + mid + lo, about 24
+// bits; written by the preprocess kernel in the MMA's core-matrix layout).  The MMA then leaves
+// S^T - L/s and dP^T - D in tensor memory, so P^T = exp2((S^T - L/s) s log2e) and
+// dS^T = P^T (dP^T - D) need no per-query value from shared memory (the broadcast loads of L and
+// D cost as many shared-memory wavefronts as the MMA operands of a GEMM).
 // dS^T (bf16) goes to a shared tile, from which both dQ^T and dK (dS^T Q_i, both operands in
 // shared memory) read it.  Reuse is ordered by completion barriers, never by issue order:
 // S^T(i+1) is issued once dV(i) has completed, dP^T(i+1) once dQ^T(i) has been read out.
@@ -31,15 +38,6 @@
 // after dK(i), which leaves the tensor core no gap while the MMA thread waits for dV(i).
 #ifndef FA_BWDQ_EARLY_S
 #define FA_BWDQ_EARLY_S 1
-#endif
-// FA_BWDQ_DO_STAGES: dO_i buffers (1 or 2).  FA_BWDQ_SEP_STAGE: 1 gives the dQ staging its own
-// 32 KB instead of the dS^T tile's space (then the dS^T writes need not wait for the reduce to
-// read the staging).  Shared memory holds at most one of the two extra tiles.
-#ifndef FA_BWDQ_DO_STAGES
-#define FA_BWDQ_DO_STAGES 1
-#endif
-#ifndef FA_BWDQ_SEP_STAGE
-#define FA_BWDQ_SEP_STAGE 1
 #endif
 // FA_BWDQ_DK_SS: 1 reads dS^T for dK from the shared tile (both operands in shared memory), so
 // dQ^T may overwrite R2 as soon as dS^T is ready and is issued first; 0 reads dS^T from tensor
@@ -83,16 +81,24 @@ struct BwdQ128Cfg {
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
   static constexpr int OFF_Q = OFF_V + TILE;        // 2 stages
-  static constexpr int DO_STAGES = FA_BWDQ_DO_STAGES;
-  static constexpr bool SEP = FA_BWDQ_SEP_STAGE != 0;
-  static constexpr int OFF_DO = OFF_Q + 2 * TILE;            // DO_STAGES x dO_i
+  static constexpr int DO_STAGES = 1;
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;            // dO_i
   static constexpr int OFF_DS = OFF_DO + DO_STAGES * TILE;   // dS^T [2 q halves][128 keys][64 q]
-  static constexpr int OFF_STG = SEP ? OFF_DS + TILE : OFF_DS;  // dQ staging: 2 x [64 q][64 d] f32
-  static constexpr int OFF_ROWS = OFF_STG + TILE;            // 2 stages x (L2[128], D[128]) fp32
+  static constexpr int OFF_STG = OFF_DS + TILE;              // dQ staging: one [64 q][64 d] f32
+  static constexpr int STG_BYTES = 64 * 64 * 4;
+  // row-statistics operands of the ninth K step (no swizzle: 8-row x 16-byte core matrices,
+  // 8-row groups 128 B apart, the second 8 K-elements AUG_LBO bytes on):
+  //   AUG [2 stages][2 K halves: -L/s terms | -D terms][16 query groups][8 rows][8 bf16]
+  //   ONES [ones | zeros | ones], each [16 groups][8 rows][1, 1, 1, 0, 0, 0, 0, 0]: the S^T step
+  //   reads (ones, zeros) and so picks the -L/s terms, the dP^T step (zeros, ones) the -D terms
+  static constexpr int AUG_LBO = 2048;
+  static constexpr int AUG_BYTES = 2 * AUG_LBO;              // per 128-query block
+  static constexpr int OFF_AUG = OFF_STG + STG_BYTES;
+  static constexpr int OFF_ONES = OFF_AUG + 2 * AUG_BYTES;
   // barriers: kv, q_full[2], q_empty[2], do_full[2], do_empty[2], s_full, p_full, dp_full,
   //           ds_full, dv_done, dk_done, dq_full, dq_empty, ds_free, drain
   static constexpr int NBAR = 19;
-  static constexpr int OFF_BAR = OFF_ROWS + 2 * 2 * BR * 4;
+  static constexpr int OFF_BAR = OFF_ONES + 3 * AUG_LBO;
   static constexpr int OFF_MISC = OFF_BAR + 160;
   static constexpr int SMEM_NEED = OFF_MISC + 16;             // from a 1024-aligned base
   static constexpr int SMEM_MAX = 227 * 1024;                 // opt-in limit per CTA on sm_100
@@ -100,13 +106,17 @@ struct BwdQ128Cfg {
   static constexpr int SMEM_BYTES = SMEM_NEED + 1024 < SMEM_MAX ? SMEM_NEED + 1024 : SMEM_MAX;
   static_assert(NBAR * 8 <= 160, "barrier area");
   static_assert(SMEM_NEED <= SMEM_MAX, "shared memory budget");
-  static_assert(DO_STAGES == 1 || DO_STAGES == 2, "dO stages");
-  // dK reading the dS^T tile after dQ^T's completion is signalled: the staging must not share it
-  static_assert(SEP || !FA_BWDQ_DK_SS, "dK from shared dS^T needs separate dQ staging");
   static constexpr uint32_t IDESC_ST = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
   static constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, 0, 1);  // dV, dK (A in TMEM)
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, 128, 1, 1);  // dQ^T = K^T dS^T
 };
+
+// Descriptor of a no-swizzle K-major operand (layout code 0): core matrices of 8 rows x 16
+// bytes, K-adjacent ones `lbo` bytes apart, 8-row groups `sbo` bytes apart.
+__device__ __forceinline__ uint64_t sdesc_interleave(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
+         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
 
 template <bool CAUSAL>
 __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
@@ -181,10 +191,18 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
     tmem_relinquish();
     tc_fence_before();
   }
+  {
+    // the constant A operands of the ninth K step: [ones | zeros | ones], each 128 rows of
+    // [1, 1, 1, 0, 0, 0, 0, 0] (bf16) or of zeros, as 16-byte core-matrix rows
+    uint4* ones = reinterpret_cast<uint4*>(smem + C::OFF_ONES);
+    for (int i = threadIdx.x; i < 3 * C::AUG_LBO / 16; i += C::THREADS)
+      ones[i] = (i / (C::AUG_LBO / 16)) == 1 ? make_uint4(0u, 0u, 0u, 0u)
+                                             : make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);
+    fence_async_smem();
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const float* rows_smem = reinterpret_cast<const float*>(smem + C::OFF_ROWS);
 
   if (warp >= C::PRODUCER_WARP) {
     // ================================================================ control warpgroup
@@ -206,16 +224,15 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
         const int i = cur.i, head = cur.head;
         cur.next();
         const int s = t & 1;
-        // Q_i, L2_i and D_i into stage s once dK of step t-2 has released it
+        // Q_i and its row-statistics operand into stage s once dK of step t-2 has released it
         if (!W.wait(BAR_QE(s), ((t >> 1) & 1) ^ 1, 31)) break;
-        mbar_arrive_expect_tx(BAR_QF(s), C::TILE + 2 * C::BR * 4);
+        mbar_arrive_expect_tx(BAR_QF(s), C::TILE + C::AUG_BYTES);
         for (int kb = 0; kb < 2; ++kb)
           tma_load_3d(sbase + C::OFF_Q + s * C::TILE + kb * C::BLK, &tmQ, BAR_QF(s), kb * 64,
                       i * C::BR, head);
-        const size_t roff = size_t(head) * p.Npad + size_t(i) * C::BR;
-        const uint32_t rdst = sbase + C::OFF_ROWS + s * 2 * C::BR * 4;
-        bulk_load(rdst, p.L2 + roff, C::BR * 4, BAR_QF(s));
-        bulk_load(rdst + C::BR * 4, p.Drow + roff, C::BR * 4, BAR_QF(s));
+        const size_t aoff = (size_t(head) * (p.Npad / C::BR) + size_t(i)) * C::AUG_BYTES;
+        bulk_load(sbase + C::OFF_AUG + s * C::AUG_BYTES,
+                  reinterpret_cast<const uint8_t*>(p.aug) + aoff, C::AUG_BYTES, BAR_QF(s));
         ++tq;
         FA_TRACE_EV(20, t);
         // dO_i into its buffer once dP^T and dV of the step that used it last have read it
@@ -240,15 +257,22 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       const uint32_t ds_addr = sbase + C::OFF_DS;
       auto q_addr = [&](int s) { return sbase + C::OFF_Q + s * C::TILE; };
       auto do_addr = [&](int t) { return sbase + C::OFF_DO + (t % DS_) * C::TILE; };
-      // [S^T | dP^T] (128 keys x 128 queries) = A (keys x d) * B (queries x d)^T, both K-major
-      auto issue_st = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
+      // [S^T | dP^T] (128 keys x 128 queries) = A (keys x d) * B (queries x d)^T, both K-major,
+      // then the ninth step adds -L/s (ones at K 0-2 of the A block) or -D (ones at K 8-10) of
+      // each query from the stage's statistics operand
+      auto issue_st = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base, uint32_t ones_addr,
+                          uint32_t aug_addr) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
           mma_ss(tmem + d_col, sdesc_sw128(a_base + off, 16, 1024),
                  sdesc_sw128(b_base + off, 16, 1024), C::IDESC_ST, kk > 0 ? 1u : 0u);
         }
+        mma_ss(tmem + d_col, sdesc_interleave(ones_addr, C::AUG_LBO, 128),
+               sdesc_interleave(aug_addr, C::AUG_LBO, 128), C::IDESC_ST, 1u);
       };
+      const uint32_t ones_s = sbase + C::OFF_ONES, ones_dp = ones_s + C::AUG_LBO;
+      auto aug_addr = [&](int t) { return sbase + C::OFF_AUG + (t & 1) * C::AUG_BYTES; };
       // [dV | dK] (128 keys x 128 d) += A (TMEM, bf16 keys x queries: query half h packed at
       // columns 96h..96h+31) * B (queries x d, MN-major; the two 64-wide d blocks BLK apart)
       auto issue_kv = [&](uint32_t d_col, uint32_t a_col, uint32_t b_base, bool acc) {
@@ -278,7 +302,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
         if (!W.wait(BAR_QF((t + 1) & 1), ((t + 1) >> 1) & 1, 45)) return false;
         FA_TRACE_EV(3, t);
         tc_fence_after();
-        issue_st(C::T_S, k_addr, q_addr((t + 1) & 1));
+        issue_st(C::T_S, k_addr, q_addr((t + 1) & 1), ones_s, aug_addr(t + 1));
         tc_commit(BAR_SF);
         return true;
       };
@@ -286,13 +310,13 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       if (ok) ok = W.wait(BAR_QF(0), 0, 41);
       if (ok) {
         tc_fence_after();
-        issue_st(C::T_S, k_addr, q_addr(0));
+        issue_st(C::T_S, k_addr, q_addr(0), ones_s, aug_addr(0));
         tc_commit(BAR_SF);
         ok = W.wait(BAR_DOF(0), 0, 42);
       }
       if (ok) {
         tc_fence_after();
-        issue_st(C::T_DP, v_addr, do_addr(0));
+        issue_st(C::T_DP, v_addr, do_addr(0), ones_dp, aug_addr(0));
         tc_commit(BAR_DPF);
       }
       for (int t = 0; ok && t < nit; ++t) {
@@ -335,12 +359,15 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
           tc_commit(BAR_DQF);
         }
         if (more) {
-          // dP^T(t+1) into R2 once dQ^T(t) has been read out
+          // dP^T(t+1) into R2 once dQ^T(t) has been read out (its statistics operand came with
+          // Q_{t+1}, which S^T(t+1) has already waited for)
           if (!(ok = W.wait(BAR_DQE, t & 1, 48))) break;
           if (!(ok = W.wait(BAR_DOF((t + 1) % DS_), ((t + 1) / DS_) & 1, 49))) break;
+          if (!FA_BWDQ_EARLY_S && !(ok = W.wait(BAR_QF((t + 1) & 1), ((t + 1) >> 1) & 1, 45)))
+            break;
           FA_TRACE_EV(7, t);
           tc_fence_after();
-          issue_st(C::T_DP, v_addr, do_addr(t + 1));
+          issue_st(C::T_DP, v_addr, do_addr(t + 1), ones_dp, aug_addr(t + 1));
           tc_commit(BAR_DPF);
         }
       }
@@ -363,11 +390,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
     for (int t = 0; t < nit; ++t) {
       const int i = cur.i;
       cur.next();
-      const int s = t & 1;
-      const float* L2s = rows_smem + s * 2 * C::BR + c0;
-      const float* Ds = rows_smem + s * 2 * C::BR + C::BR + c0;
       if (!(ok = W.wait_warp(BAR_SF, t & 1, 50))) break;
-      if (!(ok = W.wait_warp(BAR_QF(s), (t >> 1) & 1, 51))) break;
       FA_TRACE_EV(11, t);
       tc_fence_after();
       uint32_t sv[2][32];
@@ -376,26 +399,26 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       tmem_wait_ld(sv[0]);
       tmem_wait_ld(sv[1]);
       FA_TRACE_EV(15, t);
-      // P^T = exp2(S^T s log2e - L2); zero for masked (causal key > query) and padded keys.
-      // Only the diagonal block (i == j) and a ragged last key block need the test.
+      // P^T = exp2((S^T - L/s) s log2e) (the MMA has subtracted L/s); zero for masked (causal
+      // key > query) and padded keys.  Only the diagonal block (i == j) and a ragged last key
+      // block need the test.
       uint32_t pk[32];
       const bool need_mask = !key_ok || (CAUSAL && i == j);
+      const uint64_t sl2 = f2pack(p.scale_log2, p.scale_log2);
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 l4 = reinterpret_cast<const float4*>(L2s)[c4];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-        float pr[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * c4 + e;
-          pr[e] = ex2(fmaf(__uint_as_float(sv[c >> 5][c & 31]), p.scale_log2, -lv[e]));
-          if (need_mask) {
-            const bool valid = key_ok && (!CAUSAL || r <= c0 + c);
-            pr[e] = valid ? pr[e] : 0.f;
-          }
+      for (int c2 = 0; c2 < 32; ++c2) {
+        const int c = 2 * c2;
+        float x0, x1;
+        f2unpack(fmul2(f2pack(__uint_as_float(sv[c >> 5][c & 31]),
+                              __uint_as_float(sv[c >> 5][(c & 31) + 1])),
+                       sl2),
+                 x0, x1);
+        float p0 = ex2(x0), p1 = ex2(x1);
+        if (need_mask) {
+          p0 = (key_ok && (!CAUSAL || r <= c0 + c)) ? p0 : 0.f;
+          p1 = (key_ok && (!CAUSAL || r <= c0 + c + 1)) ? p1 : 0.f;
         }
-        pk[2 * c4] = pack_bf16(pr[0], pr[1]);
-        pk[2 * c4 + 1] = pack_bf16(pr[2], pr[3]);
+        pk[c2] = pack_bf16(p0, p1);
       }
       // P^T over this thread's own S^T columns (the whole warpgroup has read them)
       FA_TRACE_EV(16, t);
@@ -415,31 +438,23 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       tmem_wait_ld(sv[0]);
       tmem_wait_ld(sv[1]);
       FA_TRACE_EV(18, t);
+      // the MMA has subtracted D: dS^T = P^T dP'^T, one paired multiply per two queries
       uint32_t dsk[32];
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 d4 = reinterpret_cast<const float4*>(Ds)[c4];
-        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = 4 * c4 + 2 * e;
-          const uint32_t pp = pk[c >> 1];
-          const float p0 = __uint_as_float(pp << 16);
-          const float p1 = __uint_as_float(pp & 0xffff0000u);
-          const float d0 = p0 * (__uint_as_float(sv[c >> 5][c & 31]) - dv4[2 * e]);
-          const float d1 = p1 * (__uint_as_float(sv[(c + 1) >> 5][(c + 1) & 31]) - dv4[2 * e + 1]);
-          dsk[c >> 1] = pack_bf16(d0, d1);
-        }
+      for (int c2 = 0; c2 < 32; ++c2) {
+        const int c = 2 * c2;
+        const uint32_t pp = pk[c2];
+        float d0, d1;
+        f2unpack(fmul2(f2pack(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u)),
+                       f2pack(__uint_as_float(sv[c >> 5][c & 31]),
+                              __uint_as_float(sv[c >> 5][(c & 31) + 1]))),
+                 d0, d1);
+        dsk[c2] = pack_bf16(d0, d1);
       }
       // dS^T into the shared tile (for dQ^T, and for dK when it reads shared memory) and, when dK
-      // reads tensor memory, over this thread's own dP^T columns; with shared staging the tile
-      // is free once the drain warps' reduce of the previous step has read its staging
+      // reads tensor memory, over this thread's own dP^T columns
       FA_TRACE_EV(19, t);
       if (!FA_BWDQ_DK_SS) tmem_st32(tmem + lane_base + C::T_DP + 96 * h, dsk);
-      if (!C::SEP && t > 0 && !(ok = W.wait_warp(BAR_DSFREE, (t - 1) & 1, 54))) {
-        if (!FA_BWDQ_DK_SS) tmem_wait_st();
-        break;
-      }
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const uint4 v = make_uint4(dsk[4 * c], dsk[4 * c + 1], dsk[4 * c + 2], dsk[4 * c + 3]);
@@ -475,18 +490,19 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
     tc_fence_before();
   } else {
     // ================================================================ dQ drain warpgroup
-    // dQ^T (d on TMEM lanes, 128 query columns) -> x scale -> two [64 queries][64 d] fp32
-    // staging slots in the dS^T tile's space -> TMA bulk reduce-add into the accumulator, one
-    // query half at a time (rows past N are clipped by the tensor map; halves wholly past N
-    // are skipped).
+    // dQ^T (d on TMEM lanes, 128 query columns) -> x scale -> a [64 queries][64 d] fp32 staging
+    // block -> TMA bulk reduce-add into the accumulator, one (query half, d half) at a time:
+    // the two warps holding that d half fill the block, the others wait (rows past N are
+    // clipped by the tensor map; query halves wholly past N are skipped).  The whole dQ^T is
+    // read out of tensor memory first, so the MMA warp may reuse its columns at once.
     regs_inc<C::DQ_REGS>();
     const int wq = warp - C::DQ_WARP0;
     const int tq = threadIdx.x - C::DQ_WARP0 * 32;  // 0..127
     const bool issuer = tq == 0;
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     const int drow = wq * 32 + lane;                // d index == TMEM lane
-    float* slots = reinterpret_cast<float*>(smem + C::OFF_STG);
-    float* my_slot = slots + (drow >> 6) * (64 * 64) + (drow & 63);
+    float* slot = reinterpret_cast<float*>(smem + C::OFF_STG);
+    float* my_col = slot + (drow & 63);
     if (issuer) tma_prefetch_desc(&tmdQ);
     BwdCursor cur(grp);
     for (int t = 0; t < nit; ++t) {
@@ -509,26 +525,23 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       for (int qh = 0; qh < 2; ++qh) {
         const int row0 = i * C::BR + 64 * qh;
         if (row0 >= p.N) break;  // uniform over the warpgroup
-        if (qh == 1 || C::SEP) {
-          if (issuer) bulk_wait_group_read<0>();  // the previous reduce has read the slots
-          named_bar_sync(1, 128);
-        }
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          my_slot[c * 64] = __uint_as_float(v[2 * qh + (c >> 5)][c & 31]) * p.scale;
-        fence_async_smem();
-        named_bar_sync(1, 128);
-        FA_TRACE_EV(62 + qh, t);
-        if (issuer) {
-          tma_reduce_add_3d(&tmdQ, smem_u32(slots), 0, row0, head);
-          tma_reduce_add_3d(&tmdQ, smem_u32(slots + 64 * 64), 64, row0, head);
-          bulk_commit_group();
+        for (int db = 0; db < 2; ++db) {
+          if (issuer) bulk_wait_group_read<0>();  // the previous reduce has read the block
+          named_bar_sync(1, 128);
+          if ((drow >> 6) == db) {  // warp-uniform
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              my_col[c * 64] = __uint_as_float(v[2 * qh + (c >> 5)][c & 31]) * p.scale;
+          }
+          fence_async_smem();
+          named_bar_sync(1, 128);
+          FA_TRACE_EV(62 + qh, t);
+          if (issuer) {
+            tma_reduce_add_3d(&tmdQ, smem_u32(slot), 64 * db, row0, head);
+            bulk_commit_group();
+          }
         }
-      }
-      // the dS^T tile may be rewritten once the reduces have read their staging
-      if (!C::SEP && issuer) {
-        bulk_wait_group_read<0>();
-        mbar_arrive(BAR_DSFREE);
       }
     }
     if (issuer) bulk_wait_group_all();

@@ -21,6 +21,7 @@
 #include "bwd_q128.cuh"
 #include "merge.cuh"
 #include "fwd.cuh"
+#include "fwd_fp8.cuh"
 
 namespace {
 
@@ -74,6 +75,23 @@ int make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_row
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return FA_OK;
+}
+
+// e4m3 [BH, N, d] map (one byte per element): box = min(d, 128) bytes x box_rows rows x 1 head,
+// 128-byte swizzle for d >= 128 (d / 128 boxes across a row), 64-byte swizzle for d = 64.
+int make_map_e4m3(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(d), cuuint64_t(N) * cuuint64_t(d)};
+  cuuint32_t box[3] = {cuuint32_t(d >= 128 ? 128 : d), cuuint32_t(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  d >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled (e4m3) failed (%d)", int(r));
   return FA_OK;
 }
 
@@ -242,6 +260,38 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   return FA_OK;
 }
 
+template <int D, bool CAUSAL, int NQT>
+int launch_fwd_fp8(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   fattn::FwdParams p, float v_scale, int BH, cudaStream_t st) {
+  using C = fattn::Fp8Cfg<D, NQT>;
+  auto kern = fattn::fa_fwd_fp8_kernel<D, CAUSAL, NQT>;
+  int rc = set_smem(kern, C::SMEM_BYTES);
+  if (rc) return rc;
+  if (C::REALLOC) {
+    static std::atomic<int> checked{0};  // 0 unknown, 1 ok, 2 bad
+    int chk = checked.load(std::memory_order_relaxed);
+    if (chk == 0) {
+      cudaFuncAttributes fa_attr;
+      cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+      chk = (fa_attr.numRegs * C::THREADS >= C::CTRL_REGS * 128 + C::SOFTMAX_REGS * 256) ? 1 : 2;
+      checked.store(chk, std::memory_order_relaxed);
+    }
+    if (chk == 2)
+      return fail(FA_ERR_UNSUPPORTED, "fa_fwd_fp8 kernel built with too few launch registers for "
+                                      "its register split");
+  }
+  p.BH = BH;
+  p.nqb = (p.Nq + NQT * C::BM - 1) / (NQT * C::BM);
+  p.units = BH * p.nqb;
+  const int G = p.units < sm_count() ? p.units : sm_count();
+  TimedLaunch tl(FA_KERNEL_FWD, st);
+  kern<<<dim3(unsigned(G)), C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, p, v_scale);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fa_fwd_fp8 launch");
+  return FA_OK;
+}
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // d = 128 backward: 128-query steps (fa_bwd_kernel_q128); 0 selects the 64-query kernel.
@@ -392,6 +442,9 @@ int bwd_dispatch(const void* q, const void* k, const void* v, const void* o, con
   p.dq_acc = reinterpret_cast<float*>(ws);
   p.L2 = reinterpret_cast<float*>(ws + dq_bytes);
   p.Drow = reinterpret_cast<float*>(ws + dq_bytes + row_bytes);
+  // d = 128 (128-query kernel): the row statistics as MMA operands, 32 B per padded row
+  const size_t aug_bytes = (d == 128 && FA_BWD_Q128) ? size_t(BH) * npad * 32 : 0;
+  p.aug = aug_bytes ? ws + dq_bytes + 2 * row_bytes : nullptr;
   p.BH = BH;
   p.N = N;
   p.Npad = int(npad);
@@ -423,8 +476,8 @@ int bwd_dispatch(const void* q, const void* k, const void* v, const void* o, con
   }
   if (p.gsplit > 1) {
     const size_t kv_bytes = round_up(size_t(p.BHkv) * size_t(N) * size_t(d) * 4, 256);
-    p.dk_acc = reinterpret_cast<float*>(ws + dq_bytes + 2 * row_bytes);
-    p.dv_acc = reinterpret_cast<float*>(ws + dq_bytes + 2 * row_bytes + kv_bytes);
+    p.dk_acc = reinterpret_cast<float*>(ws + dq_bytes + 2 * row_bytes + aug_bytes);
+    p.dv_acc = reinterpret_cast<float*>(ws + dq_bytes + 2 * row_bytes + aug_bytes + kv_bytes);
   }
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -513,6 +566,48 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   return FA_OK;
 }
 
+int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_scale, float k_scale,
+               float v_scale, void* o, float* lse, int B, int H, int N, int d, int causal,
+               float scale, void* stream) {
+  g_msg[0] = 0;
+  if (!q8 || !k8 || !v8 || !o || !lse) return fail(FA_ERR_INVALID_ARG, "null tensor pointer");
+  int rc = check_common(B, H, N, d, scale);
+  if (rc) return rc;
+  for (float x : {q_scale, k_scale, v_scale})
+    if (!std::isfinite(x) || !(x > 0.f))
+      return fail(FA_ERR_INVALID_ARG, "q_scale, k_scale and v_scale must be finite and > 0");
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || !aligned16(lse))
+    return fail(FA_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+  if ((rc = check_device())) return rc;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if ((rc = make_map_e4m3(&mq, q8, BH, N, d, 128))) return rc;
+  if ((rc = make_map_e4m3(&mk, k8, BH, N, d, 128))) return rc;
+  if ((rc = make_map_e4m3(&mv, v8, BH, N, d, 128))) return rc;
+  fattn::FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.Nq = N;
+  p.Nk = N;
+  p.off = 0;
+  p.H = H;
+  p.G = 1;
+  p.splits = 1;
+  p.kv_chunk = (N + 127) / 128;
+  p.Hkv = H;
+  p.scale_log2 = scale * q_scale * k_scale * 1.4426950408889634f;
+  p.limit_ns = wait_limit_ns();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return causal ? launch_fwd_fp8<64, true, 2>(mq, mk, mv, p, v_scale, BH, st)
+                  : launch_fwd_fp8<64, false, 2>(mq, mk, mv, p, v_scale, BH, st);
+  if (d == 128)
+    return causal ? launch_fwd_fp8<128, true, 2>(mq, mk, mv, p, v_scale, BH, st)
+                  : launch_fwd_fp8<128, false, 2>(mq, mk, mv, p, v_scale, BH, st);
+  return causal ? launch_fwd_fp8<256, true, 1>(mq, mk, mv, p, v_scale, BH, st)
+                : launch_fwd_fp8<256, false, 1>(mq, mk, mv, p, v_scale, BH, st);
+}
+
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
            int d, int causal, float scale, void* stream) {
   return fa_fwd_gqa(q, k, v, o, lse, B, H, H, N, d, causal, scale, stream);
@@ -524,7 +619,8 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   const size_t npad = round_up(size_t(N), 128);
   const size_t dq = round_up(bh * size_t(N) * size_t(d) * 4, 256);
   const size_t rows = round_up(bh * npad * 4, 256);
-  return dq + 2 * rows;
+  const size_t aug = (d == 128 && FA_BWD_Q128) ? bh * npad * 32 : 0;
+  return dq + 2 * rows + aug;
 }
 
 size_t fa_bwd_gqa_workspace_size(int B, int H, int H_kv, int N, int d) {

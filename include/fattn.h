@@ -67,7 +67,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 /*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for this shape:
  * an fp32 dQ accumulator [B,H,N,d] plus two fp32 row vectors [B,H,roundup(N,128)]
- * (the logsumexp in base 2 and D_i = sum_c dO_ic O_ic).  Returns 0 for invalid sizes.
+ * (the logsumexp in base 2 and D_i = sum_c dO_ic O_ic), and for d = 128 a further 32 bytes per
+ * padded row (the same statistics laid out as a tensor-core operand).  Returns 0 for invalid
+ * sizes.
  * The workspace is O(N) per head: no N x N buffer exists on any path.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
@@ -102,7 +104,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
  * GPU on which the library's kernels are loaded holds that array until the process exits.
  * Shapes whose fa_bwd_workspace_size exceeds it return FA_ERR_WORKSPACE before any launch
  * (for example B=8, H=12, N=1024, d=64 needs about 26 MB and fits; B=2, H=16, N=8192, d=128
- * needs 130 MB and does not).  The entry point calls no cudaMalloc, cudaFree or other allocating
+ * needs 145 MB and does not).  The entry point calls no cudaMalloc, cudaFree or other allocating
  * routine.
  *
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress,
@@ -120,6 +122,26 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
 int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                    const void* dO, void* dq, void* dk, void* dv,
                    int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * fa_fwd_fp8 -- forward pass on FP8 inputs, the low-precision forward the pages attribute to
+ * FlashAttention-3 (robocikowo.com "Flash Attention", the FA-3 entry; systems-analysis.info
+ * "FlashAttention (PL)", section "FlashAttention-3 (2024)"; dexblog.ro, the dtype row: FP8 in
+ * the forward).  The attended tensors are q_scale*Q8, k_scale*K8 and v_scale*V8:
+ *     O = softmax(scale * (q_scale Q8)(k_scale K8)^T [masked]) (v_scale V8),  L as for fa_fwd.
+ *   q8, k8, v8 : e4m3 codes [B, H, N, d], one byte per element (1 sign, 4 exponent bits with
+ *                bias 7, 3 mantissa bits; S.1111.111 is NaN and must not occur)
+ *   q_scale, k_scale, v_scale : per-tensor factors, finite and > 0 (else FA_ERR_INVALID_ARG)
+ *   o          : bfloat16 [B, H, N, d];  lse : float32 [B, H, N] (natural log, as for fa_fwd)
+ * Both GEMMs run on e4m3 operands with fp32 accumulation; the softmax weights are rounded to
+ * e4m3 (scaled so the largest weight of a row is 256, exactly representable) before they
+ * multiply V8, so O carries that rounding -- at most 2^-4 of sum_j P_ij |v_j| per element,
+ * usually far less -- while lse is computed from the fp32 exponentials.  Layout, alignment,
+ * ownership, streams and errors as for fa_fwd (no backward: the pages name FP8 for the forward).
+ */
+int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_scale, float k_scale,
+               float v_scale, void* o, float* lse, int B, int H, int N, int d, int causal,
+               float scale, void* stream);
 
 /*
  * Grouped-query attention (GQA): H query heads share H_kv key/value heads.  H_kv = 1 is the

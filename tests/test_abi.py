@@ -37,8 +37,11 @@ def test_version():
 def test_workspace_size_formula():
     B, H, N, d = 2, 16, 8192, 128
     npad = (N + 127) // 128 * 128
-    want = B * H * N * d * 4 + 2 * B * H * npad * 4
+    # fp32 dQ accumulator + two fp32 row vectors; d = 128 adds the row statistics as 32 bytes
+    # of MMA operand per padded row
+    want = B * H * N * d * 4 + 2 * B * H * npad * 4 + B * H * npad * 32
     assert fa.fa_bwd_workspace_size(B, H, N, d) == want
+    assert fa.fa_bwd_workspace_size(B, H, N, 64) == B * H * N * 64 * 4 + 2 * B * H * npad * 4
     # ragged N: the row vectors are padded to 128
     got = fa.fa_bwd_workspace_size(1, 1, 129, 64)
     assert got >= 129 * 64 * 4 + 2 * 256 * 4
@@ -60,6 +63,30 @@ def fwd(**kw):
     a = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, N=128, d=64, causal=0, scale=0.125, stream=None)
     a.update(kw)
     return fa.fa_fwd(**a)
+
+
+def fwd_fp8(**kw):
+    a = dict(q8=A, k8=A, v8=A, q_scale=0.01, k_scale=0.01, v_scale=0.01, o=A, lse=A, B=1, H=1,
+             N=128, d=64, causal=0, scale=0.125, stream=None)
+    a.update(kw)
+    return fa.fa_fwd_fp8(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q8=None), fa.FA_ERR_INVALID_ARG),
+    (dict(v8=None), fa.FA_ERR_INVALID_ARG),
+    (dict(N=0), fa.FA_ERR_INVALID_ARG),
+    (dict(d=32), fa.FA_ERR_UNSUPPORTED),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(q_scale=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(k_scale=-1.0), fa.FA_ERR_INVALID_ARG),
+    (dict(v_scale=float("inf")), fa.FA_ERR_INVALID_ARG),
+    (dict(k8=A + 1), fa.FA_ERR_MISALIGNED),
+    (dict(lse=A + 4), fa.FA_ERR_MISALIGNED),
+])
+def test_fwd_fp8_rejects(kw, code):
+    assert fwd_fp8(**kw) == code
+    assert fa.fa_last_error() != ""
 
 
 def bwd(**kw):

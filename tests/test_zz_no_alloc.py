@@ -50,7 +50,7 @@ def test_noalloc_matches_fa_bwd_twice(B, H, N, d, causal):
 
 
 def test_noalloc_rejects_shapes_beyond_the_scratch():
-    """The long-context shape needs ~130 MB of workspace: rejected on the host, nothing launched."""
+    """The long-context shape needs ~145 MB of workspace: rejected on the host, nothing launched."""
     A = 1 << 20
     need = fa.fa_bwd_workspace_size(2, 16, 8192, 128)
     assert need > fa.FA_NOALLOC_SCRATCH_BYTES
