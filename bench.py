@@ -68,6 +68,9 @@ def parse_args(argv=None):
                     help="B,H,N,d,causal override (profiling runs on a smaller case)")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="key/value heads per batch (grouped-query attention; default: H)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one line per workload: the GPT-2-small and BERT-large shapes and the 30 "
+                         "points of the B*H*N = 131072 sweep (fwd+bwd, bf16)")
     ap.add_argument("--fp8", action="store_true",
                     help="time the FP8 (e4m3) forward on the workload instead of the bf16 step")
     ap.add_argument("--decode", default=None,
@@ -642,10 +645,37 @@ def run_fp8(args):
     return 0
 
 
+def sweep_workloads():
+    """(name, B, H, N, d, causal) of every parity workload that has a fwd+bwd step, besides the
+    headline one: GPT-2-small shape, BERT-large shape, and the B*H*N = 131072 sweep."""
+    out = [("GPT-2-small-shaped causal fwd+bwd, B=8 H=12 N=1024 d=64 bf16", 8, 12, 1024, 64, True),
+           ("BERT-large-shaped non-causal fwd+bwd, B=16 H=16 N=512 d=64 bf16", 16, 16, 512, 64,
+            False)]
+    for pt in ai.sweep_points():
+        out.append((f"sweep point B*H*N=131072: B={pt['B']} H={pt['H']} N={pt['N']} d={pt['d']} "
+                    f"{'causal' if pt['causal'] else 'non-causal'} fwd+bwd bf16",
+                    pt["B"], pt["H"], pt["N"], pt["d"], pt["causal"]))
+    return out
+
+
+def run_sweep(args):
+    global WORKLOAD_NAME
+    args.no_cpu_baseline = True
+    args.e2e_steps = 0
+    for (name, B, H, N, d, causal) in sweep_workloads():
+        WORKLOAD.clear()
+        WORKLOAD.update(B=B, H=H, N=N, d=d, causal=causal)
+        WORKLOAD_NAME = name
+        run_gpu(args)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     if args.decode is not None:
         return run_decode(args)
     if args.fp8:

@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
     L.fa_version.restype = i
     L.fa_fwd_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, i, f, vp]
     L.fa_fwd_fp8.restype = i
+    L.fa_selftest_exp2_fma.argtypes = [vp, vp, i, vp]
+    L.fa_selftest_exp2_fma.restype = i
     L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
     L.fa_bwd_noalloc.restype = i
     L.fa_timer_enable.argtypes = [i]
@@ -115,6 +117,10 @@ def fa_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, d, causal
                stream) -> int:
     return lib().fa_fwd_fp8(q8, k8, v8, float(q_scale), float(k_scale), float(v_scale), o, lse,
                             B, H, N, d, int(causal), float(scale), stream)
+
+
+def fa_selftest_exp2_fma(x, y, n, stream) -> int:
+    return lib().fa_selftest_exp2_fma(x, y, n, stream)
 
 
 def fa_bwd_gqa_workspace_size(B, H, H_kv, N, d) -> int:

@@ -84,8 +84,8 @@ struct BwdQ128Cfg {
   static constexpr int DO_STAGES = 1;
   static constexpr int OFF_DO = OFF_Q + 2 * TILE;            // dO_i
   static constexpr int OFF_DS = OFF_DO + DO_STAGES * TILE;   // dS^T [2 q halves][128 keys][64 q]
-  static constexpr int OFF_STG = OFF_DS + TILE;              // dQ staging: one [64 q][64 d] f32
-  static constexpr int STG_BYTES = 64 * 64 * 4;
+  static constexpr int OFF_STG = OFF_DS + TILE;              // dQ staging: 4 x [32 q][32 d] f32
+  static constexpr int STG_BYTES = 4 * 32 * 32 * 4;
   // row-statistics operands of the ninth K step (no swizzle: 8-row x 16-byte core matrices,
   // 8-row groups 128 B apart, the second 8 K-elements AUG_LBO bytes on):
   //   AUG [2 stages][2 K halves: -L/s terms | -D terms][16 query groups][8 rows][8 bf16]
@@ -490,26 +490,24 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
     tc_fence_before();
   } else {
     // ================================================================ dQ drain warpgroup
-    // dQ^T (d on TMEM lanes, 128 query columns) -> x scale -> a [64 queries][64 d] fp32 staging
-    // block -> TMA bulk reduce-add into the accumulator, one (query half, d half) at a time:
-    // the two warps holding that d half fill the block, the others wait (rows past N are
-    // clipped by the tensor map; query halves wholly past N are skipped).  The whole dQ^T is
+    // dQ^T (d on TMEM lanes, 128 query columns) -> x scale -> shared staging -> TMA bulk
+    // reduce-add into the fp32 accumulator.  Each drain warp owns 32 d rows and its own 4 KB
+    // staging block ([32 queries][32 d]); it works through the step's four 32-query quarters on
+    // its own, with no barrier shared with the other drain warps: write a quarter, hand it to
+    // the TMA unit, and before the next one wait until that reduce has read the block (rows past
+    // N are clipped by the tensor map; quarters wholly past N are skipped).  The whole dQ^T is
     // read out of tensor memory first, so the MMA warp may reuse its columns at once.
     regs_inc<C::DQ_REGS>();
     const int wq = warp - C::DQ_WARP0;
-    const int tq = threadIdx.x - C::DQ_WARP0 * 32;  // 0..127
-    const bool issuer = tq == 0;
+    const bool issuer = lane == 0;
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
-    const int drow = wq * 32 + lane;                // d index == TMEM lane
-    float* slot = reinterpret_cast<float*>(smem + C::OFF_STG);
-    float* my_col = slot + (drow & 63);
+    float* wslot = reinterpret_cast<float*>(smem + C::OFF_STG) + wq * (32 * 32);
     if (issuer) tma_prefetch_desc(&tmdQ);
     BwdCursor cur(grp);
     for (int t = 0; t < nit; ++t) {
       const int i = cur.i, head = cur.head;
       cur.next();
-      // the four drain warps leave the loop together (they share named barriers below)
-      if (!named_bar_and(1, 128, W.wait_warp(BAR_DQF, t & 1, 60))) break;
+      if (!(W.wait_warp(BAR_DQF, t & 1, 60))) break;
       FA_TRACE_EV(60, t);
       tc_fence_after();
       uint32_t v[4][32];
@@ -522,25 +520,19 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       if (lane == 0) mbar_arrive(BAR_DQE);
       FA_TRACE_EV(61, t);
 #pragma unroll
-      for (int qh = 0; qh < 2; ++qh) {
-        const int row0 = i * C::BR + 64 * qh;
-        if (row0 >= p.N) break;  // uniform over the warpgroup
+      for (int qq = 0; qq < 4; ++qq) {
+        const int row0 = i * C::BR + 32 * qq;
+        if (row0 >= p.N) break;  // uniform over the warp
+        if (issuer) bulk_wait_group_read<0>();  // this warp's previous reduce has read the block
+        __syncwarp();
 #pragma unroll
-        for (int db = 0; db < 2; ++db) {
-          if (issuer) bulk_wait_group_read<0>();  // the previous reduce has read the block
-          named_bar_sync(1, 128);
-          if ((drow >> 6) == db) {  // warp-uniform
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              my_col[c * 64] = __uint_as_float(v[2 * qh + (c >> 5)][c & 31]) * p.scale;
-          }
-          fence_async_smem();
-          named_bar_sync(1, 128);
-          FA_TRACE_EV(62 + qh, t);
-          if (issuer) {
-            tma_reduce_add_3d(&tmdQ, smem_u32(slot), 64 * db, row0, head);
-            bulk_commit_group();
-          }
+        for (int c = 0; c < 32; ++c) wslot[c * 32 + lane] = __uint_as_float(v[qq][c]) * p.scale;
+        fence_async_smem();
+        __syncwarp();
+        FA_TRACE_EV(62, t);
+        if (issuer) {
+          tma_reduce_add_3d(&tmdQ, smem_u32(wslot), 32 * wq, row0, head);
+          bulk_commit_group();
         }
       }
     }

@@ -123,16 +123,16 @@ struct TimedLaunch {
   }
 };
 
-// fp32 [BH, N, d] map for the dQ accumulator: box 64 columns x 64 rows x 1 head, no swizzle
-// (the reduce-add source in shared memory is a dense [64][64] fp32 tile).
-int make_map_f32(CUtensorMap* m, void* base, int BH, int N, int d) {
+// fp32 [BH, N, d] map for the dQ accumulator: box `box` columns x `box` rows x 1 head, no
+// swizzle (the reduce-add source in shared memory is a dense [box][box] fp32 tile).
+int make_map_f32(CUtensorMap* m, void* base, int BH, int N, int d, int box = 64) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
   cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(N) * cuuint64_t(d) * 4};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t boxd[3] = {cuuint32_t(box), cuuint32_t(box), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, boxd, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled (f32) failed (%d)", int(r));
@@ -339,6 +339,7 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
                                       "register split");
     if ((rc = make_map(&mq, q, p.BH, p.N, D, CQ::BR))) return rc;
     if ((rc = make_map(&mdo, p.dO, p.BH, p.N, D, CQ::BR))) return rc;
+    if ((rc = make_map_f32(&mdq, p.dq_acc, p.BH, p.N, D, 32))) return rc;  // per-warp blocks
     dim3 grid(unsigned(p.BHkv) * unsigned(p.nkb) * unsigned(p.gsplit));
     {
       TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
@@ -606,6 +607,20 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_scale, fl
                   : launch_fwd_fp8<128, false, 2>(mq, mk, mv, p, v_scale, BH, st);
   return causal ? launch_fwd_fp8<256, true, 1>(mq, mk, mv, p, v_scale, BH, st)
                 : launch_fwd_fp8<256, false, 1>(mq, mk, mv, p, v_scale, BH, st);
+}
+
+int fa_selftest_exp2_fma(const float* x, float* y, int n, void* stream) {
+  g_msg[0] = 0;
+  if (!x || !y || n < 0) return fail(FA_ERR_INVALID_ARG, "null pointer or negative count");
+  if (n == 0) return FA_OK;
+  int rc = check_device();
+  if (rc) return rc;
+  const int threads = 256, pairs = (n + 1) / 2;
+  fattn::fa_selftest_exp2_fma_kernel<<<(pairs + threads - 1) / threads, threads, 0,
+                                       static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fa_selftest_exp2_fma launch");
+  return FA_OK;
 }
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,

@@ -30,6 +30,10 @@
 
 namespace fattn {
 
+// Self-test kernel for exp2_fma2 (used only by fa_selftest_exp2_fma).
+__global__ void fa_selftest_exp2_fma_kernel(const float* __restrict__ x, float* __restrict__ y,
+                                            int n);
+
 // D[tmem] (+)= A[smem] * B[smem]^T with e4m3 A and B (kind::f8f6f4), fp32 accumulate.
 __device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                           uint32_t idesc, uint32_t accumulate) {
@@ -64,6 +68,38 @@ __device__ __forceinline__ uint64_t sdesc_swz(uint32_t saddr, uint32_t lbo, uint
                                               uint32_t layout) {
   return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
          (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (uint64_t(layout) << 61);
+}
+
+// FA_FP8_POLY_MASK: bit e set sends the e-th group of four scores of every 32 through exp2_fma2
+// (the FMA pipe) instead of the MUFU unit; at the fp8 MMA rate the exponentials, not the tensor
+// core, bound the kernel, so moving a share of them to the FMA pipe shortens each softmax step.
+#ifndef FA_FP8_POLY_MASK
+#define FA_FP8_POLY_MASK 0x00
+#endif
+
+// 2^x for two values on the FMA pipe (paired fp32 instructions), after Cody and Waite's argument
+// reduction: n = round(x) by the 1.5 * 2^23 shifter (exact for |x| < 2^22), f = x - n in
+// [-1/2, 1/2], 2^f by a cubic, and n added to the exponent field.  The cubic's coefficients are
+// our own fit (exact_io_aware_43_b200/fit_exp2.py: least largest relative error on [-1/2, 1/2],
+// 7.5e-5; the GPU self-test checks the device result against that bound).  Inputs are clamped
+// at -126 (masked scores give 2^-126, which e4m3 rounding and the fp32 row sum both absorb).
+__device__ __forceinline__ void exp2_fma2(float x0, float x1, float& p0, float& p1) {
+  const float kShift = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t xc = f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = fadd2(xc, f2pack(kShift, kShift));
+  const uint64_t n = fadd2(t, f2pack(-kShift, -kShift));
+  const uint64_t f = ffma2(n, f2pack(-1.f, -1.f), xc);
+  uint64_t q = ffma2(f, f2pack(5.5171668530e-02f, 5.5171668530e-02f),
+                     f2pack(2.4261112511e-01f, 2.4261112511e-01f));
+  q = ffma2(q, f, f2pack(6.9326096773e-01f, 6.9326096773e-01f));
+  q = ffma2(q, f, f2pack(9.9992805719e-01f, 9.9992805719e-01f));
+  float q0, q1, t0, t1;
+  f2unpack(q, q0, q1);
+  f2unpack(t, t0, t1);
+  // the shifter leaves n in the low mantissa bits of t: shifting them up by 23 adds n to the
+  // exponent field of q
+  p0 = __uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(q0));
+  p1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(q1));
 }
 
 // Four fp32 values -> four e4m3 codes in one 32-bit word (value k in byte k), round to nearest
@@ -387,7 +423,16 @@ __global__ void __launch_bounds__(Fp8Cfg<D, NQT>::THREADS, 1)
                                   __uint_as_float(s[c][4 * e + 3])),
                            sc2, nm2),
                      x2, x3);
-            const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+            float p0, p1, p2, p3;
+            if ((FA_FP8_POLY_MASK >> e) & 1) {
+              exp2_fma2(x0, x1, p0, p1);
+              exp2_fma2(x2, x3, p2, p3);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+              p2 = ex2(x2);
+              p3 = ex2(x3);
+            }
             pk[8 * c + e] = pack_e4m3x4(p0, p1, p2, p3);
             sum2[e & 1] = fadd2(sum2[e & 1], fadd2(f2pack(p0, p1), f2pack(p2, p3)));
           }
@@ -455,6 +500,17 @@ __global__ void __launch_bounds__(Fp8Cfg<D, NQT>::THREADS, 1)
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+__global__ void fa_selftest_exp2_fma_kernel(const float* __restrict__ x, float* __restrict__ y,
+                                            int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    exp2_fma2(x[i], x[i + 1], y[i], y[i + 1]);
+  } else if (i < n) {
+    float d;
+    exp2_fma2(x[i], x[i], y[i], d);
   }
 }
 

@@ -231,6 +231,15 @@ const char* fa_last_error(void);
  */
 int fa_device_status(void* stream);
 
+/*
+ * fa_selftest_exp2_fma -- test support, not part of the attention computation: y[i] = 2^x[i] for
+ * n floats (device pointers) as computed by the FP8 forward's FMA-pipe exponential (argument
+ * reduction n = round(x), f = x - n, our own cubic for 2^f with relative error at most 7.5e-5 on
+ * [-1/2, 1/2]; inputs below -126 are clamped there).  Lets a test check the device function
+ * against exp2 with that bound.  Errors: FA_ERR_INVALID_ARG for null pointers or n < 0.
+ */
+int fa_selftest_exp2_fma(const float* x, float* y, int n, void* stream);
+
 /* Library version as major*10000 + minor*100 + patch. */
 int fa_version(void);
 

@@ -89,6 +89,12 @@ def test_fwd_fp8_rejects(kw, code):
     assert fa.fa_last_error() != ""
 
 
+def test_selftest_exp2_rejects_bad_arguments():
+    assert fa.fa_selftest_exp2_fma(None, A, 4, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_selftest_exp2_fma(A, A, -1, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_selftest_exp2_fma(A, A, 0, None) == fa.FA_OK  # nothing to do, nothing launched
+
+
 def bwd(**kw):
     a = dict(q=A, k=A, v=A, o=A, lse=A, dO=A, dq=A, dk=A, dv=A, B=1, H=1, N=128, d=64, causal=0,
              scale=0.125, workspace=A, workspace_bytes=1 << 30, stream=None)

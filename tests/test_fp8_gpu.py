@@ -87,3 +87,27 @@ def test_deterministic():
     o2, l2 = fa.forward_fp8(dev["q"], dev["k"], dev["v"], *sc, True)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fma_pipe_exp2_within_its_bound():
+    """The FP8 softmax's FMA-pipe exponential (fa_selftest_exp2_fma runs the device function)
+    against exp2 in fp64: relative error at most 7.5e-5 (the fitted cubic's bound on [-1/2, 1/2],
+    plus float32 rounding of the reduction and the result) wherever the result is a normal float,
+    and inputs at or below -126 clamp to 2^-126."""
+    import torch
+    import exact_io_aware_43_b200 as fa
+    x = np.concatenate([np.linspace(-125.0, 20.0, 1 << 20), np.array([0.0, 8.0, -1.0, 0.5, -0.5]),
+                        np.random.default_rng(0).uniform(-30.0, 8.5, 1 << 18)]).astype(np.float32)
+    xd = torch.from_numpy(x).cuda()
+    y = torch.empty_like(xd)
+    assert fa.fa_selftest_exp2_fma(xd.data_ptr(), y.data_ptr(), x.size,
+                                   torch.cuda.current_stream().cuda_stream) == fa.FA_OK
+    torch.cuda.synchronize()
+    ref = np.exp2(x.astype(np.float64))
+    rel = np.abs(y.cpu().numpy().astype(np.float64) / ref - 1.0)
+    assert rel.max() <= 7.5e-5 + 2.4e-7, rel.max()
+    low = torch.tensor([-126.0, -200.0, -1e30], device="cuda")
+    out = torch.empty_like(low)
+    assert fa.fa_selftest_exp2_fma(low.data_ptr(), out.data_ptr(), 3, None) == fa.FA_OK
+    torch.cuda.synchronize()
+    assert np.allclose(out.cpu().numpy(), 2.0 ** -126, rtol=1e-4, atol=0)
