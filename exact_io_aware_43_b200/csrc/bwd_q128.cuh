@@ -1,4 +1,4 @@
-// bwd_q128.cuh -- attention backward main kernel for d = 128 with 128-query steps (sm_100a).
+// bwd_q128.cuh -- attention backward main kernel for d = 64 and 128 with 128-query steps (sm_100a).
 //
 // Same mathematics as fa_bwd_kernel (robocikowo.com "Flash Attention": the backward recomputes
 // P from the saved L; the gradient formulas are those of the definition), with a different
@@ -48,12 +48,18 @@
 
 namespace fattn {
 
+template <int D_>
 struct BwdQ128Cfg {
-  static constexpr int D = 128;
+  static constexpr int D = D_;            // 64 or 128
+  static constexpr int KB = D / 64;       // 128-byte swizzle blocks across d
   static constexpr int BC = 128;          // keys per CTA
   static constexpr int BR = 128;          // queries per step
   static constexpr int BLK = 128 * 128;   // one 64-column (128-byte-row) block of a 128-row tile
-  static constexpr int TILE = 2 * BLK;    // a 128 x 128 bf16 tile
+  static constexpr int TILE = KB * BLK;   // a 128-row x D bf16 tile (K_j, V_j, Q_i, dO_i)
+  static constexpr int DS_TILE = 2 * BLK; // dS^T: [2 query halves][128 keys][64 queries] bf16
+  // dQ^T has d on its rows: M = 128 puts row 32w + i in lane i of warp w's lane quarter; M = 64
+  // puts rows 16w .. 16w + 15 in lanes 0 .. 15 of it (lanes 16 .. 31 hold nothing)
+  static constexpr int DW = D == 128 ? 32 : 16;  // d rows per drain warp
   static constexpr int THREADS = 512;
   static constexpr int CMP_WARPS = 8;
   static constexpr int DQ_WARP0 = 8;
@@ -75,7 +81,7 @@ struct BwdQ128Cfg {
   static_assert(2 * 128 * CMP_REGS + 128 * DQ_REGS + 128 * CTRL_REGS <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
   // tensor memory columns
-  static constexpr int T_S = 0, T_DP = 128, T_DQ = 128, T_DV = 256, T_DK = 384;
+  static constexpr int T_S = 0, T_DP = 128, T_DQ = 128, T_DV = 256, T_DK = 256 + D;
   static constexpr int TMEM_COLS = 512;
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int OFF_K = 0;
@@ -84,8 +90,8 @@ struct BwdQ128Cfg {
   static constexpr int DO_STAGES = 1;
   static constexpr int OFF_DO = OFF_Q + 2 * TILE;            // dO_i
   static constexpr int OFF_DS = OFF_DO + DO_STAGES * TILE;   // dS^T [2 q halves][128 keys][64 q]
-  static constexpr int OFF_STG = OFF_DS + TILE;              // dQ staging: 4 x [32 q][32 d] f32
-  static constexpr int STG_BYTES = 4 * 32 * 32 * 4;
+  static constexpr int OFF_STG = OFF_DS + DS_TILE;           // dQ staging: 4 x [32 q][DW d] f32
+  static constexpr int STG_BYTES = 4 * 32 * DW * 4;
   // row-statistics operands of the ninth K step (no swizzle: 8-row x 16-byte core matrices,
   // 8-row groups 128 B apart, the second 8 K-elements AUG_LBO bytes on):
   //   AUG [2 stages][2 K halves: -L/s terms | -D terms][16 query groups][8 rows][8 bf16]
@@ -107,8 +113,8 @@ struct BwdQ128Cfg {
   static_assert(NBAR * 8 <= 160, "barrier area");
   static_assert(SMEM_NEED <= SMEM_MAX, "shared memory budget");
   static constexpr uint32_t IDESC_ST = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
-  static constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, 0, 1);  // dV, dK (A in TMEM)
-  static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, 128, 1, 1);  // dQ^T = K^T dS^T
+  static constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A in TMEM)
+  static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(D, 128, 1, 1);    // dQ^T = K^T dS^T
 };
 
 // Descriptor of a no-swizzle K-major operand (layout code 0): core matrices of 8 rows x 16
@@ -118,14 +124,14 @@ __device__ __forceinline__ uint64_t sdesc_interleave(uint32_t saddr, uint32_t lb
          (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
-template <bool CAUSAL>
-__global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
     fa_bwd_kernel_q128(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmdO,
                        const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
-  using C = BwdQ128Cfg;
+  using C = BwdQ128Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the swizzled tiles need a 1024-byte-aligned base; with the largest layouts there is less
   // than 1 KB of slack, so a base that cannot be aligned within it is reported, not used
@@ -214,7 +220,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
       mbar_arrive_expect_tx(BAR_KV, 2 * C::TILE);
-      for (int kb = 0; kb < 2; ++kb) {
+      for (int kb = 0; kb < C::KB; ++kb) {
         tma_load_3d(sbase + C::OFF_K + kb * C::BLK, &tmK, BAR_KV, kb * 64, k0, kvh);
         tma_load_3d(sbase + C::OFF_V + kb * C::BLK, &tmV, BAR_KV, kb * 64, k0, kvh);
       }
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
         // Q_i and its row-statistics operand into stage s once dK of step t-2 has released it
         if (!W.wait(BAR_QE(s), ((t >> 1) & 1) ^ 1, 31)) break;
         mbar_arrive_expect_tx(BAR_QF(s), C::TILE + C::AUG_BYTES);
-        for (int kb = 0; kb < 2; ++kb)
+        for (int kb = 0; kb < C::KB; ++kb)
           tma_load_3d(sbase + C::OFF_Q + s * C::TILE + kb * C::BLK, &tmQ, BAR_QF(s), kb * 64,
                       i * C::BR, head);
         const size_t aoff = (size_t(head) * (p.Npad / C::BR) + size_t(i)) * C::AUG_BYTES;
@@ -239,7 +245,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
         const int sd = t % DS_;
         if (!W.wait(BAR_DOE(sd), ((t / DS_) & 1) ^ 1, 32)) break;
         mbar_arrive_expect_tx(BAR_DOF(sd), C::TILE);
-        for (int kb = 0; kb < 2; ++kb)
+        for (int kb = 0; kb < C::KB; ++kb)
           tma_load_3d(sbase + C::OFF_DO + sd * C::TILE + kb * C::BLK, &tmdO, BAR_DOF(sd), kb * 64,
                       i * C::BR, head);
         ++td;
@@ -263,7 +269,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
       auto issue_st = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base, uint32_t ones_addr,
                           uint32_t aug_addr) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
           mma_ss(tmem + d_col, sdesc_sw128(a_base + off, 16, 1024),
                  sdesc_sw128(b_base + off, 16, 1024), C::IDESC_ST, kk > 0 ? 1u : 0u);
@@ -501,7 +507,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
     const int wq = warp - C::DQ_WARP0;
     const bool issuer = lane == 0;
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
-    float* wslot = reinterpret_cast<float*>(smem + C::OFF_STG) + wq * (32 * 32);
+    float* wslot = reinterpret_cast<float*>(smem + C::OFF_STG) + wq * (32 * C::DW);
     if (issuer) tma_prefetch_desc(&tmdQ);
     BwdCursor cur(grp);
     for (int t = 0; t < nit; ++t) {
@@ -525,13 +531,16 @@ __global__ void __launch_bounds__(BwdQ128Cfg::THREADS, 1)
         if (row0 >= p.N) break;  // uniform over the warp
         if (issuer) bulk_wait_group_read<0>();  // this warp's previous reduce has read the block
         __syncwarp();
+        if (lane < C::DW) {  // d row DW * wq + lane (see DW)
 #pragma unroll
-        for (int c = 0; c < 32; ++c) wslot[c * 32 + lane] = __uint_as_float(v[qq][c]) * p.scale;
+          for (int c = 0; c < 32; ++c)
+            wslot[c * C::DW + lane] = __uint_as_float(v[qq][c]) * p.scale;
+        }
         fence_async_smem();
         __syncwarp();
         FA_TRACE_EV(62, t);
         if (issuer) {
-          tma_reduce_add_3d(&tmdQ, smem_u32(wslot), 32 * wq, row0, head);
+          tma_reduce_add_3d(&tmdQ, smem_u32(wslot), C::DW * wq, row0, head);
           bulk_commit_group();
         }
       }

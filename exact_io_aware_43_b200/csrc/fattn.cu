@@ -123,14 +123,15 @@ struct TimedLaunch {
   }
 };
 
-// fp32 [BH, N, d] map for the dQ accumulator: box `box` columns x `box` rows x 1 head, no
-// swizzle (the reduce-add source in shared memory is a dense [box][box] fp32 tile).
-int make_map_f32(CUtensorMap* m, void* base, int BH, int N, int d, int box = 64) {
+// fp32 [BH, N, d] map for the dQ accumulator: box `box_cols` columns x `box_rows` rows x 1 head,
+// no swizzle (the reduce-add source in shared memory is a dense [box_rows][box_cols] fp32 tile).
+int make_map_f32(CUtensorMap* m, void* base, int BH, int N, int d, int box_cols = 64,
+                 int box_rows = 64) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
   cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(N) * cuuint64_t(d) * 4};
-  cuuint32_t boxd[3] = {cuuint32_t(box), cuuint32_t(box), 1};
+  cuuint32_t boxd[3] = {cuuint32_t(box_cols), cuuint32_t(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, boxd, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -294,7 +295,7 @@ int launch_fwd_fp8(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// d = 128 backward: 128-query steps (fa_bwd_kernel_q128); 0 selects the 64-query kernel.
+// d = 64 and 128 backward: 128-query steps (fa_bwd_kernel_q128); 0 selects the 64-query kernel.
 #ifndef FA_BWD_Q128
 #define FA_BWD_Q128 1
 #endif
@@ -317,10 +318,10 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fa_bwd preprocess launch");
-  if (D == 128 && FA_BWD_Q128) {
-    // d = 128: 128-query steps (every GEMM of a step is 128 x 128 x 128)
-    using CQ = fattn::BwdQ128Cfg;
-    auto kq = fattn::fa_bwd_kernel_q128<CAUSAL>;
+  if ((D == 128 || D == 64) && FA_BWD_Q128) {
+    // d = 64, 128: 128-query steps (every GEMM of a step is 128 x 128 x d or 128 x d x 128)
+    using CQ = fattn::BwdQ128Cfg<(D == 64 ? 64 : 128)>;
+    auto kq = fattn::fa_bwd_kernel_q128<(D == 64 ? 64 : 128), CAUSAL>;
     if ((rc = set_smem(kq, CQ::SMEM_BYTES))) return rc;
     // setmaxnreg.inc draws on the registers the CTA was launched with: refuse a build whose
     // launch allocation is below the kernel's register split
@@ -339,7 +340,7 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
                                       "register split");
     if ((rc = make_map(&mq, q, p.BH, p.N, D, CQ::BR))) return rc;
     if ((rc = make_map(&mdo, p.dO, p.BH, p.N, D, CQ::BR))) return rc;
-    if ((rc = make_map_f32(&mdq, p.dq_acc, p.BH, p.N, D, 32))) return rc;  // per-warp blocks
+    if ((rc = make_map_f32(&mdq, p.dq_acc, p.BH, p.N, D, CQ::DW, 32))) return rc;  // per warp
     dim3 grid(unsigned(p.BHkv) * unsigned(p.nkb) * unsigned(p.gsplit));
     {
       TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
@@ -443,8 +444,8 @@ int bwd_dispatch(const void* q, const void* k, const void* v, const void* o, con
   p.dq_acc = reinterpret_cast<float*>(ws);
   p.L2 = reinterpret_cast<float*>(ws + dq_bytes);
   p.Drow = reinterpret_cast<float*>(ws + dq_bytes + row_bytes);
-  // d = 128 (128-query kernel): the row statistics as MMA operands, 32 B per padded row
-  const size_t aug_bytes = (d == 128 && FA_BWD_Q128) ? size_t(BH) * npad * 32 : 0;
+  // d = 64, 128 (128-query kernel): the row statistics as MMA operands, 32 B per padded row
+  const size_t aug_bytes = ((d == 128 || d == 64) && FA_BWD_Q128) ? size_t(BH) * npad * 32 : 0;
   p.aug = aug_bytes ? ws + dq_bytes + 2 * row_bytes : nullptr;
   p.BH = BH;
   p.N = N;
@@ -634,7 +635,7 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   const size_t npad = round_up(size_t(N), 128);
   const size_t dq = round_up(bh * size_t(N) * size_t(d) * 4, 256);
   const size_t rows = round_up(bh * npad * 4, 256);
-  const size_t aug = (d == 128 && FA_BWD_Q128) ? bh * npad * 32 : 0;
+  const size_t aug = ((d == 128 || d == 64) && FA_BWD_Q128) ? bh * npad * 32 : 0;
   return dq + 2 * rows + aug;
 }
 

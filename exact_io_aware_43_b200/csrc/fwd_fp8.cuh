@@ -73,8 +73,10 @@ __device__ __forceinline__ uint64_t sdesc_swz(uint32_t saddr, uint32_t lbo, uint
 // FA_FP8_POLY_MASK: bit e set sends the e-th group of four scores of every 32 through exp2_fma2
 // (the FMA pipe) instead of the MUFU unit; at the fp8 MMA rate the exponentials, not the tensor
 // core, bound the kernel, so moving a share of them to the FMA pipe shortens each softmax step.
+// Measured on the long-context causal workload (TFLOP/s): none 1128, groups 2 and 5 (a quarter)
+// 1157, groups 1, 4, 7 1125, every other group 1052 (the issue slots then bind).
 #ifndef FA_FP8_POLY_MASK
-#define FA_FP8_POLY_MASK 0x00
+#define FA_FP8_POLY_MASK 0x24
 #endif
 
 // 2^x for two values on the FMA pipe (paired fp32 instructions), after Cody and Waite's argument

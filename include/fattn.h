@@ -67,8 +67,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 /*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for this shape:
  * an fp32 dQ accumulator [B,H,N,d] plus two fp32 row vectors [B,H,roundup(N,128)]
- * (the logsumexp in base 2 and D_i = sum_c dO_ic O_ic), and for d = 128 a further 32 bytes per
- * padded row (the same statistics laid out as a tensor-core operand).  Returns 0 for invalid
+ * (the logsumexp in base 2 and D_i = sum_c dO_ic O_ic), and for d = 64 and 128 a further 32
+ * bytes per padded row (the same statistics laid out as a tensor-core operand).  Returns 0 for invalid
  * sizes.
  * The workspace is O(N) per head: no N x N buffer exists on any path.
  */
@@ -103,7 +103,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
  * The scratch is a file-scope static device array of FA_NOALLOC_SCRATCH_BYTES (32 MiB).  Every
  * GPU on which the library's kernels are loaded holds that array until the process exits.
  * Shapes whose fa_bwd_workspace_size exceeds it return FA_ERR_WORKSPACE before any launch
- * (for example B=8, H=12, N=1024, d=64 needs about 26 MB and fits; B=2, H=16, N=8192, d=128
+ * (for example B=8, H=12, N=1024, d=64 needs about 29 MB and fits; B=2, H=16, N=8192, d=128
  * needs 145 MB and does not).  The entry point calls no cudaMalloc, cudaFree or other allocating
  * routine.
  *

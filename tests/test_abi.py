@@ -37,11 +37,13 @@ def test_version():
 def test_workspace_size_formula():
     B, H, N, d = 2, 16, 8192, 128
     npad = (N + 127) // 128 * 128
-    # fp32 dQ accumulator + two fp32 row vectors; d = 128 adds the row statistics as 32 bytes
-    # of MMA operand per padded row
+    # fp32 dQ accumulator + two fp32 row vectors; d = 64 and 128 add the row statistics as 32
+    # bytes of MMA operand per padded row
     want = B * H * N * d * 4 + 2 * B * H * npad * 4 + B * H * npad * 32
     assert fa.fa_bwd_workspace_size(B, H, N, d) == want
-    assert fa.fa_bwd_workspace_size(B, H, N, 64) == B * H * N * 64 * 4 + 2 * B * H * npad * 4
+    assert fa.fa_bwd_workspace_size(B, H, N, 64) == B * H * N * 64 * 4 + 2 * B * H * npad * 4 + \
+        B * H * npad * 32
+    assert fa.fa_bwd_workspace_size(B, H, N, 256) == B * H * N * 256 * 4 + 2 * B * H * npad * 4
     # ragged N: the row vectors are padded to 128
     got = fa.fa_bwd_workspace_size(1, 1, 129, 64)
     assert got >= 129 * 64 * 4 + 2 * 256 * 4
