@@ -69,6 +69,10 @@ def lib() -> ctypes.CDLL:
     L.fa_version.restype = i
     L.fa_fwd_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, i, f, vp]
     L.fa_fwd_fp8.restype = i
+    L.fa_fwd_partial.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp]
+    L.fa_fwd_partial.restype = i
+    L.fa_merge_partials.argtypes = [vp, vp, i, vp, vp, ctypes.c_longlong, i, vp]
+    L.fa_merge_partials.restype = i
     L.fa_selftest_exp2_fma.argtypes = [vp, vp, i, vp]
     L.fa_selftest_exp2_fma.restype = i
     L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
@@ -117,6 +121,16 @@ def fa_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, d, causal
                stream) -> int:
     return lib().fa_fwd_fp8(q8, k8, v8, float(q_scale), float(k_scale), float(v_scale), o, lse,
                             B, H, N, d, int(causal), float(scale), stream)
+
+
+def fa_fwd_partial(q, k, v, o_part, lse_part, B, H, H_kv, Nq, Nk, d, causal, scale,
+                   stream) -> int:
+    return lib().fa_fwd_partial(q, k, v, o_part, lse_part, B, H, H_kv, Nq, Nk, d, int(causal),
+                                float(scale), stream)
+
+
+def fa_merge_partials(o_parts, lse_parts, n_parts, o, lse, rows, d, stream) -> int:
+    return lib().fa_merge_partials(o_parts, lse_parts, n_parts, o, lse, rows, d, stream)
 
 
 def fa_selftest_exp2_fma(x, y, n, stream) -> int:

@@ -46,6 +46,12 @@
 #define FA_BWDQ_DK_SS 1
 #endif
 
+// FA_BWDQ_POLY_MASK: bit g set computes the exponentials of query columns [8g, 8g+8) of every 64
+// on the FMA pipe (exp2_fma2) instead of the MUFU unit.
+#ifndef FA_BWDQ_POLY_MASK
+#define FA_BWDQ_POLY_MASK 0x00
+#endif
+
 namespace fattn {
 
 template <int D_>
@@ -419,7 +425,13 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
                               __uint_as_float(sv[c >> 5][(c & 31) + 1])),
                        sl2),
                  x0, x1);
-        float p0 = ex2(x0), p1 = ex2(x1);
+        float p0, p1;
+        if ((FA_BWDQ_POLY_MASK >> (c2 >> 2)) & 1) {
+          exp2_fma2(x0, x1, p0, p1);
+        } else {
+          p0 = ex2(x0);
+          p1 = ex2(x1);
+        }
         if (need_mask) {
           p0 = (key_ok && (!CAUSAL || r <= c0 + c)) ? p0 : 0.f;
           p1 = (key_ok && (!CAUSAL || r <= c0 + c + 1)) ? p1 : 0.f;

@@ -391,7 +391,7 @@ int effective_splits(int Nk, int splits) {
 // go to o_part / lse_part (see FwdParams) instead of o / lse.
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, float* o_part,
                float* lse_part, int B, int H, int H_kv, int Nq, int Nk, int d, bool causal,
-               float scale, int splits, bool pack, cudaStream_t st) {
+               float scale, int splits, bool pack, cudaStream_t st, bool partials = false) {
   int rc;
   const int BH = B * H;
   const int G = H / H_kv;
@@ -403,8 +403,8 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
   fattn::FwdParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
-  p.o_part = splits > 1 ? o_part : nullptr;
-  p.lse_part = splits > 1 ? lse_part : nullptr;
+  p.o_part = (splits > 1 || partials) ? o_part : nullptr;
+  p.lse_part = (splits > 1 || partials) ? lse_part : nullptr;
   p.Nq = Nq;
   p.Nk = Nk;
   p.off = Nk - Nq;
@@ -416,12 +416,22 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
   p.Hkv = H_kv;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.limit_ns = wait_limit_ns();
-  if (d == 64)
+  // packed query heads (decoding) fill one query tile only: the one-tile configuration, whose
+  // freed second query buffer deepens the K/V ring
+  if (d == 64) {
+    if (pack)
+      return causal ? launch_fwd<64, true, 1>(mq, mk, mv, p, BH, st)
+                    : launch_fwd<64, false, 1>(mq, mk, mv, p, BH, st);
     return causal ? launch_fwd<64, true, 2>(mq, mk, mv, p, BH, st)
                   : launch_fwd<64, false, 2>(mq, mk, mv, p, BH, st);
-  if (d == 128)
+  }
+  if (d == 128) {
+    if (pack)
+      return causal ? launch_fwd<128, true, 1>(mq, mk, mv, p, BH, st)
+                    : launch_fwd<128, false, 1>(mq, mk, mv, p, BH, st);
     return causal ? launch_fwd<128, true, 2>(mq, mk, mv, p, BH, st)
                   : launch_fwd<128, false, 2>(mq, mk, mv, p, BH, st);
+  }
   return causal ? launch_fwd<256, true, 1>(mq, mk, mv, p, BH, st)
                 : launch_fwd<256, false, 1>(mq, mk, mv, p, BH, st);
 }
@@ -608,6 +618,54 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_scale, fl
                   : launch_fwd_fp8<128, false, 2>(mq, mk, mv, p, v_scale, BH, st);
   return causal ? launch_fwd_fp8<256, true, 1>(mq, mk, mv, p, v_scale, BH, st)
                 : launch_fwd_fp8<256, false, 1>(mq, mk, mv, p, v_scale, BH, st);
+}
+
+int fa_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                   int B, int H, int H_kv, int Nq, int Nk, int d, int causal, float scale,
+                   void* stream) {
+  g_msg[0] = 0;
+  if (!q || !k || !v || !o_part || !lse_part) return fail(FA_ERR_INVALID_ARG, "null tensor pointer");
+  int rc = check_common(B, H, Nq, d, scale);
+  if (rc) return rc;
+  if ((rc = check_common(B, H, Nk, d, scale))) return rc;
+  if ((rc = check_groups(H, H_kv))) return rc;
+  if (causal && Nq > Nk)
+    return fail(FA_ERR_INVALID_ARG, "causal attention needs Nq <= Nk (got Nq=%d, Nk=%d)", Nq, Nk);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part) || !aligned16(lse_part))
+    return fail(FA_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+  if ((rc = check_device())) return rc;
+  return fwd_launch(q, k, v, nullptr, nullptr, o_part, lse_part, B, H, H_kv, Nq, Nk, d,
+                    causal != 0, scale, 1, true, static_cast<cudaStream_t>(stream), true);
+}
+
+int fa_merge_partials(const float* o_parts, const float* lse_parts, int n_parts, void* o,
+                      float* lse, long long rows, int d, void* stream) {
+  g_msg[0] = 0;
+  if (!o_parts || !lse_parts || !o || !lse) return fail(FA_ERR_INVALID_ARG, "null tensor pointer");
+  if (n_parts < 1 || rows < 1)
+    return fail(FA_ERR_INVALID_ARG, "n_parts and rows must be >= 1 (got %d, %lld)", n_parts, rows);
+  if (d != 64 && d != 128 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dim d=%d is not supported (64, 128 or 256)", d);
+  if (!aligned16(o_parts) || !aligned16(lse_parts) || !aligned16(o) || !aligned16(lse))
+    return fail(FA_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+  int rc = check_device();
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long want = (rows + 7) / 8;
+  const int blocks = int(want < sm_count() * 16ll ? want : sm_count() * 16ll);
+  {
+    TimedLaunch tl(FA_KERNEL_FWD_MERGE, st);
+    auto* ob = static_cast<__nv_bfloat16*>(o);
+    if (d == 64)
+      fattn::fa_fwd_merge_kernel<64><<<blocks, 256, 0, st>>>(o_parts, lse_parts, ob, lse, n_parts, rows);
+    else if (d == 128)
+      fattn::fa_fwd_merge_kernel<128><<<blocks, 256, 0, st>>>(o_parts, lse_parts, ob, lse, n_parts, rows);
+    else
+      fattn::fa_fwd_merge_kernel<256><<<blocks, 256, 0, st>>>(o_parts, lse_parts, ob, lse, n_parts, rows);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fa_merge_partials launch");
+  return FA_OK;
 }
 
 int fa_selftest_exp2_fma(const float* x, float* y, int n, void* stream) {

@@ -37,6 +37,11 @@
 #ifndef FA_FWD_RSUM
 #define FA_FWD_RSUM 2
 #endif
+// FA_FWD_POLY_MASK: bit g set computes the exponentials of scores [4g, 4g+4) of every 32 on the
+// FMA pipe (exp2_fma2) instead of the MUFU unit.
+#ifndef FA_FWD_POLY_MASK
+#define FA_FWD_POLY_MASK 0x00
+#endif
 #ifndef FA_FWD_RESCALE
 #define FA_FWD_RESCALE 8.0f
 #endif
@@ -81,7 +86,10 @@ struct FwdCfg {
   static constexpr int KB = D / 64;              // 128-byte swizzle blocks across d
   static constexpr int QTILE_BYTES = BM * D * 2;
   static constexpr int KVTILE_BYTES = BN * D * 2;
-  static constexpr int STAGES = (D == 64) ? 4 : (D == 128 ? 2 : 1);
+  // K/V ring depth.  With one query tile (d = 256, and packed decoding at d = 64 / 128, where
+  // a second tile would stay empty) the freed query buffer holds more stages.
+  static constexpr int STAGES = NQT == 1 ? (D == 64 ? 6 : (D == 128 ? 3 : 1))
+                                         : (D == 64 ? 4 : (D == 128 ? 2 : 1));
   static constexpr int SOFTMAX_WARPS = 4 * NQT;
   static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;  // control warpgroup: producer, MMA, 2 idle
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
@@ -468,6 +476,134 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       float m = -INFINITY;
       float l = 0.f;   // sum of the fp32 exponentials (for L)
       float lr = 0.f;  // sum of the bf16-rounded exponentials (divides O)
+      if (SPLIT && packed && p.pack * p.Nq <= 16) {
+        // ---- decoding: at most 16 valid rows, all in lanes 0-15 of the first warp.  Each row is
+        // spread over four threads (the 16-lane TMEM shapes), so a row's exponentials take a
+        // quarter of the time they would on one thread; the other three warps only keep the
+        // barrier phases in step.  Row statistics live in the four threads of the row and are
+        // combined with two shuffles; at the end they move to thread = row for the epilogue.
+        const bool worker = (warp & 3) == 0;
+        const bool two_sets = p.pack * p.Nq > 8;  // rows 8-15 in use (second register set)
+        const int g4 = lane >> 2, c2 = 2 * (lane & 3);
+        float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f, rA = 0.f, rB = 0.f;
+        for (int j = 0; j < n; ++j, ++tit) {
+          if (!(ok = W.wait_warp(BAR_SF(t), tit & 1, 20))) break;
+          tc_fence_after();
+          float alphaA = 1.f, alphaB = 1.f;
+          if (worker) {
+            uint32_t sv[64];
+            tmem_ld16x256b_x16(tS, sv);
+            tmem_wait_ld64(sv);
+            const int key0 = (un.kt0 + j) * C::BN;
+            uint32_t wd[32];
+#pragma unroll
+            for (int set = 0; set < 2; ++set) {
+              if (set == 1 && !two_sets) {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) wd[2 * k + 1] = 0u;
+                break;
+              }
+              const int lrow = g4 + 8 * set;  // tile row == lane
+              const int qi = lrow % p.Nq;
+              const int lim = CAUSAL ? min(qi + p.off, p.Nk - 1) - key0 : (p.Nk - 1) - key0;
+              float mx = -INFINITY;
+#pragma unroll
+              for (int k = 0; k < 16; ++k)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  if (8 * k + c2 + e > lim) sv[4 * k + 2 * set + e] = __float_as_uint(-INFINITY);
+                  mx = fmaxf(mx, __uint_as_float(sv[4 * k + 2 * set + e]));
+                }
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+              float& mr = set ? mB : mA;
+              const float m_tile = mx * p.scale_log2;
+              const float m_use = (j == 0 || m_tile > mr + kRescale) ? fmaxf(mr, m_tile) : mr;
+              const float alpha = (j == 0 || m_use == mr) ? 1.f : ex2(mr - m_use);
+              const float m_ref = m_use == -INFINITY ? 0.f : m_use;
+              const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
+              const uint64_t nm2 = f2pack(-m_ref, -m_ref);
+              uint64_t sx = 0ull;
+              float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+              for (int k = 0; k < 16; ++k) {
+                float x0, x1;
+                f2unpack(ffma2(f2pack(__uint_as_float(sv[4 * k + 2 * set]),
+                                      __uint_as_float(sv[4 * k + 2 * set + 1])),
+                               sc2, nm2),
+                         x0, x1);
+                const float p0 = ex2(x0), p1 = ex2(x1);
+                const uint32_t pk = pack_bf16(p0, p1);
+                wd[2 * k + set] = pk;
+                sx = fadd2(sx, f2pack(p0, p1));
+                if (C::EXTRA == 0) add_bf16pair_f32(pk, s0, s1);
+              }
+              float a0, a1;
+              f2unpack(sx, a0, a1);
+              float ls = a0 + a1, rs = s0 + s1;
+              ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+              ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+              rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+              rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+              if (set == 0) {
+                lA = lA * alpha + ls;
+                rA = rA * alpha + rs;
+                alphaA = alpha;
+              } else {
+                lB = lB * alpha + ls;
+                rB = rB * alpha + rs;
+                alphaB = alpha;
+              }
+              mr = m_use;
+            }
+            // P~ (bf16 pairs) over the first 64 columns of S_t, rows 0-15
+            tmem_st16x128b_x16(tS, wd);
+            // the row factors to thread = row for the 32x32b rescale of O
+            const float aA = __shfl_sync(0xffffffffu, alphaA, 4 * (lane & 7));
+            const float aB = __shfl_sync(0xffffffffu, alphaB, 4 * (lane & 7));
+            const float alpha = lane < 8 ? aA : (lane < 16 ? aB : 1.f);
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+              if (!(ok = W.wait_warp(BAR_OD(t), (tit - 1) & 1, 21))) {
+                tmem_wait_st();
+                break;
+              }
+              tc_fence_after();
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + 32 * c, o);
+                tmem_wait_ld(o);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                tmem_st32(tO + 32 * c, o);
+              }
+              if constexpr (C::EXTRA > 0) {
+                uint32_t o[16];
+                tmem_ld16(tO + D, o);
+                tmem_wait_ld16(o);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                tmem_st16(tO + D, o);
+              }
+            }
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR_PF(t));
+        }
+        if (!ok) break;
+        // row statistics to thread = row (lanes 0-15 of the first warp) for the epilogue
+        const float vmA = __shfl_sync(0xffffffffu, mA, 4 * (lane & 7));
+        const float vmB = __shfl_sync(0xffffffffu, mB, 4 * (lane & 7));
+        const float vlA = __shfl_sync(0xffffffffu, lA, 4 * (lane & 7));
+        const float vlB = __shfl_sync(0xffffffffu, lB, 4 * (lane & 7));
+        const float vrA = __shfl_sync(0xffffffffu, rA, 4 * (lane & 7));
+        const float vrB = __shfl_sync(0xffffffffu, rB, 4 * (lane & 7));
+        m = lane < 8 ? vmA : vmB;
+        l = lane < 8 ? vlA : vlB;
+        lr = lane < 8 ? vrA : vrB;
+      } else
       for (int j = 0; j < n; ++j, ++tit) {
         FA_TRACE_EV(10, j);
         if (!(ok = W.wait_warp(BAR_SF(t), tit & 1, 20))) break;
@@ -529,8 +665,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
             f2unpack(ffma2(f2pack(__uint_as_float(s[c][2 * e]), __uint_as_float(s[c][2 * e + 1])),
                            sc2, nm2),
                      x0, x1);
-            p0 = ex2(x0);
-            p1 = ex2(x1);
+            if ((FA_FWD_POLY_MASK >> (e >> 1)) & 1) {
+              exp2_fma2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
             pk[e] = pack_bf16(p0, p1);
             sum_x[e & 1] = fadd2(sum_x[e & 1], f2pack(p0, p1));
 #if FA_FWD_RSUM == 1

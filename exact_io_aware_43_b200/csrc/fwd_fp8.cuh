@@ -79,31 +79,6 @@ __device__ __forceinline__ uint64_t sdesc_swz(uint32_t saddr, uint32_t lbo, uint
 #define FA_FP8_POLY_MASK 0x24
 #endif
 
-// 2^x for two values on the FMA pipe (paired fp32 instructions), after Cody and Waite's argument
-// reduction: n = round(x) by the 1.5 * 2^23 shifter (exact for |x| < 2^22), f = x - n in
-// [-1/2, 1/2], 2^f by a cubic, and n added to the exponent field.  The cubic's coefficients are
-// our own fit (exact_io_aware_43_b200/fit_exp2.py: least largest relative error on [-1/2, 1/2],
-// 7.5e-5; the GPU self-test checks the device result against that bound).  Inputs are clamped
-// at -126 (masked scores give 2^-126, which e4m3 rounding and the fp32 row sum both absorb).
-__device__ __forceinline__ void exp2_fma2(float x0, float x1, float& p0, float& p1) {
-  const float kShift = 12582912.0f;  // 1.5 * 2^23
-  const uint64_t xc = f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t t = fadd2(xc, f2pack(kShift, kShift));
-  const uint64_t n = fadd2(t, f2pack(-kShift, -kShift));
-  const uint64_t f = ffma2(n, f2pack(-1.f, -1.f), xc);
-  uint64_t q = ffma2(f, f2pack(5.5171668530e-02f, 5.5171668530e-02f),
-                     f2pack(2.4261112511e-01f, 2.4261112511e-01f));
-  q = ffma2(q, f, f2pack(6.9326096773e-01f, 6.9326096773e-01f));
-  q = ffma2(q, f, f2pack(9.9992805719e-01f, 9.9992805719e-01f));
-  float q0, q1, t0, t1;
-  f2unpack(q, q0, q1);
-  f2unpack(t, t0, t1);
-  // the shifter leaves n in the low mantissa bits of t: shifting them up by 23 adds n to the
-  // exponent field of q
-  p0 = __uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(q0));
-  p1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(q1));
-}
-
 // Four fp32 values -> four e4m3 codes in one 32-bit word (value k in byte k), round to nearest
 // even, saturating to the finite range.
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {

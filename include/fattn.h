@@ -195,6 +195,32 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
                    int splits, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Partial results and their merge: the building blocks of ring (context-parallel) attention,
+ * where each rank holds a shard of the sequence and the key/value shards travel around the
+ * ranks.  A query shard's attention over all keys is assembled from its attention over each key
+ * shard by the associativity of the online-softmax update (robocikowo.com "Flash Attention": the
+ * rescale rule; chipfoundryservices.com glossary "Impact on Sequence Length": the method is what
+ * lets the sequence grow; the ring across GPUs is this library's extension of it).
+ *
+ * fa_fwd_partial -- attention of Nq queries against Nk keys (as for fa_fwd_splitkv: q [B, H, Nq,
+ * d] bf16, k and v [B, H_kv, Nk, d] bf16, causal aligned to the END of the keys and needing
+ * Nq <= Nk), written unrounded: o_part fp32 [B, H, Nq, d] (normalised over these keys only) and
+ * lse_part fp32 [B, H, Nq] (natural log; -inf for a row that sees none of the keys, whose o_part
+ * row is then 0).  Errors as for fa_fwd_splitkv.
+ *
+ * fa_merge_partials -- o bf16 [rows, d] and lse fp32 [rows] from n_parts partial results
+ * o_parts fp32 [n_parts, rows, d] and lse_parts fp32 [n_parts, rows] of the same query rows
+ * over disjoint key sets: lse = ln sum_s exp(lse_s), o = sum_s exp(lse_s - lse) o_s, exactly
+ * the attention over the union of the key sets.  rows is B*H*Nq of the partials.  d must be 64,
+ * 128 or 256; n_parts, rows >= 1; 16-byte aligned pointers.
+ */
+int fa_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                   int B, int H, int H_kv, int Nq, int Nk, int d, int causal, float scale,
+                   void* stream);
+int fa_merge_partials(const float* o_parts, const float* lse_parts, int n_parts, void* o,
+                      float* lse, long long rows, int d, void* stream);
+
+/*
  * fa_fwd_bwd_host -- forward and backward from HOST buffers, for callers whose tensors live in
  * host memory.  The B*H heads are independent, so they are cut into `chunks` groups of
  * consecutive heads: while group c runs fa_fwd + fa_bwd on `stream`, group c+1's inputs are

@@ -91,6 +91,22 @@ def test_fwd_fp8_rejects(kw, code):
     assert fa.fa_last_error() != ""
 
 
+def test_partial_and_merge_reject_bad_arguments():
+    P = dict(q=A, k=A, v=A, o_part=A, lse_part=A, B=1, H=2, H_kv=1, Nq=64, Nk=128, d=128,
+             causal=1, scale=0.1, stream=None)
+    assert fa.fa_fwd_partial(**{**P, "o_part": None}) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_partial(**{**P, "Nq": 200}) == fa.FA_ERR_INVALID_ARG  # causal, Nq > Nk
+    assert fa.fa_fwd_partial(**{**P, "H_kv": 3}) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_partial(**{**P, "d": 96}) == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_fwd_partial(**{**P, "lse_part": A + 4}) == fa.FA_ERR_MISALIGNED
+    M = dict(o_parts=A, lse_parts=A, n_parts=2, o=A, lse=A, rows=100, d=64, stream=None)
+    assert fa.fa_merge_partials(**{**M, "n_parts": 0}) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_merge_partials(**{**M, "rows": 0}) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_merge_partials(**{**M, "d": 32}) == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_merge_partials(**{**M, "o": None}) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_merge_partials(**{**M, "o": A + 2}) == fa.FA_ERR_MISALIGNED
+
+
 def test_selftest_exp2_rejects_bad_arguments():
     assert fa.fa_selftest_exp2_fma(None, A, 4, None) == fa.FA_ERR_INVALID_ARG
     assert fa.fa_selftest_exp2_fma(A, A, -1, None) == fa.FA_ERR_INVALID_ARG
