@@ -112,15 +112,22 @@ struct FwdCfg {
   static constexpr int TMEM_O = NQT * BN;        // O_t at TMEM_O + t*OCOLS
   static constexpr int TMEM_COLS = 512;
   static_assert(NQT * (BN + OCOLS) <= TMEM_COLS, "tensor memory budget");
+  // One query tile: tensor memory has room for a second score buffer, so consecutive key tiles
+  // alternate between S buffers (column 0 and TMEM_S1) and S(j+1) need not wait for PV(j).
+  static constexpr bool DBUF = NQT == 1;
+  static constexpr int TMEM_S1 = TMEM_O + OCOLS <= 256 ? 256 : 384;
+  static_assert(!DBUF || TMEM_S1 + BN <= TMEM_COLS, "tensor memory budget (second S buffer)");
+  static constexpr int NB = DBUF ? 2 : NQT;      // score / P / PV-done barrier slots
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQT * QTILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KVTILE_BYTES;
   static constexpr int OFF_ONES = OFF_V + STAGES * KVTILE_BYTES;  // [BN keys][64] bf16 ones
   static constexpr int OFF_BAR = OFF_ONES + (EXTRA ? BN * 128 : 0);
-  // barriers: q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT],
-  //           p_full[NQT], o_done[NQT], o_free[NQT], drain
-  static constexpr int NBAR = 2 + 4 * STAGES + 4 * NQT + 1;
+  // barriers: q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NB],
+  //           p_full[NB], o_done[NB], o_free[NQT], drain (slot = query tile, or with one query
+  //           tile the S buffer)
+  static constexpr int NBAR = 2 + 4 * STAGES + 3 * NB + NQT + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem address + abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);   // Q, K both K-major
@@ -212,10 +219,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
   auto BAR_KE = [&](int s) { return bar(2 + C::STAGES + s); };
   auto BAR_VF = [&](int s) { return bar(2 + 2 * C::STAGES + s); };
   auto BAR_VE = [&](int s) { return bar(2 + 3 * C::STAGES + s); };
-  auto BAR_SF = [&](int t) { return bar(2 + 4 * C::STAGES + t); };
-  auto BAR_PF = [&](int t) { return bar(2 + 4 * C::STAGES + NQT + t); };
-  auto BAR_OD = [&](int t) { return bar(2 + 4 * C::STAGES + 2 * NQT + t); };
-  auto BAR_OF = [&](int t) { return bar(2 + 4 * C::STAGES + 3 * NQT + t); };
+  auto BAR_SF = [&](int b) { return bar(2 + 4 * C::STAGES + b); };
+  auto BAR_PF = [&](int b) { return bar(2 + 4 * C::STAGES + C::NB + b); };
+  auto BAR_OD = [&](int b) { return bar(2 + 4 * C::STAGES + 2 * C::NB + b); };
+  auto BAR_OF = [&](int t) { return bar(2 + 4 * C::STAGES + 3 * C::NB + t); };
+  // With the double score buffer (one query tile), key tile g (counted over the CTA's whole run)
+  // uses S buffer / barrier slot g & 1, and is the (g >> 1)-th use of that slot.
+  auto sbuf_col = [&](int g) -> uint32_t { return (g & 1) ? C::TMEM_S1 : C::TMEM_S; };
   const uint32_t BAR_DRAIN = bar(C::NBAR - 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
@@ -230,12 +240,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       mbar_init(BAR_VF(s), 1);
       mbar_init(BAR_VE(s), 1);
     }
-    for (int t = 0; t < NQT; ++t) {
-      mbar_init(BAR_SF(t), 1);
-      mbar_init(BAR_PF(t), 4);
-      mbar_init(BAR_OD(t), 1);
-      mbar_init(BAR_OF(t), 4);
+    for (int b = 0; b < C::NB; ++b) {
+      mbar_init(BAR_SF(b), 1);
+      mbar_init(BAR_PF(b), 4);
+      mbar_init(BAR_OD(b), 1);
     }
+    for (int t = 0; t < NQT; ++t) mbar_init(BAR_OF(t), 4);
     mbar_init(BAR_DRAIN, 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -343,6 +353,92 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           }
         }
       }
+    } else if (warp == C::MMA_WARP && C::DBUF) {
+      // -------------------------------------------------------------- MMA issuer, one query tile
+      // Key tile g's scores go to S buffer g & 1, so S(g+1) only has to wait for PV(g-1), which
+      // read the P that buffer held.  S(g+1) is issued ahead of PV(g) whenever K(g+1) has landed
+      // (and PV(g-1) is done), so the next tile's scores are ready when the softmax warpgroup
+      // turns to them; otherwise it follows PV(g).
+      if (lane == 0) {
+        auto issue_s = [&](int g, uint32_t k_addr) {
+          const uint32_t q_addr = sbase + C::OFF_Q;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_ss(tmem + sbuf_col(g), sdesc_sw128(q_addr + koff, 16, 1024),
+                   sdesc_sw128(k_addr + koff, 16, 1024), C::IDESC_S, kk > 0);
+          }
+          tc_commit(BAR_SF(g & 1));
+        };
+        // S buffer g & 1 is free once PV(g - 2) has completed (it read the P held there)
+        auto sbuf_free = [&](int g, int site) -> bool {
+          return g < 2 || W.wait(BAR_OD(g & 1), ((g - 2) >> 1) & 1, site);
+        };
+        int g = 0, kv_it = 0, kq = 0, nun = 0;
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+          const int u = fwd_unit_of(k, cta, G, p.units);
+          if (u < 0) break;
+          const Unit un(u, p);
+          const int J = un.J;
+          if (J == 0) continue;
+          const int s0 = kv_it % C::STAGES;
+          if (!(ok = W.wait(BAR_Q, kq & 1, 10))) break;
+          if (!(ok = W.wait(BAR_KF(s0), (kv_it / C::STAGES) & 1, 11))) break;
+          if (!(ok = sbuf_free(g, 12))) break;
+          tc_fence_after();
+          issue_s(g, sbase + C::OFF_K + s0 * C::KVTILE_BYTES);
+          tc_commit(BAR_KE(s0));
+          if (J == 1) tc_commit(BAR_QE);
+          for (int j = 0; ok && j < J; ++j) {
+            const int gg = g + j;
+            const int s = (kv_it + j) % C::STAGES;
+            const int s1 = (kv_it + j + 1) % C::STAGES;
+            const uint32_t kph1 = ((kv_it + j + 1) / C::STAGES) & 1;
+            bool s_next = j + 1 < J;
+            if (s_next && mbar_test_wait(BAR_KF(s1), kph1) &&
+                (gg + 1 < 2 || mbar_test_wait(BAR_OD((gg + 1) & 1), ((gg - 1) >> 1) & 1))) {
+              tc_fence_after();
+              issue_s(gg + 1, sbase + C::OFF_K + s1 * C::KVTILE_BYTES);
+              tc_commit(BAR_KE(s1));
+              if (j + 2 == J) tc_commit(BAR_QE);  // every S of this unit is issued
+              s_next = false;
+            }
+            if (!(ok = W.wait(BAR_VF(s), ((kv_it + j) / C::STAGES) & 1, 13))) break;
+            if (!(ok = W.wait(BAR_PF(gg & 1), (gg >> 1) & 1, 14))) break;
+            // the first PV of a unit overwrites O: the previous epilogue must have read it
+            if (j == 0 && nun > 0 && !(ok = W.wait(BAR_OF(0), (nun - 1) & 1, 15))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C::BN / 16; ++kk) {
+              mma_ts(tmem + C::TMEM_O, tmem + sbuf_col(gg) + kk * 8,
+                     sdesc_sw128(sbase + C::OFF_V + s * C::KVTILE_BYTES + kk * 2048,
+                                 C::EXTRA ? uint32_t(C::OFF_ONES - C::OFF_V - s * C::KVTILE_BYTES)
+                                          : uint32_t(C::BN * 128),
+                                 1024),
+                     C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(BAR_OD(gg & 1));
+            tc_commit(BAR_VE(s));
+            if (s_next) {
+              if (!(ok = W.wait(BAR_KF(s1), kph1, 16))) break;
+              if (!(ok = sbuf_free(gg + 1, 17))) break;
+              tc_fence_after();
+              issue_s(gg + 1, sbase + C::OFF_K + s1 * C::KVTILE_BYTES);
+              tc_commit(BAR_KE(s1));
+              if (j + 2 == J) tc_commit(BAR_QE);
+            }
+          }
+          if (!ok) break;
+          g += J;
+          kv_it += J;
+          ++kq;
+          ++nun;
+        }
+        // every MMA issued above has completed before the tensor memory is released
+        tc_commit(BAR_DRAIN);
+        W.drain(BAR_DRAIN, 0);
+      }
     } else if (warp == C::MMA_WARP) {
       // -------------------------------------------------------------- MMA issuer
       // Order per KV tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  S_t(j+1) overwrites the
@@ -449,7 +545,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     const int t = warp >> 2;                  // query tile of this warpgroup
     const int r = threadIdx.x & 127;          // row within the tile == TMEM lane
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + C::TMEM_S + t * C::BN;
+    // key tile gi's score buffer and barrier slot / phase (see sbuf_col)
+    auto tS_of = [&](int gi) -> uint32_t {
+      return tmem + lane_base + (C::DBUF ? sbuf_col(gi) : uint32_t(C::TMEM_S + t * C::BN));
+    };
+    auto slot = [&](int gi) { return C::DBUF ? (gi & 1) : t; };
+    auto sph = [&](int gi) -> uint32_t { return C::DBUF ? uint32_t((gi >> 1) & 1) : uint32_t(gi & 1); };
     const uint32_t tO = tmem + lane_base + C::TMEM_O + t * C::OCOLS;
     // m: reference max (log2 units of the scaled scores) that the exponentials and l are taken
     // against.  It only moves when a row's max grows by more than kRescale (2^8 in value): the
@@ -487,12 +588,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         const int g4 = lane >> 2, c2 = 2 * (lane & 3);
         float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f, rA = 0.f, rB = 0.f;
         for (int j = 0; j < n; ++j, ++tit) {
-          if (!(ok = W.wait_warp(BAR_SF(t), tit & 1, 20))) break;
+          if (!(ok = W.wait_warp(BAR_SF(slot(tit)), sph(tit), 20))) break;
           tc_fence_after();
           float alphaA = 1.f, alphaB = 1.f;
           if (worker) {
             uint32_t sv[64];
-            tmem_ld16x256b_x16(tS, sv);
+            tmem_ld16x256b_x16(tS_of(tit), sv);
             tmem_wait_ld64(sv);
             const int key0 = (un.kt0 + j) * C::BN;
             uint32_t wd[32];
@@ -557,13 +658,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
               mr = m_use;
             }
             // P~ (bf16 pairs) over the first 64 columns of S_t, rows 0-15
-            tmem_st16x128b_x16(tS, wd);
+            tmem_st16x128b_x16(tS_of(tit), wd);
             // the row factors to thread = row for the 32x32b rescale of O
             const float aA = __shfl_sync(0xffffffffu, alphaA, 4 * (lane & 7));
             const float aB = __shfl_sync(0xffffffffu, alphaB, 4 * (lane & 7));
             const float alpha = lane < 8 ? aA : (lane < 16 ? aB : 1.f);
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-              if (!(ok = W.wait_warp(BAR_OD(t), (tit - 1) & 1, 21))) {
+              if (!(ok = W.wait_warp(BAR_OD(slot(tit - 1)), sph(tit - 1), 21))) {
                 tmem_wait_st();
                 break;
               }
@@ -590,7 +691,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(BAR_PF(t));
+          if (lane == 0) mbar_arrive(BAR_PF(slot(tit)));
         }
         if (!ok) break;
         // row statistics to thread = row (lanes 0-15 of the first warp) for the epilogue
@@ -606,12 +707,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       } else
       for (int j = 0; j < n; ++j, ++tit) {
         FA_TRACE_EV(10, j);
-        if (!(ok = W.wait_warp(BAR_SF(t), tit & 1, 20))) break;
+        if (!(ok = W.wait_warp(BAR_SF(slot(tit)), sph(tit), 20))) break;
         FA_TRACE_EV(11, j);
         tc_fence_after();
         uint32_t s[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS_of(tit) + 32 * c, s[c]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_wait_ld(s[c]);
         FA_TRACE_EV(15, j);
@@ -697,8 +798,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         }
         FA_TRACE_EV(12, j);
         // P~ (bf16) over the first 64 columns of S_t
-        tmem_st32(tS + 0, s[0]);
-        tmem_st32(tS + 32, s[2]);
+        tmem_st32(tS_of(tit) + 0, s[0]);
+        tmem_st32(tS_of(tit) + 32, s[2]);
         {
           float a0, a1, b0, b1;
           f2unpack(fadd2(sum_x[0], sum_x[1]), a0, a1);
@@ -710,7 +811,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
           FA_TRACE_EV(14, j);
           // O_t holds PV_t(j-1) (S_t(j) was issued only after it completed); rescale it
-          if (!(ok = W.wait_warp(BAR_OD(t), (tit - 1) & 1, 21))) break;
+          if (!(ok = W.wait_warp(BAR_OD(slot(tit - 1)), sph(tit - 1), 21))) break;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -733,13 +834,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(BAR_PF(t));
+        if (lane == 0) mbar_arrive(BAR_PF(slot(tit)));
         FA_TRACE_EV(13, j);
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 -> global; L = (m + log2 l) * ln 2.  O_t is released to the
       // next unit's first PV once its last chunk has been read.
-      if (!(ok = W.wait_warp(BAR_OD(t), (tit - 1) & 1, 22))) break;
+      if (!(ok = W.wait_warp(BAR_OD(slot(tit - 1)), sph(tit - 1), 22))) break;
       tc_fence_after();
       // a row with no visible key in this split (split mode only) gets O = 0 and L = -inf
       if constexpr (C::EXTRA > 0) {  // the MMA's row sum of the rounded weights

@@ -80,9 +80,11 @@ def cuda_partial(q, k, v, causal: bool, scale: float | None = None):
     """(O_part fp32 [B, H, n, d], L_part fp32 [B, H, n]) through fa_fwd_partial."""
     import torch
 
-    from . import _check, _default_scale, _kv_heads, _shape, _stream_handle, fa_fwd_partial
+    from . import _check, _default_scale, _shape, _stream_handle, fa_fwd_partial
     B, H, n, d = _shape(q)
-    Hkv = _kv_heads(q, k)
+    if k.dim() != 4 or k.shape[0] != B or k.shape[3] != d or k.shape[1] < 1 or H % k.shape[1]:
+        raise ValueError("k, v must be [B, H_kv, Nk, d] with H_kv dividing q's H")
+    Hkv = int(k.shape[1])
     scale = _default_scale(d) if scale is None else float(scale)
     o = torch.empty((B, H, n, d), dtype=torch.float32, device=q.device)
     lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)

@@ -41,9 +41,9 @@ def test_ring_ranks_on_one_gpu(W, n, d, Hkv, causal):
         assert_fwd(to_np(o), O[:, :, sl], to_np(lse), L[:, :, sl], f"ring rank {r} of {W}")
 
 
-def test_partial_of_a_hidden_shard_has_no_weight():
-    """A query shard that sees none of a key shard (causal, end-aligned with Nq > visible) gets
-    lse = -inf there; merged with a real partial it changes nothing."""
+def test_partial_with_no_weight_changes_nothing():
+    """A partial whose logsumexp is -inf (a key shard the rows cannot see) has weight 0 in the
+    merge: merging it beside a real partial of 128 queries over 256 keys changes no bit."""
     import torch
     from exact_io_aware_43_b200.ring import cuda_merge, cuda_partial
     dev, _ = cuda_inputs(1, 2, 256, 128, seed=9, with_do=False)
