@@ -46,6 +46,12 @@
 #define FA_BWDQ_DK_SS 1
 #endif
 
+// FA_BWDQ_PIPE_LD: 1 loads the second 32 columns of S^T / dP^T while the first 32 are worked on
+// (one tcgen05.wait::ld covers all of a thread's loads, so the second load is issued after the
+// first wait); 0 loads both, then waits.
+#ifndef FA_BWDQ_PIPE_LD
+#define FA_BWDQ_PIPE_LD 0
+#endif
 // FA_BWDQ_POLY_MASK: bit g set computes the exponentials of query columns [8g, 8g+8) of every 64
 // on the FMA pipe (exp2_fma2) instead of the MUFU unit.
 #ifndef FA_BWDQ_POLY_MASK
@@ -407,9 +413,10 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
       tc_fence_after();
       uint32_t sv[2][32];
       tmem_ld32(tmem + lane_base + C::T_S + c0, sv[0]);
-      tmem_ld32(tmem + lane_base + C::T_S + c0 + 32, sv[1]);
+      if (!FA_BWDQ_PIPE_LD) tmem_ld32(tmem + lane_base + C::T_S + c0 + 32, sv[1]);
       tmem_wait_ld(sv[0]);
-      tmem_wait_ld(sv[1]);
+      if (FA_BWDQ_PIPE_LD) tmem_ld32(tmem + lane_base + C::T_S + c0 + 32, sv[1]);
+      else tmem_wait_ld(sv[1]);
       FA_TRACE_EV(15, t);
       // P^T = exp2((S^T - L/s) s log2e) (the MMA has subtracted L/s); zero for masked (causal
       // key > query) and padded keys.  Only the diagonal block (i == j) and a ragged last key
@@ -420,6 +427,8 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
 #pragma unroll
       for (int c2 = 0; c2 < 32; ++c2) {
         const int c = 2 * c2;
+        // with FA_BWDQ_PIPE_LD the second 32 columns arrive while the first are worked on
+        if (FA_BWDQ_PIPE_LD && c2 == 16) tmem_wait_ld(sv[1]);
         float x0, x1;
         f2unpack(fmul2(f2pack(__uint_as_float(sv[c >> 5][c & 31]),
                               __uint_as_float(sv[c >> 5][(c & 31) + 1])),
@@ -452,15 +461,17 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
       FA_TRACE_EV(13, t);
       tc_fence_after();
       tmem_ld32(tmem + lane_base + C::T_DP + c0, sv[0]);
-      tmem_ld32(tmem + lane_base + C::T_DP + c0 + 32, sv[1]);
+      if (!FA_BWDQ_PIPE_LD) tmem_ld32(tmem + lane_base + C::T_DP + c0 + 32, sv[1]);
       tmem_wait_ld(sv[0]);
-      tmem_wait_ld(sv[1]);
+      if (FA_BWDQ_PIPE_LD) tmem_ld32(tmem + lane_base + C::T_DP + c0 + 32, sv[1]);
+      else tmem_wait_ld(sv[1]);
       FA_TRACE_EV(18, t);
       // the MMA has subtracted D: dS^T = P^T dP'^T, one paired multiply per two queries
       uint32_t dsk[32];
 #pragma unroll
       for (int c2 = 0; c2 < 32; ++c2) {
         const int c = 2 * c2;
+        if (FA_BWDQ_PIPE_LD && c2 == 16) tmem_wait_ld(sv[1]);
         const uint32_t pp = pk[c2];
         float d0, d1;
         f2unpack(fmul2(f2pack(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u)),
