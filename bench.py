@@ -39,6 +39,34 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 
 
+class L2Flush:
+    """Empties the 126 MB L2 between timed steps, outside the timed events: a 256 MiB buffer is
+    written (nothing the next step reads stays cached), then a second 256 MiB buffer is read, so
+    that the dirty lines of the write are written back here and not during the next timed
+    kernel (which would otherwise pay up to 126 MB of write-back traffic)."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.max()
+
+
+def pass_bytes(B, H, Hkv, N, d, forward: bool) -> int:
+    """Compulsory HBM bytes of one pass: each input read once and each output written once.
+    Forward: Q, K, V in, O (bf16) and L (fp32) out.  Backward main kernel: Q, dO, K, V, L, D in,
+    dQ, dK, dV out (the fp32 dQ accumulator's traffic is not counted: it is the kernel's own)."""
+    q = B * H * N * d * 2
+    kv = B * Hkv * N * d * 2
+    rows = B * H * N * 4
+    if forward:
+        return q + 2 * kv + q + rows
+    return 2 * q + 2 * kv + 2 * rows + q + 2 * kv
+
+
 def flops(B, H, N, d, causal):
     fwd = 4.0 * B * H * N * N * d * (0.5 if causal else 1.0)
     return fwd, 2.5 * fwd
@@ -135,27 +163,56 @@ def barrier(device=None):
 
 # ---------------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks and throttle reasons, sampled every 20 ms while running.
+
+    start() returns once the first sample has been written, so that sampling is live before the
+    timed region begins; begin() / end() mark the timed region on the host clock (call them right
+    after the synchronize on each side), and stop() keeps the samples whose timestamps fall inside
+    it.  A region shorter than the sampling interval may hold none: then the samples nearest to
+    it on either side are kept and the result says so ("window": "nearest")."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 20
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
-    def start(self):
+    def start(self, wait_s: float = 5.0):
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
                 stdout=self.out, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        t_end = time.time() + wait_s
+        while time.time() < t_end and self.proc.poll() is None:
+            self.out.flush()
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.01)
+
+    def begin(self):
+        self.t0 = time.time()
+
+    def end(self):
+        self.t1 = time.time()
+
+    @staticmethod
+    def _stamp(s: str):
+        import datetime
+        try:
+            return datetime.datetime.strptime(s, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
 
     def stop(self):
         if self.proc is None:
@@ -170,9 +227,21 @@ class ClockSampler:
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
+                if len(parts) >= 10:
+                    rows.append((self._stamp(parts[0]), parts[1:]))
         os.unlink(self.path)
+        window = "timed region"
+        if self.t0 is not None and self.t1 is not None and all(t is not None for t, _ in rows):
+            inside = [r for t, r in rows if self.t0 <= t <= self.t1]
+            if not inside:
+                before = [r for t, r in rows if t < self.t0][-1:]
+                after = [r for t, r in rows if t > self.t1][:1]
+                inside = before + after
+                window = "nearest"
+            rows = inside
+        else:
+            rows = [r for _, r in rows]
+            window = "whole run"
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
@@ -183,7 +252,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(pw) if pw else None}
+                "power_w_max": max(pw) if pw else None, "window": window}
 
 
 # ---------------------------------------------------------------------------------- oracle leg
@@ -260,19 +329,22 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------------- GPU arm
-def kernel_traffic(kernel_name: str):
-    """DRAM bytes per launch from a committed ncu capture, if it was taken on the current source."""
+def kernel_traffic(kernel_name: str, workload: dict):
+    """DRAM bytes per launch of `kernel_name` on `workload` from a committed ncu capture, if one
+    was taken for that kernel and workload on the current source (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f).get(kernel_name)
-    except (OSError, ValueError):
+            recs = json.load(f).get("records", [])
+    except (OSError, ValueError, AttributeError):
         return None
-    if not rec:
-        return None
-    if rec.get("csrc_sha256") != csrc_code_hash():
-        return None
-    return rec.get("bytes_per_launch")
+    for rec in recs:
+        if rec.get("kernel") != kernel_name or rec.get("workload") != workload:
+            continue
+        if rec.get("csrc_sha256") != csrc_code_hash():
+            return None
+        return rec.get("bytes_per_launch")
+    return None
 
 
 def csrc_code_hash() -> str:
@@ -310,14 +382,14 @@ def run_gpu(args):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(fa.fa_bwd_gqa_workspace_size(B, H, W.get("H_kv", H), N, d), dtype=torch.uint8,
                      device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def step():
         fa.forward(q, k, v, causal, s, out=o, lse=lse)
         fa.backward(q, k, v, o, lse, do, causal, s, workspace=ws, grads=(dq, dk, dv))
 
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     assert fa.fa_device_status() == 0, "a kernel reported a timeout during warm-up"
@@ -330,13 +402,15 @@ def run_gpu(args):
           for _ in range(args.steps)]
     barrier(dev)
     torch.cuda.synchronize()
+    sampler.begin()
     fa.fa_timer_enable(True)
     for i in range(args.steps):
-        flush.zero_()  # L2 flushed before every step, outside the timed events
+        flush()  # L2 flushed before every step, outside the timed events
         ev[i][0].record()
         step()
         ev[i][1].record()
     torch.cuda.synchronize()
+    sampler.end()
     fa.fa_timer_enable(False)
     barrier(dev)
     clocks = sampler.stop()
@@ -356,12 +430,25 @@ def run_gpu(args):
     n_l, tot = ktimes[dom]
     avg_ms = tot / max(1, n_l)
     if dom in (fa.FA_KERNEL_FWD, fa.FA_KERNEL_BWD_MAIN):
+        # the binding roof is the one with the longer ideal time: FLOPs at the tensor peak, or
+        # the pass's compulsory HBM bytes (every input read once, every output written once) at
+        # the copy bandwidth; short sequences are HBM bound, long ones tensor bound
         work = ff if dom == fa.FA_KERNEL_FWD else fb
-        achieved = work / (avg_ms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
-                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak)}
+        nbytes = pass_bytes(B, H, W.get("H_kv", H), N, d, dom == fa.FA_KERNEL_FWD)
+        t_tensor = work / (peaks["bf16_tflops"] * 1e12)
+        t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+        tensor = {"bound": "tensor", "achieved": work / (avg_ms * 1e-3) / 1e12,
+                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                  "peak_source": f"{peak_src} bf16_tflops (burst)"}
+        tensor["frac"] = tensor["achieved"] / tensor["peak"]
+        tensor["frac_of_sustained"] = tensor["achieved"] / peaks.get("bf16_tflops_sustained",
+                                                                     tensor["peak"])
+        hbm = {"bound": "hbm", "achieved": nbytes / (avg_ms * 1e-3) / 1e9,
+               "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs",
+               "algorithmic_bytes": nbytes}
+        hbm["frac"] = hbm["achieved"] / hbm["peak"]
+        roof, other = (hbm, tensor) if t_hbm > t_tensor else (tensor, hbm)
+        roof["other_roof"] = {k: other[k] for k in ("bound", "achieved", "unit", "frac")}
     else:
         nbytes = (B * H * N * d * 2 * 2 + B * H * N * 4 + B * H * N * d * 4 + 2 * B * H * N * 4
                   if dom == fa.FA_KERNEL_BWD_PRE else B * H * N * d * (4 + 2))
@@ -372,7 +459,10 @@ def run_gpu(args):
     roof["kernel"] = fa.KERNEL_NAMES[dom]
     roof["launches"] = n_l
     roof["avg_ms"] = avg_ms
-    roof["traffic"] = kernel_traffic(fa.KERNEL_NAMES[dom])
+    roof["traffic"] = kernel_traffic(fa.KERNEL_NAMES[dom],
+                                     {"pass": "bf16 fwd+bwd", "B": B, "H": H,
+                                      "H_kv": W.get("H_kv", H), "N": N, "d": d,
+                                      "causal": bool(causal)})
     shares = {fa.KERNEL_NAMES[kk]: ktimes[kk][1] / max(1e-9, sum(t for _, t in ktimes.values()))
               for kk in range(4)}
 
@@ -432,7 +522,7 @@ def run_gpu(args):
             "data": "synthetic",
             "config": {"workload": WORKLOAD_NAME, **WORKLOAD, "scale": s,
                        "flops_per_step_per_gpu": ff + fb,
-                       "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                       "l2": "flushed before every timed step (256 MiB write, then 256 MiB read so no dirty line is left; outside the events)",
                        "parallelism": f"heads: {world} independent replicas, no collective"},
             "pct_of_peak": value / world / peaks["bf16_tflops"] * 100.0,
             "fwd_tflops": ff / (fwd_ms * 1e-3) / 1e12, "bwd_tflops": fb / (bwd_ms * 1e-3) / 1e12,
@@ -474,13 +564,13 @@ def run_decode(args):
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
     ws = torch.empty(max(16, fa.fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, splits)),
                      dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def step():
         fa.forward_splitkv(q, k, v, True, s, splits=splits, out=o, lse=lse, workspace=ws)
 
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     assert fa.fa_device_status() == 0, "a kernel reported a timeout during warm-up"
@@ -492,13 +582,15 @@ def run_decode(args):
           for _ in range(args.steps)]
     barrier(dev)
     torch.cuda.synchronize()
+    sampler.begin()
     fa.fa_timer_enable(True)
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         ev[i][0].record()
         step()
         ev[i][1].record()
     torch.cuda.synchronize()
+    sampler.end()
     fa.fa_timer_enable(False)
     barrier(dev)
     clocks = sampler.stop()
@@ -514,7 +606,10 @@ def run_decode(args):
             "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": algo_bytes / (fwd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
             "peak_source": f"{peak_src} hbm_gbs", "kernel": "fa_fwd_kernel", "launches": n_f,
-            "avg_ms": fwd_ms, "traffic": None,
+            "avg_ms": fwd_ms,
+            "traffic": kernel_traffic("fa_fwd_kernel", {"pass": "decode", "B": B, "H": H,
+                                                        "H_kv": Hkv, "Nq": Nq, "Nk": Nk, "d": d,
+                                                        "splits": splits}),
             "algorithmic_bytes": algo_bytes}
     if rank == 0:
         line = {
@@ -525,7 +620,7 @@ def run_decode(args):
             "config": {"workload": f"decode: B={B} H={H} H_kv={Hkv} Nq={Nq} Nk={Nk} d={d} causal, "
                                    f"{splits} key ranges", "B": B, "H": H, "H_kv": Hkv,
                        "Nq": Nq, "Nk": Nk, "d": d, "splits": splits,
-                       "l2": "flushed before every timed step (256 MiB write, outside the events)"},
+                       "l2": "flushed before every timed step (256 MiB write, then 256 MiB read so no dirty line is left; outside the events)"},
             "kernel_ms": {"fa_fwd_kernel": fwd_ms,
                           "fa_fwd_merge_kernel": kt[fa.FA_KERNEL_FWD_MERGE][1] /
                           max(1, kt[fa.FA_KERNEL_FWD_MERGE][0])},
@@ -559,13 +654,13 @@ def run_fp8(args):
     q, k, v = (host[t].to(dev) for t in ("q", "k", "v"))
     o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def step():
         fa.forward_fp8(q, k, v, sc["q"], sc["k"], sc["v"], causal, s, out=o, lse=lse)
 
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     assert fa.fa_device_status() == 0, "a kernel reported a timeout during warm-up"
@@ -576,13 +671,15 @@ def run_fp8(args):
           for _ in range(args.steps)]
     barrier(dev)
     torch.cuda.synchronize()
+    sampler.begin()
     fa.fa_timer_enable(True)
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         ev[i][0].record()
         step()
         ev[i][1].record()
     torch.cuda.synchronize()
+    sampler.end()
     fa.fa_timer_enable(False)
     barrier(dev)
     clocks = sampler.stop()
@@ -598,7 +695,10 @@ def run_fp8(args):
             "frac": achieved / peak,
             "peak_source": f"{peak_src} bf16_tflops (burst) x 2, the nominal fp8/bf16 ratio",
             "frac_of_bf16_peak": achieved / peaks["bf16_tflops"], "kernel": "fa_fwd_fp8_kernel",
-            "launches": n_f, "avg_ms": kern_ms, "traffic": None}
+            "launches": n_f, "avg_ms": kern_ms,
+            "traffic": kernel_traffic("fa_fwd_fp8_kernel", {"pass": "fp8 fwd", "B": B, "H": H,
+                                                            "N": N, "d": d,
+                                                            "causal": bool(causal)})}
     # end to end through the public API: e4m3 codes from pinned host memory, O and L back
     e2e = None
     if args.e2e_steps > 0:
@@ -634,7 +734,7 @@ def run_fp8(args):
             "data": "synthetic",
             "config": {"workload": f"FP8 forward, B={B} H={H} N={N} d={d} causal={causal}",
                        **WORKLOAD, "scale": s, "flops_per_step_per_gpu": ff,
-                       "l2": "flushed before every timed step (256 MiB write, outside the events)"},
+                       "l2": "flushed before every timed step (256 MiB write, then 256 MiB read so no dirty line is left; outside the events)"},
             "roofline": roof, "e2e": e2e, "clocks": clocks, "gpu_launches": n_f,
             "device_status": status,
         }
