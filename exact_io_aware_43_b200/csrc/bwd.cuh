@@ -1,8 +1,10 @@
 // bwd.cuh -- attention backward for sm_100a, by recomputation (robocikowo.com "Flash Attention":
 // the backward recomputes the attention matrix from the saved O and L instead of storing it).
 //
-// Three kernels on the caller's stream (the main kernel for d = 128 is fa_bwd_kernel_q128, in
-// bwd_q128.cuh, with 128-query steps; this file's fa_bwd_kernel serves d = 64 and d = 256):
+// Three kernels on the caller's stream.  The main kernel is fa_bwd_kernel_q128 (bwd_q128.cuh,
+// 128-query steps) for d = 64 and 128, and fa_bwd_kernel_pair (bwd_pair.cuh, CTA pairs) for
+// d = 256; this file's fa_bwd_kernel is the alternative the build selects with FA_BWD_Q128=0 or
+// FA_BWD_PAIR=0:
 //   fa_bwd_pre_kernel   D_i = sum_c dO_ic O_ic, L2_i = L_i log2(e) (padded rows: +inf, 0),
 //                       and zeroes the fp32 dQ accumulator (and the dK, dV accumulators when
 //                       a group's query heads are split over CTAs).                  (HBM bound)

@@ -19,6 +19,7 @@
 #include "../../include/fattn.h"
 #include "bwd.cuh"
 #include "bwd_q128.cuh"
+#include "bwd_pair.cuh"
 #include "merge.cuh"
 #include "fwd.cuh"
 #include "fwd_fp8.cuh"
@@ -299,6 +300,11 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 #ifndef FA_BWD_Q128
 #define FA_BWD_Q128 1
 #endif
+// d = 256 backward: CTA pairs exchanging P and dS through distributed shared memory
+// (fa_bwd_kernel_pair); 0 selects the kernel whose two CTAs per key block each recompute S^T, dP^T.
+#ifndef FA_BWD_PAIR
+#define FA_BWD_PAIR 1
+#endif
 
 template <int D, bool CAUSAL>
 int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, cudaStream_t st) {
@@ -346,6 +352,33 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
       TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
       kq<<<grid, CQ::THREADS, CQ::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, p);
     }
+  } else if (D == 256 && FA_BWD_PAIR) {
+    using CP = fattn::BwdPairCfg;
+    auto kp = fattn::fa_bwd_kernel_pair<CAUSAL>;
+    if ((rc = set_smem(kp, CP::SMEM_BYTES))) return rc;
+    if ((rc = make_map(&mq, q, p.BH, p.N, D, CP::BR))) return rc;
+    if ((rc = make_map(&mdo, p.dO, p.BH, p.N, D, CP::BR))) return rc;
+    if ((rc = make_map(&mk, k, p.BHkv, p.N, D, CP::BC))) return rc;
+    if ((rc = make_map(&mv, v, p.BHkv, p.N, D, CP::BC))) return rc;
+    if ((rc = make_map_f32(&mdq, p.dq_acc, p.BH, p.N, D, 32, 32))) return rc;  // per drain warp
+    // one cluster of two CTAs per (key block, key/value head [, share of the group's heads])
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2u * unsigned(p.BHkv) * unsigned(p.nkb) * unsigned(p.gsplit));
+    cfg.blockDim = dim3(CP::THREADS);
+    cfg.dynamicSmemBytes = CP::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    {
+      TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
+      e = cudaLaunchKernelEx(&cfg, kp, mq, mk, mv, mdo, mdq, p);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "fa_bwd (pair) launch");
   } else {
     auto kern = fattn::fa_bwd_kernel<D, CAUSAL>;
     if ((rc = set_smem(kern, C::SMEM_BYTES))) return rc;

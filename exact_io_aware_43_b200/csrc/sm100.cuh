@@ -19,24 +19,26 @@ namespace fattn {
 __device__ int g_status[2];
 
 // ------------------------------------------------------------------------------------------
-// Optional pipeline trace (compiled in only with -DFA_TRACE): lane 0 of each warp of one chosen
-// CTA appends (SM clock, warp, event, iteration) records; fa_trace_read copies them out.
+// Optional pipeline trace (compiled in only with -DFA_TRACE): lane 0 of each of the first 16
+// warps of two chosen CTAs (FA_TRACE_CTA and its neighbour, the pair of a two-CTA cluster)
+// appends (SM clock, CTA, warp, event, iteration) records; fa_trace_read copies them out.
 // ------------------------------------------------------------------------------------------
 #ifdef FA_TRACE
 #ifndef FA_TRACE_CTA
 #define FA_TRACE_CTA 300
 #endif
-constexpr unsigned kTraceWarps = 16, kTracePerWarp = 4096, kTraceMax = kTraceWarps * kTracePerWarp;
+constexpr unsigned kTraceWarps = 32, kTracePerWarp = 4096, kTraceMax = kTraceWarps * kTracePerWarp;
 __device__ unsigned long long g_trace[2 * kTraceMax];
 __device__ unsigned int g_trace_n;
 // per-warp slots, plain stores (no atomics): the record costs a few issue cycles only
 #define FA_TRACE_EV(code, it)                                                                  \
   do {                                                                                         \
-    if (blockIdx.x == FA_TRACE_CTA && (threadIdx.x & 31) == 0 && (threadIdx.x >> 5) < 16 &&    \
-        fa_trace_k < ::fattn::kTracePerWarp) {                                                 \
-      const unsigned k_ = (threadIdx.x >> 5) * ::fattn::kTracePerWarp + fa_trace_k++;          \
+    if ((blockIdx.x | 1u) == (FA_TRACE_CTA | 1u) && (threadIdx.x & 31) == 0 &&                 \
+        (threadIdx.x >> 5) < 16 && fa_trace_k < ::fattn::kTracePerWarp) {                      \
+      const unsigned w_ = (blockIdx.x & 1u) * 16 + (threadIdx.x >> 5);                         \
+      const unsigned k_ = w_ * ::fattn::kTracePerWarp + fa_trace_k++;                          \
       ::fattn::g_trace[2 * k_] = clock64();                                                    \
-      ::fattn::g_trace[2 * k_ + 1] = ((unsigned long long)(threadIdx.x >> 5) << 40) |          \
+      ::fattn::g_trace[2 * k_ + 1] = ((unsigned long long)w_ << 40) |                          \
                                      ((unsigned long long)(code) << 32) | (unsigned)(it);      \
     }                                                                                          \
   } while (0)
