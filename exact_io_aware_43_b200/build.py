@@ -18,11 +18,13 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB_DIR = os.path.join(HERE, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libfattn.so")
-# Test-only variant: the forward's producer leaves one K/V tile unissued (FA_TEST_STARVE) and the
-# waits are bounded at 1 ms, so a test can watch a bounded wait run out and the kernel report
-# FA_ERR_TIMEOUT without any fault or hang.  The product path never loads it.
+# Test-only variant: the forward's producer leaves one K/V tile unissued, and the d = 256
+# backward's one dO tile (FA_TEST_STARVE); the waits are bounded at 1 ms and the pair kernel's
+# teardown hand-back wait at 20 ms, so a test can watch a bounded wait run out and the kernel
+# report FA_ERR_TIMEOUT without any fault or hang.  The product path never loads it.
 STARVE_PATH = os.path.join(LIB_DIR, "libfattn_starve.so")
-STARVE_DEFINES = ["-DFA_TEST_STARVE", "-DFA_DEFAULT_WAIT_LIMIT_NS=1000000ull"]
+STARVE_DEFINES = ["-DFA_TEST_STARVE", "-DFA_DEFAULT_WAIT_LIMIT_NS=1000000ull",
+                  "-DFA_PAIR_HANDBACK_LIMIT_NS=20000000ull"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 NVCC_FLAGS = [

@@ -122,6 +122,10 @@ __device__ __forceinline__ void cluster_barrier() {
                ::: "memory");
 }
 
+#ifndef FA_PAIR_HANDBACK_LIMIT_NS
+#define FA_PAIR_HANDBACK_LIMIT_NS 4000000000ull
+#endif
+
 // Bounded waits for a CTA of a pair: like Waiter, with cluster-scope acquire, and giving up
 // also raises the peer's abort flag.
 struct PairWaiter {
@@ -157,12 +161,14 @@ struct PairWaiter {
     }
     return true;
   }
-  // Teardown wait on a barrier the peer arrives on (cluster-scope acquire), ignoring the abort
-  // flag, bounded by the drain limit.
+  // Teardown wait for the peer's hand-back of a tile this warp sent (cluster-scope acquire),
+  // ignoring the abort flag.  After an abort the hand-back may never come; the bound only has to
+  // exceed the landing time of the asynchronous stores (microseconds).
+  static constexpr uint64_t kHandBackLimitNs = FA_PAIR_HANDBACK_LIMIT_NS;
   __device__ __forceinline__ void drain_warp(uint32_t bar, uint32_t parity) const {
     const uint64_t t0 = global_ns();
     while (!mbar_try_wait_cluster(bar, parity)) {
-      if (global_ns() - t0 > Waiter::kDrainLimitNs) break;
+      if (global_ns() - t0 > kHandBackLimitNs) break;
     }
     __syncwarp();
   }
@@ -302,11 +308,21 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
         tma_load_3d(sbase + C::OFF_A + kb * C::KV_BLK, tmA, bar(C::B_KV), kb * 64, k0, kvh);
       const float* rows_src = role == 0 ? p.L2 : p.Drow;
       int it = 0;
+      bool starved = false;
       BwdCursor cur(grp);
       for (; it < nit; ++it) {
         const int i = cur.i, head = cur.head;
         cur.next();
         const int s = it % NS;
+#ifdef FA_TEST_STARVE
+        // Test build only (libfattn_starve.so): CTA 1 of the first cluster never issues its second
+        // dO_i tile, so the bounded waits for it run out on both CTAs of the pair, which must
+        // report FA_ERR_TIMEOUT and tear down cleanly.  The loads issued so far are drained below.
+        if (blockIdx.x == 1 && it == 1) {
+          starved = true;
+          break;
+        }
+#endif
         if (!W.wait(bar(C::B_LE + s), ((it / NS) & 1) ^ 1, 70)) break;
         FA_TRACE_EV(30, it);
         mbar_arrive_expect_tx(bar(C::B_LF + s), C::STAGE + C::BR * 4);
@@ -317,7 +333,7 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
                   rows_src + size_t(head) * p.Npad + size_t(i) * C::BR, C::BR * 4,
                   bar(C::B_LF + s));
       }
-      if (W.aborted()) {
+      if (W.aborted() || starved) {
         W.drain(bar(C::B_KV), 0);
         for (int jj = max(0, it - NS); jj < it; ++jj)
           W.drain(bar(C::B_LF + jj % NS), (jj / NS) & 1);

@@ -1,7 +1,8 @@
 """Failure detection on the GPU without a fault: a bounded wait that runs out.
 
 ``libfattn_starve.so`` is the library built with one change (FA_TEST_STARVE) and a 1 ms wait
-bound: in the forward, CTA 0's producer warp never issues the second K/V tile of its first unit.
+bound: in the forward, CTA 0's producer warp never issues the second K/V tile of its first unit;
+in the d = 256 backward (CTA pairs), CTA 1 of the first cluster never issues its second dO tile.
 Nothing is left in flight -- the copies it did issue are drained before the CTA exits -- so the
 MMA warp's bounded wait for that tile simply runs out.  The kernel must then record
 FA_ERR_TIMEOUT in its device status word, let every role of the CTA fall through to the teardown
@@ -10,6 +11,7 @@ usable: a normal call right after it must still meet the parity bound against th
 """
 import ctypes
 import os
+import re
 import time
 
 import pytest
@@ -35,6 +37,11 @@ def starve_lib():
     L.fa_device_status.restype = i
     L.fa_last_error.argtypes = []
     L.fa_last_error.restype = ctypes.c_char_p
+    sz = ctypes.c_size_t
+    L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    L.fa_bwd_workspace_size.restype = sz
+    L.fa_bwd.argtypes = [vp] * 9 + [i] * 5 + [f, vp, sz, vp]
+    L.fa_bwd.restype = i
     return L
 
 
@@ -95,3 +102,44 @@ def test_starve_build_is_otherwise_the_same_library():
     assert L.fa_device_status(stream) == fa.FA_OK
     O, Lr = attention_forward(f64["q"], f64["k"], f64["v"], True, s)
     assert_fwd(to_np(o), O, to_np(lse), Lr, "starve build, single key tile")
+
+
+def test_starved_pair_backward_reports_timeout_and_context_survives():
+    """The d = 256 backward runs on two-CTA clusters that exchange tiles through each other's
+    shared memory.  With one dO tile of the first cluster never issued, a bounded wait runs out
+    on one CTA, the abort reaches the other through its abort flag, both tear down (each sender
+    waits, bounded, for the hand-back of the tiles it sent, then the cluster barrier), and the
+    call returns with FA_ERR_TIMEOUT and a usable context."""
+    import torch
+    L = starve_lib()
+    B, H, N, d = 1, 1, 256, 256
+    dev, f64 = cuda_inputs(B, H, N, d, seed=43)
+    s = ai.default_scale(d)
+    o, lse = fa.forward(dev["q"], dev["k"], dev["v"], True, s)  # product library: O and L
+    torch.cuda.synchronize()
+    dq, dk, dv = (torch.empty_like(dev[t]) for t in ("q", "k", "v"))
+    ws = torch.empty(L.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    t0 = time.perf_counter()
+    rc = L.fa_bwd(dev["q"].data_ptr(), dev["k"].data_ptr(), dev["v"].data_ptr(), o.data_ptr(),
+                  lse.data_ptr(), dev["do"].data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                  dv.data_ptr(), B, H, N, d, 1, s, ws.data_ptr(), ws.numel(), stream)
+    assert rc == fa.FA_OK, L.fa_last_error()
+    status = L.fa_device_status(stream)  # synchronises the stream
+    elapsed = time.perf_counter() - t0
+    assert status == fa.FA_ERR_TIMEOUT, (status, L.fa_last_error())
+    msg = L.fa_last_error().decode()
+    m = re.search(r"site (\d+)", msg)
+    assert m and 70 <= int(m.group(1)) <= 89, msg  # a wait of the pair kernel
+    # 1 ms wait bound, 20 ms hand-back bound in this build: well under a second
+    assert elapsed < 1.0, elapsed
+    assert L.fa_device_status(stream) == fa.FA_OK
+
+    # the context is intact: the product library's d = 256 backward meets parity
+    dq, dk, dv = fa.backward(dev["q"], dev["k"], dev["v"], o, lse, dev["do"], True, s)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == fa.FA_OK
+    O, Lr = attention_forward(f64["q"], f64["k"], f64["v"], True, s)
+    assert_fwd(to_np(o), O, to_np(lse), Lr, "d=256 after the starved pair")
+    g = attention_backward(f64["q"], f64["k"], f64["v"], O, Lr, f64["do"], True, s)
+    assert_bwd(tuple(to_np(t) for t in (dq, dk, dv)), g, "d=256 after the starved pair")
