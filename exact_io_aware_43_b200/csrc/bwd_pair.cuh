@@ -237,7 +237,9 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmdO,
-                       const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
+                       const __grid_constant__ CUtensorMap tmdQ,
+                       const __grid_constant__ CUtensorMap tmdK,
+                       const __grid_constant__ CUtensorMap tmdV, const BwdParams p) {
   using C = BwdPairCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -524,16 +526,40 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
       ok = W.wait_warp(bar(C::B_DRAIN), 0, 85);
       if (ok) {
         tc_fence_after();
-        const size_t base = (size_t(kvh) * p.N + key) * C::D + 128 * h;
         const float mul = role == 0 ? p.scale : 1.f;
-        __nv_bfloat16* dst = (role == 0 ? p.dk : p.dv) + base;
-        float* acc = p.gsplit > 1 ? (role == 0 ? p.dk_acc : p.dv_acc) + base : nullptr;
+        if (p.gsplit > 1) {
+          // a group's query heads split over CTAs: fp32 reduce-adds into the accumulators
+          const size_t base = (size_t(kvh) * p.N + key) * C::D + 128 * h;
+          float* acc = (role == 0 ? p.dk_acc : p.dv_acc) + base;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t vv[32];
-          tmem_ld32(tmem + lane_base + C::T_ACC + 128 * h + 32 * c, vv);
-          tmem_wait_ld(vv);
-          bwd_store_chunk(vv, mul, key_ok, dst + 32 * c, acc ? acc + 32 * c : nullptr);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t vv[32];
+            tmem_ld32(tmem + lane_base + C::T_ACC + 128 * h + 32 * c, vv);
+            tmem_wait_ld(vv);
+            bwd_store_chunk(vv, mul, key_ok, nullptr, acc + 32 * c);
+          }
+        } else {
+          // staged as a swizzled tile (d columns [128h, 128h + 128): two 64-column blocks) in
+          // stage h, no longer read once every MMA has completed, then written by TMA tensor
+          // stores in whole rows (rows past N are clipped)
+          uint8_t* tile = smem + C::OFF_S + h * C::STAGE;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t vv[32];
+            tmem_ld32(tmem + lane_base + C::T_ACC + 128 * h + 32 * c, vv);
+            tmem_wait_ld(vv);
+            bwd_stage_chunk(vv, mul, tile, r, c);
+          }
+          fence_async_smem();
+          named_bar_sync(1 + h, 128);
+          if ((warp & 3) == 0 && lane == 0) {
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb)
+              tma_store_3d(role == 0 ? &tmdK : &tmdV, stage_addr(h) + kb * C::KV_BLK,
+                           (2 * h + kb) * 64, k0, kvh);
+            bulk_commit_group();
+            bulk_wait_group_read<0>();  // the tile is read before the CTA's memory goes away
+          }
         }
       }
     }

@@ -142,7 +142,9 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmdO,
-                       const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
+                       const __grid_constant__ CUtensorMap tmdQ,
+                       const __grid_constant__ CUtensorMap tmdK,
+                       const __grid_constant__ CUtensorMap tmdV, const BwdParams p) {
   using C = BwdQ128Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the swizzled tiles need a 1024-byte-aligned base; with the largest layouts there is less
@@ -158,6 +160,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   FA_TRACE_DECL;
+  FA_TRACE_EV(90, 0);  // CTA start
 
   // ---- work unit: (key block j, key/value head) in the order of BwdUnit; for each query head
   // of the group (see BwdGroup), query blocks i from j (causal) or 0 to the last
@@ -219,6 +222,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
     fence_async_smem();
   }
   __syncthreads();
+  FA_TRACE_EV(91, 0);  // set-up done
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -325,7 +329,9 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
         return true;
       };
       bool ok = W.wait(BAR_KV, 0, 40);
+      FA_TRACE_EV(92, 0);  // K_j, V_j landed
       if (ok) ok = W.wait(BAR_QF(0), 0, 41);
+      FA_TRACE_EV(93, 0);  // first Q_i landed
       if (ok) {
         tc_fence_after();
         issue_st(C::T_S, k_addr, q_addr(0), ones_s, aug_addr(0));
@@ -500,19 +506,43 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
     if (ok) {
       // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale), bf16
       ok = W.wait_warp(BAR_DKD, (nit - 1) & 1, 55);
+      FA_TRACE_EV(94, 0);  // epilogue start
       if (ok) {
         tc_fence_after();
-        const size_t base = (size_t(kvh) * p.N + key) * C::D;
         const uint32_t col = h == 0 ? C::T_DV : C::T_DK;
         const float mul = h == 0 ? 1.f : p.scale;
-        __nv_bfloat16* dst = (h == 0 ? p.dv : p.dk) + base;
-        float* acc = p.gsplit > 1 ? (h == 0 ? p.dv_acc : p.dk_acc) + base : nullptr;
+        if (p.gsplit > 1) {
+          // a group's query heads split over CTAs: fp32 reduce-adds into the accumulators
+          const size_t base = (size_t(kvh) * p.N + key) * C::D;
+          float* acc = (h == 0 ? p.dv_acc : p.dk_acc) + base;
 #pragma unroll
-        for (int c = 0; c < C::D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_base + col + 32 * c, v);
-          tmem_wait_ld(v);
-          bwd_store_chunk(v, mul, key_ok, dst + 32 * c, acc ? acc + 32 * c : nullptr);
+          for (int c = 0; c < C::D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_base + col + 32 * c, v);
+            tmem_wait_ld(v);
+            bwd_store_chunk(v, mul, key_ok, nullptr, acc + 32 * c);
+          }
+        } else {
+          // staged as a swizzled tile in Q stage h (no longer read: every MMA has completed),
+          // then written by TMA tensor stores in whole rows (rows past N are clipped)
+          uint8_t* tile = smem + C::OFF_Q + h * C::TILE;
+#pragma unroll
+          for (int c = 0; c < C::D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_base + col + 32 * c, v);
+            tmem_wait_ld(v);
+            bwd_stage_chunk(v, mul, tile, r, c);
+          }
+          fence_async_smem();
+          named_bar_sync(1 + h, 128);
+          if ((warp & 3) == 0 && lane == 0) {
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb)
+              tma_store_3d(h == 0 ? &tmdV : &tmdK, sbase + C::OFF_Q + h * C::TILE + kb * C::BLK,
+                           kb * 64, k0, kvh);
+            bulk_commit_group();
+            bulk_wait_group_read<0>();  // the tile is read before the CTA's memory goes away
+          }
         }
       }
     }
@@ -572,6 +602,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
     tc_fence_before();
   }
 
+  FA_TRACE_EV(95, 0);  // role done
   __syncthreads();
   if (warp == C::MMA_WARP) {
     tc_fence_after();

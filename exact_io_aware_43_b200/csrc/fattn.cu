@@ -347,10 +347,14 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
     if ((rc = make_map(&mq, q, p.BH, p.N, D, CQ::BR))) return rc;
     if ((rc = make_map(&mdo, p.dO, p.BH, p.N, D, CQ::BR))) return rc;
     if ((rc = make_map_f32(&mdq, p.dq_acc, p.BH, p.N, D, CQ::DW, 32))) return rc;  // per warp
+    // dK, dV written by TMA tensor stores from swizzled shared tiles (same boxes as K, V)
+    CUtensorMap mdk, mdv;
+    if ((rc = make_map(&mdk, p.dk, p.BHkv, p.N, D, CQ::BC))) return rc;
+    if ((rc = make_map(&mdv, p.dv, p.BHkv, p.N, D, CQ::BC))) return rc;
     dim3 grid(unsigned(p.BHkv) * unsigned(p.nkb) * unsigned(p.gsplit));
     {
       TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
-      kq<<<grid, CQ::THREADS, CQ::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, p);
+      kq<<<grid, CQ::THREADS, CQ::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p);
     }
   } else if (D == 256 && FA_BWD_PAIR) {
     using CP = fattn::BwdPairCfg;
@@ -361,6 +365,9 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
     if ((rc = make_map(&mk, k, p.BHkv, p.N, D, CP::BC))) return rc;
     if ((rc = make_map(&mv, v, p.BHkv, p.N, D, CP::BC))) return rc;
     if ((rc = make_map_f32(&mdq, p.dq_acc, p.BH, p.N, D, 32, 32))) return rc;  // per drain warp
+    CUtensorMap mdk, mdv;  // dK, dV written by TMA tensor stores (same boxes as K, V)
+    if ((rc = make_map(&mdk, p.dk, p.BHkv, p.N, D, CP::BC))) return rc;
+    if ((rc = make_map(&mdv, p.dv, p.BHkv, p.N, D, CP::BC))) return rc;
     // one cluster of two CTAs per (key block, key/value head [, share of the group's heads])
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(2u * unsigned(p.BHkv) * unsigned(p.nkb) * unsigned(p.gsplit));
@@ -376,7 +383,7 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
     cfg.numAttrs = 1;
     {
       TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
-      e = cudaLaunchKernelEx(&cfg, kp, mq, mk, mv, mdo, mdq, p);
+      e = cudaLaunchKernelEx(&cfg, kp, mq, mk, mv, mdo, mdq, mdk, mdv, p);
     }
     if (e != cudaSuccess) return cuda_fail(e, "fa_bwd (pair) launch");
   } else {
