@@ -548,7 +548,7 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
             uint32_t vv[32];
             tmem_ld32(tmem + lane_base + C::T_ACC + 128 * h + 32 * c, vv);
             tmem_wait_ld(vv);
-            bwd_stage_chunk(vv, mul, tile, r, c);
+            stage_chunk_sw128(vv, mul, tile, r, c);
           }
           fence_async_smem();
           named_bar_sync(1 + h, 128);

@@ -531,7 +531,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
             uint32_t v[32];
             tmem_ld32(tmem + lane_base + col + 32 * c, v);
             tmem_wait_ld(v);
-            bwd_stage_chunk(v, mul, tile, r, c);
+            stage_chunk_sw128(v, mul, tile, r, c);
           }
           fence_async_smem();
           named_bar_sync(1 + h, 128);

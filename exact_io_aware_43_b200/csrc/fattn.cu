@@ -219,7 +219,7 @@ int sm_count() {
 
 template <int D, bool CAUSAL, int NQT>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-               fattn::FwdParams p, int BH, cudaStream_t st) {
+               const CUtensorMap& mo, fattn::FwdParams p, int BH, cudaStream_t st) {
   using C = fattn::FwdCfg<D, NQT>;
   const bool general = p.o_part != nullptr || p.pack > 1;
   auto kern = general ? fattn::fa_fwd_kernel<D, CAUSAL, NQT, true>
@@ -256,7 +256,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   const int G = FA_FWD_PERSISTENT ? (p.units < sm_count() ? p.units : sm_count()) : p.units;
   dim3 grid(static_cast<unsigned>(G));
   TimedLaunch tl(FA_KERNEL_FWD, st);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, p);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fa_fwd launch");
   return FA_OK;
@@ -440,6 +440,11 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((rc = pack ? make_map(&mq, q, BH, Nq, d, Nq, G) : make_map(&mq, q, BH, Nq, d, 128))) return rc;
   if ((rc = make_map(&mk, k, B * H_kv, Nk, d, 128))) return rc;
   if ((rc = make_map(&mv, v, B * H_kv, Nk, d, 128))) return rc;
+  // O map for the TMA stores of the plain forward (split and packed outputs store rows
+  // directly; they get a placeholder)
+  CUtensorMap mo = mq;
+  const bool plain_out = !(splits > 1 || partials) && !pack;
+  if (plain_out && (rc = make_map(&mo, o, BH, Nq, d, 128))) return rc;
   fattn::FwdParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -460,20 +465,20 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
   // freed second query buffer deepens the K/V ring
   if (d == 64) {
     if (pack)
-      return causal ? launch_fwd<64, true, 1>(mq, mk, mv, p, BH, st)
-                    : launch_fwd<64, false, 1>(mq, mk, mv, p, BH, st);
-    return causal ? launch_fwd<64, true, 2>(mq, mk, mv, p, BH, st)
-                  : launch_fwd<64, false, 2>(mq, mk, mv, p, BH, st);
+      return causal ? launch_fwd<64, true, 1>(mq, mk, mv, mo, p, BH, st)
+                    : launch_fwd<64, false, 1>(mq, mk, mv, mo, p, BH, st);
+    return causal ? launch_fwd<64, true, 2>(mq, mk, mv, mo, p, BH, st)
+                  : launch_fwd<64, false, 2>(mq, mk, mv, mo, p, BH, st);
   }
   if (d == 128) {
     if (pack)
-      return causal ? launch_fwd<128, true, 1>(mq, mk, mv, p, BH, st)
-                    : launch_fwd<128, false, 1>(mq, mk, mv, p, BH, st);
-    return causal ? launch_fwd<128, true, 2>(mq, mk, mv, p, BH, st)
-                  : launch_fwd<128, false, 2>(mq, mk, mv, p, BH, st);
+      return causal ? launch_fwd<128, true, 1>(mq, mk, mv, mo, p, BH, st)
+                    : launch_fwd<128, false, 1>(mq, mk, mv, mo, p, BH, st);
+    return causal ? launch_fwd<128, true, 2>(mq, mk, mv, mo, p, BH, st)
+                  : launch_fwd<128, false, 2>(mq, mk, mv, mo, p, BH, st);
   }
-  return causal ? launch_fwd<256, true, 1>(mq, mk, mv, p, BH, st)
-                : launch_fwd<256, false, 1>(mq, mk, mv, p, BH, st);
+  return causal ? launch_fwd<256, true, 1>(mq, mk, mv, mo, p, BH, st)
+                : launch_fwd<256, false, 1>(mq, mk, mv, mo, p, BH, st);
 }
 
 int bwd_dispatch(const void* q, const void* k, const void* v, const void* o, const float* lse,

@@ -123,7 +123,15 @@ struct FwdCfg {
   static constexpr int OFF_K = OFF_Q + NQT * QTILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KVTILE_BYTES;
   static constexpr int OFF_ONES = OFF_V + STAGES * KVTILE_BYTES;  // [BN keys][64] bf16 ones
-  static constexpr int OFF_BAR = OFF_ONES + (EXTRA ? BN * 128 : 0);
+  // O written by TMA tensor stores from swizzled shared blocks of [128 rows][64 columns] (16 KB):
+  // one per query tile at d = 64 (two tiles), two alternating at d = 256.  d = 128 stores its
+  // rows directly: there the staging's warpgroup barriers cost more than the stores save (long
+  // causal forward 1023 vs 1044 TFLOP/s), and the one-tile configurations of d = 64 / 128 have no
+  // room for it.
+  static constexpr bool TMA_EPI = (NQT == 2 && D == 64) || D == 256;
+  static constexpr int STG_BLK = BM * 128;
+  static constexpr int OFF_STG = OFF_ONES + (EXTRA ? BN * 128 : 0);
+  static constexpr int OFF_BAR = OFF_STG + (TMA_EPI ? 2 * STG_BLK : 0);
   // barriers: q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NB],
   //           p_full[NB], o_done[NB], o_free[NQT], drain (slot = query tile, or with one query
   //           tile the S buffer)
@@ -199,7 +207,8 @@ struct FwdUnit {
 template <int D, bool CAUSAL, int NQT, bool SPLIT>
 __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const FwdParams p) {
   using C = FwdCfg<D, NQT>;
   using Unit = FwdUnit<NQT, CAUSAL, SPLIT>;
   extern __shared__ uint8_t smem_raw[];
@@ -850,6 +859,44 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         lr = __uint_as_float(o[0]);
       }
       const float inv_l = (!SPLIT || lr > 0.f) ? 1.f / lr : 0.f;
+      if constexpr (!SPLIT && C::TMA_EPI) {
+        // O / l as bf16 into this warpgroup's staging block(s), one 64-column block at a time,
+        // each written by a TMA tensor store in whole rows (rows past Nq are clipped)
+        constexpr int NBUF = NQT == 2 ? 1 : 2;
+        uint8_t* stg = smem + C::OFF_STG + (NQT == 2 ? t * C::STG_BLK : 0);
+        const bool issuer = (warp & 3) == 0 && lane == 0;
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb) {
+          uint8_t* buf = stg + (kb % NBUF) * C::STG_BLK;
+          // the previous store out of this block (this unit's or the last unit's) has read it
+          if (issuer) {
+            if (NBUF == 1) bulk_wait_group_read<0>();
+            else bulk_wait_group_read<1>();
+          }
+          named_bar_sync(1 + t, 128);
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const int c = 2 * kb + c2;
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_wait_ld(o);
+            if (c == D / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(BAR_OF(t));
+            }
+            stage_chunk_sw128(o, inv_l, buf, r, c2);
+          }
+          fence_async_smem();
+          named_bar_sync(1 + t, 128);
+          if (issuer) {
+            tma_store_3d(&tmO, smem_u32(buf), kb * 64, un.q0 + t * C::BM, un.head);
+            bulk_commit_group();
+          }
+        }
+        if (valid) p.lse[size_t(qh) * p.Nq + row] = (m + lg2(l)) * 0.69314718055994531f;
+        continue;
+      }
       const bool part = SPLIT && p.o_part != nullptr;
       const size_t prow = (size_t(un.split) * p.BH + qh) * p.Nq + row;
       __nv_bfloat16* orow = p.o + (size_t(qh) * p.Nq + row) * D;
@@ -894,6 +941,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           p.lse[size_t(qh) * p.Nq + row] = L;
       }
     }
+    // the last O stores have read their staging blocks before the CTA's memory goes away
+    if constexpr (!SPLIT && C::TMA_EPI)
+      if ((warp & 3) == 0 && lane == 0) bulk_wait_group_all();
     tc_fence_before();
   }
 

@@ -549,4 +549,23 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// One 32-column chunk (columns 32c .. 32c + 31) of row r of an output tile (O, dK, dV), x mul, as
+// bf16 into a shared tile laid out like a TMA tile with 128-byte swizzle: 64-column blocks of
+// [128 rows][128 bytes], the 16-byte chunk k of row r at position k ^ (r & 7).  A TMA tensor
+// store then writes the tile to global memory in whole rows.
+__device__ __forceinline__ void stage_chunk_sw128(const uint32_t (&v)[32], float mul, uint8_t* tile,
+                                                int r, int c) {
+  uint8_t* row = tile + (c >> 1) * (128 * 128) + r * 128;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    uint4 q;
+    q.x = pack_bf16(__uint_as_float(v[8 * e]) * mul, __uint_as_float(v[8 * e + 1]) * mul);
+    q.y = pack_bf16(__uint_as_float(v[8 * e + 2]) * mul, __uint_as_float(v[8 * e + 3]) * mul);
+    q.z = pack_bf16(__uint_as_float(v[8 * e + 4]) * mul, __uint_as_float(v[8 * e + 5]) * mul);
+    q.w = pack_bf16(__uint_as_float(v[8 * e + 6]) * mul, __uint_as_float(v[8 * e + 7]) * mul);
+    const int k = (c & 1) * 4 + e;
+    *reinterpret_cast<uint4*>(row + ((k ^ (r & 7)) << 4)) = q;
+  }
+}
+
 }  // namespace fattn
