@@ -11,24 +11,27 @@
 // therefore split the work by what they accumulate, and compute every product once:
 //
 //   CTA 0 ("S" CTA):  K_j resident, Q_i streamed.  S^T -> P^T (exponentials) -> P^T into CTA 1's
-//                     shared memory;  dK_j += dS^T Q_i and dQ_i += dS K_j with dS^T received
-//                     from CTA 1.
-//   CTA 1 ("dP" CTA): V_j resident, dO_i streamed.  dP^T;  dS^T = P^T (dP^T - D) with P^T
-//                     received from CTA 0 -> dS^T into CTA 0's shared memory;  dV_j += P^T dO_i.
+//                     shared memory;  dK_j += dS^T Q_i and dQ_i[:, 0:128] += dS K_j[:, 0:128] with
+//                     the dS^T it receives.
+//   CTA 1 ("dP" CTA): V_j resident in TENSOR memory (the A operand of dP^T), K_j[:, 128:256] in
+//                     shared memory, dO_i streamed.  dP^T;  dS^T = P^T (dP^T - D) with the P^T it
+//                     receives -> dS^T into CTA 0's shared memory and its own;  dV_j += P^T dO_i
+//                     and dQ_i[:, 128:256] += dS K_j[:, 128:256].
 //
-// Per step CTA 0 issues six 128 x 64 x 128-equivalent GEMM units (S^T: two, dK: two, dQ: two)
-// and CTA 1 four (dP^T, dV), ten in all, where two independent CTAs that each recompute S^T and
-// dP^T for a 128-wide slice of d issue fourteen.  The exchanged tiles (P^T and dS^T, 16 KB each
-// per step) travel as asynchronous remote stores (st.async) whose bytes complete a transaction
-// count on the receiver's mbarrier, so the data announces its own arrival; each side has two
-// buffers, and a buffer is handed back (a remote arrival) once its last reader -- an MMA, and
-// for P^T also CTA 1's dS warps -- has finished.
+// Each CTA issues five 128 x 64 x 128-equivalent GEMM units per step, ten in all, where two
+// independent CTAs that each recompute S^T and dP^T for a 128-wide slice of d issue fourteen, and
+// each reduces half of dQ.  Keeping V_j in tensor memory is what makes room in CTA 1's shared
+// memory for K_j's upper half, two dS^T tiles and dQ staging.  The exchanged tiles (P^T and dS^T,
+// 16 KB each per step) travel as asynchronous remote stores (st.async) whose bytes complete a
+// transaction count on the receiver's mbarrier, so the data announces its own arrival; each side
+// has two buffers, and a buffer is handed back (a remote arrival) once its last reader -- an MMA,
+// and for P^T also CTA 1's dS warps -- has finished.
 //
 // Warp roles: warps 0-7 exponentials (CTA 0) or dS (CTA 1), thread = key row = TMEM lane, the two
-// warpgroups on query columns [0, 32) and [32, 64) of every step (FA_PAIR_SPLIT); warps 8-11 of
-// CTA 0 drain dQ^T (32 d rows each, two 4 KB staging blocks each) into the fp32 accumulator with
-// TMA bulk reduce-adds, and warp 8 of CTA 1 hands P^T tiles back; warp 12 issues TMA loads;
-// warp 13 allocates tensor memory and issues the MMAs, as independent ready-driven streams.
+// warpgroups on query columns [0, 32) and [32, 64) of every step; warps 8-11 drain this CTA's
+// dQ^T half (32 d rows each, two 4 KB staging blocks each) into the fp32 accumulator with TMA
+// bulk reduce-adds; warp 12 issues TMA loads; warp 13 allocates tensor memory and issues the
+// MMAs as independent ready-driven streams; warp 14 of CTA 1 hands P^T tiles back.
 //
 // Every wait is bounded.  A CTA that gives up sets its own and its peer's abort flag, so both
 // fall through to the teardown, where each sender first waits (bounded) for the hand-back of its
@@ -174,11 +177,6 @@ struct PairWaiter {
   }
 };
 
-// FA_PAIR_SPLIT: 1, both warpgroups of exponential / dS warps work on every step (32 query
-// columns each); 0, they take alternate steps (64 columns each).
-#ifndef FA_PAIR_SPLIT
-#define FA_PAIR_SPLIT 1
-#endif
 // FA_PAIR_POLL_NS: the MMA thread's pause between rounds of barrier probes that found nothing
 // ready (nanoseconds).
 #ifndef FA_PAIR_POLL_NS
@@ -194,40 +192,51 @@ struct BwdPairCfg {
   static constexpr int STAGE = 4 * Q_BLK;        // a Q_i or dO_i tile, [64][256]: 32 KB
   static constexpr int XT = BC * BR * 2;         // a P^T or dS^T tile, [128 keys][64 q]: 16 KB
   static constexpr int NS = 3;                   // Q_i (CTA 0) or dO_i (CTA 1) stages
-  static constexpr bool SPLIT = FA_PAIR_SPLIT != 0;
-  static constexpr int WPS = SPLIT ? 8 : 4;      // exponential / dS warps per step
+  static constexpr int WPS = 8;                  // exponential / dS warps, all on every step
   // shared memory map (both CTAs use the same offsets; remote stores address the peer's copy)
-  static constexpr int OFF_A = 0;                    // K_j (CTA 0) or V_j (CTA 1): 64 KB
-  static constexpr int OFF_S = OFF_A + 4 * KV_BLK;   // 3 stages of Q_i (CTA 0) or dO_i (CTA 1)
-  static constexpr int OFF_X = OFF_S + 3 * STAGE;    // 2 tiles the peer writes: dS^T (CTA 0) / P^T (CTA 1)
-  static constexpr int OFF_STG = OFF_X + 2 * XT;     // CTA 0: dQ staging, 2 x 4 KB per drain warp
+  //   OFF_A   CTA 0: K_j (64 KB).  CTA 1: K_j[:, 128:256] (32 KB), then its two dS^T tiles.
+  //   OFF_S   NS stages of Q_i (CTA 0) or dO_i (CTA 1); CTA 1 first stages V_j in the first two
+  //           on its way into tensor memory
+  //   OFF_X   the two tiles the peer writes: dS^T (CTA 0) / P^T (CTA 1)
+  //   OFF_STG dQ staging, 2 x 4 KB per drain warp
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_DSL = OFF_A + 2 * KV_BLK;  // CTA 1: dS^T tiles
+  static constexpr int OFF_S = OFF_A + 4 * KV_BLK;
+  static constexpr int OFF_X = OFF_S + NS * STAGE;
+  static constexpr int OFF_STG = OFF_X + 2 * XT;
   static constexpr int OFF_ROWS = OFF_STG + 8 * 4096;  // per stage 64 floats: L2 (CTA 0) / D (CTA 1)
-  static constexpr int NBAR = 20;
+  static constexpr int NBAR = 26;
   static constexpr int OFF_BAR = OFF_ROWS + NS * BR * 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr int THREADS = 448;
-  static constexpr int DQ_WARP0 = 8, PRODUCER_WARP = 12, MMA_WARP = 13;
+  static constexpr int THREADS = 480;
+  static constexpr int DQ_WARP0 = 8, PRODUCER_WARP = 12, MMA_WARP = 13, RELAY_WARP = 14;
   // tensor memory columns
-  static constexpr int T_A = 0;      // two 64-column buffers: S^T (CTA 0) / dP^T (CTA 1)
-  static constexpr int T_ACC = 128;  // 256 columns: dK (CTA 0) / dV (CTA 1)
-  static constexpr int T_DQ = 384;   // CTA 0: dQ^T, two 64-column halves (d on lanes)
+  //   CTA 0: S^T buffers [0, 128), dK [128, 384), dQ^T half 0 [384, 448)
+  //   CTA 1: V_j as bf16 pairs (A operand of dP^T) [0, 128), dP^T [128, 192), dQ^T half 1
+  //          [192, 256), dV [256, 512)
+  static constexpr int T_S = 0, T_DK = 128, T_DQ0 = 384;
+  static constexpr int T_V = 0, T_DP = 128, T_DQ1 = 192, T_DV = 256;
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t IDESC_ST = idesc_bf16_f32(BC, BR, 0, 0);   // S^T, dP^T
   static constexpr uint32_t IDESC_ACC = idesc_bf16_f32(BC, D, 0, 1);   // dK, dV (N = 256)
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, BR, 1, 1);  // a dQ^T half = K_h^T dS^T
   // barriers
-  static constexpr int B_KV = 0;
-  static constexpr int B_LF = 1;      // + s: stage s loaded
-  static constexpr int B_LE = 4;      // + s: stage s free (MMA commit + the step's WPS warps)
-  static constexpr int B_AF = 7;      // + b: S^T / dP^T buffer b computed
-  static constexpr int B_AFREE = 9;   // + b: S^T / dP^T buffer b read out (WPS warps)
-  static constexpr int B_XF = 11;     // + b: exchange tile b written by the peer (WPS remote warps)
-  static constexpr int B_XE = 13;     // + b: the peer's exchange tile b is free (1 remote arrival)
-  static constexpr int B_XR = 15;     // + b: CTA 1: P^T tile b read (MMA commit + WPS warps)
-  static constexpr int B_DQF = 17;    // CTA 0: this step's dK and dQ^T MMAs complete
-  static constexpr int B_DQE = 18;    // CTA 0: dQ^T read out of tensor memory (4 drain warps)
-  static constexpr int B_DRAIN = 19;
+  static constexpr int B_KV = 0;      // resident K_j (CTA 0) / K_j[:, 128:256] (CTA 1) landed
+  static constexpr int B_VL = 1;      // CTA 1: V_j landed in the staging area
+  static constexpr int B_VD = 2;      // CTA 1: V_j in tensor memory (8 warps)
+  static constexpr int B_LF = 3;      // + s: stage s loaded
+  static constexpr int B_LE = 6;      // + s: stage s free (MMA commit + the step's WPS warps)
+  static constexpr int B_AF = 9;      // + b: S^T / dP^T buffer b computed
+  static constexpr int B_AFREE = 11;  // + b: S^T / dP^T buffer b read out (WPS warps)
+  static constexpr int B_XF = 13;     // + b: exchange tile b written by the peer (WPS remote warps)
+  static constexpr int B_XE = 15;     // + b: the peer's exchange tile b is free (1 remote arrival)
+  static constexpr int B_XR = 17;     // + b: CTA 1: P^T tile b read (MMA commit + WPS warps)
+  static constexpr int B_DSL = 19;    // + b: CTA 1: own dS^T tile b written (WPS warps)
+  static constexpr int B_DSLE = 21;   // + b: CTA 1: own dS^T tile b read by dQ^T (MMA commit)
+  static constexpr int B_DQF = 23;    // this step's dQ^T half complete
+  static constexpr int B_DQE = 24;    // dQ^T read out of tensor memory (4 drain warps)
+  static constexpr int B_DRAIN = 25;
 };
 static_assert(BwdPairCfg::SMEM_BYTES <= 232448, "pair backward exceeds 227 KB of shared memory");
 
@@ -248,8 +257,9 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   FA_TRACE_DECL;
-  const uint32_t role = cluster_ctarank();  // 0: S^T, P, dK, dQ;  1: dP^T, dS, dV
+  const uint32_t role = cluster_ctarank();  // 0: S^T, P, dK, dQ[:, :128];  1: dP^T, dS, dV, dQ[:, 128:]
   const uint32_t peer = role ^ 1u;
+  const int NBA = role == 0 ? 2 : 1;  // S^T / dP^T buffers in tensor memory
 
   // ---- work unit (both CTAs of the cluster take the same one)
   const BwdUnit unit(int(blockIdx.x >> 1), p, 1);
@@ -267,6 +277,8 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_KV), 1);
+    mbar_init(bar(C::B_VL), 1);
+    mbar_init(bar(C::B_VD), 8);
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar(C::B_LF + s), 1);
       mbar_init(bar(C::B_LE + s), 1 + C::WPS);
@@ -277,6 +289,8 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
       mbar_init(bar(C::B_XF + b), C::WPS);
       mbar_init(bar(C::B_XE + b), 1);
       mbar_init(bar(C::B_XR + b), 1 + C::WPS);
+      mbar_init(bar(C::B_DSL + b), C::WPS);
+      mbar_init(bar(C::B_DSLE + b), 1);
     }
     mbar_init(bar(C::B_DQF), 1);
     mbar_init(bar(C::B_DQE), 4);
@@ -302,17 +316,30 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
     // ================================================================ TMA producer
     if (lane == 0) {
       const CUtensorMap* tmS = role == 0 ? &tmQ : &tmdO;  // the streamed operand
-      const CUtensorMap* tmA = role == 0 ? &tmK : &tmV;   // the resident one
       tma_prefetch_desc(tmS);
-      tma_prefetch_desc(tmA);
-      mbar_arrive_expect_tx(bar(C::B_KV), 4 * C::KV_BLK);
-      for (int kb = 0; kb < 4; ++kb)
-        tma_load_3d(sbase + C::OFF_A + kb * C::KV_BLK, tmA, bar(C::B_KV), kb * 64, k0, kvh);
+      tma_prefetch_desc(&tmK);
+      bool ok = true;
+      if (role == 0) {
+        mbar_arrive_expect_tx(bar(C::B_KV), 4 * C::KV_BLK);
+        for (int kb = 0; kb < 4; ++kb)
+          tma_load_3d(sbase + C::OFF_A + kb * C::KV_BLK, &tmK, bar(C::B_KV), kb * 64, k0, kvh);
+      } else {
+        tma_prefetch_desc(&tmV);
+        mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_BLK);
+        for (int kb = 2; kb < 4; ++kb)
+          tma_load_3d(sbase + C::OFF_A + (kb - 2) * C::KV_BLK, &tmK, bar(C::B_KV), kb * 64, k0,
+                      kvh);
+        // V_j through the first two stages into tensor memory; the stages stream dO_i after
+        mbar_arrive_expect_tx(bar(C::B_VL), 4 * C::KV_BLK);
+        for (int kb = 0; kb < 4; ++kb)
+          tma_load_3d(sbase + C::OFF_S + kb * C::KV_BLK, &tmV, bar(C::B_VL), kb * 64, k0, kvh);
+        ok = W.wait(bar(C::B_VD), 0, 69);
+      }
       const float* rows_src = role == 0 ? p.L2 : p.Drow;
       int it = 0;
       bool starved = false;
       BwdCursor cur(grp);
-      for (; it < nit; ++it) {
+      for (; ok && it < nit; ++it) {
         const int i = cur.i, head = cur.head;
         cur.next();
         const int s = it % NS;
@@ -337,38 +364,50 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
       }
       if (W.aborted() || starved) {
         W.drain(bar(C::B_KV), 0);
+        if (role == 1) W.drain(bar(C::B_VL), 0);
         for (int jj = max(0, it - NS); jj < it; ++jj)
           W.drain(bar(C::B_LF + jj % NS), (jj / NS) & 1);
       }
     }
   } else if (warp == C::MMA_WARP) {
     // ================================================================ MMA issuer
-    // Independent streams, each in step order: S^T(t) / dP^T(t) (as soon as its tile has landed
-    // and its tensor-memory buffer has been read out); the product that needs the peer's tile
-    // of step t (dK for CTA 0, dV for CTA 1), after which the stage is released; and, for CTA 0,
-    // dQ^T(t) (which also needs the drain to have read dQ^T(t-1)).  The thread issues whichever
-    // is ready, so none waits behind another.
+    // Three independent streams, each in step order, issued as they become ready: A, S^T(t)
+    // (CTA 0, two buffers) or dP^T(t) (CTA 1, one buffer; A operand V_j from tensor memory), once
+    // the stage has landed and the buffer has been read out; B, dK (CTA 0) or dV (CTA 1), once
+    // the peer's tile of step t has arrived -- the stage is then released; C, this CTA's dQ^T
+    // half, once its dS^T tile is there (the received one on CTA 0, the CTA's own on CTA 1) and
+    // the drain has read dQ^T(t-1).
     if (lane == 0) {
-      const uint32_t a_addr = sbase + C::OFF_A;  // K_j (CTA 0) or V_j (CTA 1)
-      auto issue_a = [&](int b, uint32_t st_addr) {
-        // S^T or dP^T (128 x 64, K = 256) into buffer b; A = K_j / V_j, B = Q_i / dO_i, K-major
-#pragma unroll
-        for (int kk = 0; kk < C::D / 16; ++kk)
-          mma_ss(tmem + C::T_A + 64 * b,
-                 sdesc_sw128(a_addr + (kk >> 2) * C::KV_BLK + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(st_addr + (kk >> 2) * C::Q_BLK + (kk & 3) * 32, 16, 1024),
-                 C::IDESC_ST, kk > 0);
-      };
+      const uint32_t a_addr = sbase + C::OFF_A;  // K_j (CTA 0) or K_j[:, 128:256] (CTA 1)
       bool ok = W.wait(bar(C::B_KV), 0, 71);
-      int ns = 0, na = 0, nq = 0;  // next S^T / dP^T step, next dK / dV step, next dQ^T step
+      if (ok && role == 1) ok = W.wait(bar(C::B_VD), 0, 78);
+      int ns = 0, na = 0, nq = 0;  // next step of streams A, B, C
       uint64_t t_last = global_ns();
-      while (ok && (na < nit || (role == 0 && nq < nit))) {
+      const uint32_t t_dq = role == 0 ? C::T_DQ0 : C::T_DQ1;
+      while (ok && (na < nit || nq < nit)) {
         bool progress = false;
         if (ns < nit && mbar_test_wait(bar(C::B_LF + ns % NS), (ns / NS) & 1) &&
-            mbar_test_wait(bar(C::B_AFREE + (ns & 1)), ((ns >> 1) & 1) ^ 1)) {
+            mbar_test_wait(bar(C::B_AFREE + ns % NBA), ((ns / NBA) & 1) ^ 1)) {
           tc_fence_after();
-          issue_a(ns & 1, stage_addr(ns % NS));
-          tc_commit(bar(C::B_AF + (ns & 1)));
+          const uint32_t st_addr = stage_addr(ns % NS);
+          if (role == 0) {
+            // S^T (128 x 64, K = 256) = K_j Q_i^T, both K-major in shared memory
+#pragma unroll
+            for (int kk = 0; kk < C::D / 16; ++kk)
+              mma_ss(tmem + C::T_S + 64 * (ns & 1),
+                     sdesc_sw128(a_addr + (kk >> 2) * C::KV_BLK + (kk & 3) * 32, 16, 1024),
+                     sdesc_sw128(st_addr + (kk >> 2) * C::Q_BLK + (kk & 3) * 32, 16, 1024),
+                     C::IDESC_ST, kk > 0);
+          } else {
+            // dP^T (128 x 64, K = 256) = V_j dO_i^T: A = V_j from tensor memory (bf16 pairs,
+            // 8 columns per 16-deep step), B = dO_i K-major in shared memory
+#pragma unroll
+            for (int kk = 0; kk < C::D / 16; ++kk)
+              mma_ts(tmem + C::T_DP, tmem + C::T_V + kk * 8,
+                     sdesc_sw128(st_addr + (kk >> 2) * C::Q_BLK + (kk & 3) * 32, 16, 1024),
+                     C::IDESC_ST, kk > 0);
+          }
+          tc_commit(bar(C::B_AF + ns % NBA));
           FA_TRACE_EV(1, ns);
           ++ns;
           progress = true;
@@ -383,28 +422,29 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
           // (K-major, [128 keys][64 q]), B = Q_i / dO_i (MN-major, N = 256)
 #pragma unroll
           for (int kk = 0; kk < C::BR / 16; ++kk)
-            mma_ss(tmem + C::T_ACC, sdesc_sw128(x_addr + kk * 32, 16, 1024),
+            mma_ss(tmem + (role == 0 ? C::T_DK : C::T_DV), sdesc_sw128(x_addr + kk * 32, 16, 1024),
                    sdesc_sw128(stage_addr(s) + kk * 2048, C::Q_BLK, 1024), C::IDESC_ACC,
                    (na > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(bar(C::B_LE + s));  // the stage is read by nothing after this
+          tc_commit(bar(C::B_LE + s));  // the MMAs are the stage's last readers
           if (role == 1) tc_commit(bar(C::B_XR + b));
           FA_TRACE_EV(4, na);
           ++na;
           progress = true;
         }
-        if (role == 0 && nq < na && (nq == 0 || mbar_test_wait(bar(C::B_DQE), (nq - 1) & 1))) {
-          // dQ^T halves (128 d x 64 q, K = 128 keys): A = K_j[:, half]^T (MN-major, two
-          // 64-wide d blocks), B = the dS^T tile (MN-major)
+        if (nq < nit && (role == 0 ? nq < na
+                                   : mbar_test_wait(bar(C::B_DSL + (nq & 1)), (nq >> 1) & 1)) &&
+            (nq == 0 || mbar_test_wait(bar(C::B_DQE), (nq - 1) & 1))) {
+          // dQ^T half (128 d x 64 q, K = 128 keys): A = K_j[:, half]^T (MN-major, two 64-wide d
+          // blocks), B = the dS^T tile (MN-major)
           tc_fence_after();
-          const uint32_t x_addr = sbase + C::OFF_X + (nq & 1) * C::XT;
+          const uint32_t ds_addr = role == 0 ? sbase + C::OFF_X + (nq & 1) * C::XT
+                                             : sbase + C::OFF_DSL + (nq & 1) * C::XT;
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-            for (int kk = 0; kk < C::BC / 16; ++kk)
-              mma_ss(tmem + C::T_DQ + 64 * hf,
-                     sdesc_sw128(a_addr + 2 * hf * C::KV_BLK + kk * 2048, C::KV_BLK, 1024),
-                     sdesc_sw128(x_addr + kk * 2048, C::Q_BLK, 1024), C::IDESC_DQ, kk > 0);
+          for (int kk = 0; kk < C::BC / 16; ++kk)
+            mma_ss(tmem + t_dq, sdesc_sw128(a_addr + kk * 2048, C::KV_BLK, 1024),
+                   sdesc_sw128(ds_addr + kk * 2048, C::Q_BLK, 1024), C::IDESC_DQ, kk > 0);
           tc_commit(bar(C::B_DQF));
+          if (role == 1) tc_commit(bar(C::B_DSLE + (nq & 1)));
           FA_TRACE_EV(5, nq);
           ++nq;
           progress = true;
@@ -425,14 +465,12 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
     }
   } else if (warp < 8) {
     // ================================================================ exponentials / dS
-    // Thread = key row = TMEM lane.  FA_PAIR_SPLIT = 1: both warpgroups work on every step,
-    // warpgroup h on query columns [32h, 32h + 32), and step t uses buffers t & 1.  0: warpgroup
-    // h takes the steps t = h, h + 2, ... with all 64 columns (each has two step periods for its
-    // chain), and step t uses buffers h.
-    constexpr bool SPLIT = C::SPLIT;
-    constexpr int NCOL = SPLIT ? 32 : 64;  // query columns per thread and step
+    // Thread = key row = TMEM lane; both warpgroups work on every step, warpgroup h on query
+    // columns [32h, 32h + 32).  (Every warp waits on every phase of the per-step barriers, so
+    // no parity test can alias a phase two behind.)  Step t uses exchange tiles t & 1.
+    constexpr int NCOL = 32;  // query columns per thread and step
     const int h = warp >> 2;
-    const int c0 = SPLIT ? 32 * h : 0;
+    const int c0 = 32 * h;
     const int r = (warp & 3) * 32 + lane;  // key row within the block == TMEM lane
     const int key = k0 + r;
     const bool key_ok = key < p.N;
@@ -445,29 +483,57 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
     const uint32_t peer_xf1 = mapa_shared(bar(C::B_XF + 1), peer);
     bool ok = true;
     int sent = 0;  // steps whose tile this warp has sent to the peer
+    if (role == 1) {
+      // V_j into tensor memory as the dP^T MMA's A operand: row r (this thread's lane), d
+      // columns [128h, 128h + 128) of this warpgroup, bf16 pairs (even d in the low half)
+      if ((ok = W.wait_warp(bar(C::B_VL), 0, 79))) {
+#pragma unroll
+        for (int kb2 = 0; kb2 < 2; ++kb2) {
+          const int kb = 2 * h + kb2;
+          const uint8_t* vrow = smem + C::OFF_S + kb * C::KV_BLK + row_off;
+          uint32_t v[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 q4 = *reinterpret_cast<const uint4*>(vrow + ((c ^ (r & 7)) << 4));
+            v[4 * c] = q4.x;
+            v[4 * c + 1] = q4.y;
+            v[4 * c + 2] = q4.z;
+            v[4 * c + 3] = q4.w;
+          }
+          tmem_st32(tmem + lane_base + C::T_V + 32 * kb, v);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_VD));
+      }
+    }
     BwdCursor cur(grp);
-    if (!SPLIT && h == 1) cur.next();
-    for (int it = SPLIT ? 0 : h; it < nit; it += SPLIT ? 1 : 2) {
+    for (int it = 0; ok && it < nit; ++it) {
       const int i = cur.i;
       cur.next();
-      if (!SPLIT) cur.next();
-      const int s = it % NS, b = it & 1, u = it >> 1;  // stage, buffer, use of the buffer
-      if (!(ok = W.wait_warp(bar(C::B_AF + b), u & 1, 80))) break;
+      const int s = it % NS, b = it & 1, u = it >> 1;  // stage, exchange tile, its use
+      const int ba = it % NBA, ua = it / NBA;          // S^T / dP^T buffer, its use
+      if (!(ok = W.wait_warp(bar(C::B_AF + ba), ua & 1, 80))) break;
       if (!(ok = W.wait_warp(bar(C::B_LF + s), (it / NS) & 1, 81))) break;
       FA_TRACE_EV(10, it);
       tc_fence_after();
       uint32_t v[NCOL / 32][32];
+      const uint32_t t_a = role == 0 ? C::T_S + 64 * ba : C::T_DP;
 #pragma unroll
-      for (int q = 0; q < NCOL / 32; ++q)
-        tmem_ld32(tmem + lane_base + C::T_A + 64 * b + c0 + 32 * q, v[q]);
+      for (int q = 0; q < NCOL / 32; ++q) tmem_ld32(tmem + lane_base + t_a + c0 + 32 * q, v[q]);
 #pragma unroll
       for (int q = 0; q < NCOL / 32; ++q) tmem_wait_ld(v[q]);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_AFREE + b));
+      if (lane == 0) mbar_arrive(bar(C::B_AFREE + ba));
       FA_TRACE_EV(11, it);
       const float* rows = rows_smem + s * C::BR + c0;
-      if (role == 1 && !(ok = W.wait_warp(bar(C::B_XF + b), u & 1, 82))) break;  // P^T landed
+      if (role == 1) {
+        if (!(ok = W.wait_warp(bar(C::B_XF + b), u & 1, 82))) break;  // P^T landed
+        // own dS^T tile b is free once dQ^T of its previous use has read it
+        if (!(ok = W.wait_warp(bar(C::B_DSLE + b), (u & 1) ^ 1, 83))) break;
+      }
       // the peer's tile b is free once it has handed back the previous use
       if (!(ok = W.wait_warp(bar(C::B_XE + b), (u & 1) ^ 1, 84))) break;
       FA_TRACE_EV(16, it);
@@ -478,6 +544,7 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
       const int qbase = i * C::BR + c0;
       const bool need_mask = role == 0 && (!key_ok || (CAUSAL && key > qbase));
       const uint8_t* own_x = smem + C::OFF_X + b * C::XT + row_off;
+      uint8_t* own_ds = smem + C::OFF_DSL + b * C::XT + row_off;
 #pragma unroll
       for (int e = 0; e < NCOL / 8; ++e) {
         // columns c0 + 8e .. c0 + 8e + 7: one 16-byte chunk of the key's 128-byte tile row
@@ -508,14 +575,21 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
             pk[c] = pack_bf16(p0 * (__uint_as_float(v[e >> 2][cc]) - rv[2 * c]),
                               p1 * (__uint_as_float(v[e >> 2][cc + 1]) - rv[2 * c + 1]));
           }
+          // and into the CTA's own dS^T tile, for its dQ^T half
+          *reinterpret_cast<uint4*>(own_ds + ((ch ^ (r & 7)) << 4)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
         st_async_v4(px + ((ch ^ (r & 7)) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]), pxf);
       }
       ++sent;
+      if (role == 1) fence_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(bar(C::B_LE + s));               // this step's row vector has been read
-        if (role == 1) mbar_arrive(bar(C::B_XR + b));  // and its P^T tile
+        mbar_arrive(bar(C::B_LE + s));  // this step's row vector has been read
+        if (role == 1) {
+          mbar_arrive(bar(C::B_XR + b));   // its P^T tile too
+          mbar_arrive(bar(C::B_DSL + b));  // and the own dS^T tile is written
+        }
       }
       FA_TRACE_EV(17, it);
     }
@@ -527,6 +601,7 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
       if (ok) {
         tc_fence_after();
         const float mul = role == 0 ? p.scale : 1.f;
+        const uint32_t t_acc = role == 0 ? C::T_DK : C::T_DV;
         if (p.gsplit > 1) {
           // a group's query heads split over CTAs: fp32 reduce-adds into the accumulators
           const size_t base = (size_t(kvh) * p.N + key) * C::D + 128 * h;
@@ -534,7 +609,7 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t vv[32];
-            tmem_ld32(tmem + lane_base + C::T_ACC + 128 * h + 32 * c, vv);
+            tmem_ld32(tmem + lane_base + t_acc + 128 * h + 32 * c, vv);
             tmem_wait_ld(vv);
             bwd_store_chunk(vv, mul, key_ok, nullptr, acc + 32 * c);
           }
@@ -546,7 +621,7 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t vv[32];
-            tmem_ld32(tmem + lane_base + C::T_ACC + 128 * h + 32 * c, vv);
+            tmem_ld32(tmem + lane_base + t_acc + 128 * h + 32 * c, vv);
             tmem_wait_ld(vv);
             stage_chunk_sw128(vv, mul, tile, r, c);
           }
@@ -569,77 +644,73 @@ __global__ void __launch_bounds__(BwdPairCfg::THREADS, 1)
     // long after the stores have landed.)
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-      const int n_b = SPLIT ? (sent + 1 - b) / 2 : (b == h ? sent : 0);  // uses of buffer b
+      const int n_b = (sent + 1 - b) / 2;  // uses of buffer b
       if (n_b > 0) W.drain_warp(bar(C::B_XE + b), (n_b - 1) & 1);
     }
     tc_fence_before();
   } else if (warp < C::DQ_WARP0 + 4) {
+    // ================================================================ dQ drain
+    // This CTA's dQ^T half (d on TMEM lanes, 64 query columns) -> x scale -> staging blocks
+    // ([32 queries][32 d], two per warp) -> TMA bulk reduce-add into the fp32 accumulator (rows
+    // past N are clipped by the tensor map; quarters wholly past N are skipped).  On CTA 0, once
+    // dQ^T of a step has completed its dS^T tile has been consumed (dK was issued before), so
+    // warp 8 hands it back to CTA 1.
     const int wq = warp - C::DQ_WARP0;
+    const uint32_t lane_base = uint32_t(wq * 32) << 16;
+    const uint32_t t_dq = role == 0 ? C::T_DQ0 : C::T_DQ1;
+    const int d0 = int(role) * 128 + 32 * wq;
     const uint32_t peer_xe0 = mapa_shared(bar(C::B_XE + 0), peer);
     const uint32_t peer_xe1 = mapa_shared(bar(C::B_XE + 1), peer);
-    if (role == 1) {
-      // ============================================================ hand-back (CTA 1)
-      // P^T tile t & 1 is free once dV(t) has completed and the dS warps have read it.
-      if (wq == 0) {
-        for (int it = 0; it < nit; ++it) {
-          if (!W.wait_warp(bar(C::B_XR + (it & 1)), (it >> 1) & 1, 87)) break;
-          if (lane == 0) mbar_arrive_cluster((it & 1) == 0 ? peer_xe0 : peer_xe1);
+    float* wslot = reinterpret_cast<float*>(smem + C::OFF_STG) + wq * 2048;
+    if (lane == 0) tma_prefetch_desc(&tmdQ);
+    int group = 0;
+    BwdCursor cur(grp);
+    for (int it = 0; it < nit; ++it) {
+      const int i = cur.i, head = cur.head;
+      cur.next();
+      if (!W.wait_warp(bar(C::B_DQF), it & 1, 86)) break;
+      FA_TRACE_EV(20, it);
+      if (role == 0 && wq == 0 && lane == 0)
+        mbar_arrive_cluster((it & 1) == 0 ? peer_xe0 : peer_xe1);
+      tc_fence_after();
+      uint32_t v[2][32];
+      tmem_ld32(tmem + lane_base + t_dq, v[0]);
+      tmem_ld32(tmem + lane_base + t_dq + 32, v[1]);
+      tmem_wait_ld(v[0]);
+      tmem_wait_ld(v[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_DQE));
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        const int row0 = i * C::BR + 32 * qq;
+        if (row0 >= p.N) continue;  // uniform over the warp
+        float* slot = wslot + (group & 1) * 1024;
+        if (lane == 0) bulk_wait_group_read<1>();  // the slot's previous reduce has read it
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) slot[c * 32 + lane] = __uint_as_float(v[qq][c]) * p.scale;
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tmdQ, smem_u32(slot), d0, row0, head);
+          bulk_commit_group();
         }
+        ++group;
       }
-    } else {
-      // ============================================================ dQ drain (CTA 0)
-      // dQ^T (d on TMEM lanes, two 64-column halves of 64 queries) -> x scale -> staging
-      // blocks ([32 queries][32 d], two per warp) -> TMA bulk reduce-add into the fp32
-      // accumulator (rows past N are clipped by the tensor map; quarters wholly past N are
-      // skipped).  Once dQ^T of a step has completed, its dS^T tile has been consumed, so warp
-      // 8 hands it back to CTA 1.
-      const uint32_t lane_base = uint32_t(wq * 32) << 16;
-      float* wslot = reinterpret_cast<float*>(smem + C::OFF_STG) + wq * 2048;
-      if (lane == 0) tma_prefetch_desc(&tmdQ);
-      int group = 0;
-      BwdCursor cur(grp);
-      for (int it = 0; it < nit; ++it) {
-        const int i = cur.i, head = cur.head;
-        cur.next();
-        if (!W.wait_warp(bar(C::B_DQF), it & 1, 86)) break;
-        FA_TRACE_EV(20, it);
-        if (wq == 0 && lane == 0) mbar_arrive_cluster((it & 1) == 0 ? peer_xe0 : peer_xe1);
-        tc_fence_after();
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t v[2][32];
-          tmem_ld32(tmem + lane_base + C::T_DQ + 64 * hf, v[0]);
-          tmem_ld32(tmem + lane_base + C::T_DQ + 64 * hf + 32, v[1]);
-          tmem_wait_ld(v[0]);
-          tmem_wait_ld(v[1]);
-          if (hf == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_DQE));
-          }
-#pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            const int row0 = i * C::BR + 32 * qq;
-            if (row0 >= p.N) continue;  // uniform over the warp
-            float* slot = wslot + (group & 1) * 1024;
-            if (lane == 0) bulk_wait_group_read<1>();  // the slot's previous reduce has read it
-            __syncwarp();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) slot[c * 32 + lane] = __uint_as_float(v[qq][c]) * p.scale;
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_reduce_add_3d(&tmdQ, smem_u32(slot), 128 * hf + 32 * wq, row0, head);
-              bulk_commit_group();
-            }
-            ++group;
-          }
-        }
-        FA_TRACE_EV(21, it);
-      }
-      if (lane == 0) bulk_wait_group_all();
+      FA_TRACE_EV(21, it);
     }
+    if (lane == 0) bulk_wait_group_all();
     tc_fence_before();
+  } else if (warp == C::RELAY_WARP && role == 1) {
+    // ================================================================ hand-back (CTA 1)
+    // P^T tile t & 1 is free once dV(t) has completed and the dS warps have read it.
+    const uint32_t peer_xe0 = mapa_shared(bar(C::B_XE + 0), peer);
+    const uint32_t peer_xe1 = mapa_shared(bar(C::B_XE + 1), peer);
+    for (int it = 0; it < nit; ++it) {
+      if (!W.wait_warp(bar(C::B_XR + (it & 1)), (it >> 1) & 1, 87)) break;
+      if (lane == 0) mbar_arrive_cluster((it & 1) == 0 ? peer_xe0 : peer_xe1);
+    }
   }
 
   // neither CTA leaves while the other may still write into its shared memory or arrive on its
