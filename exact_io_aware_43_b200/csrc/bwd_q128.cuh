@@ -114,8 +114,8 @@ struct BwdQ128Cfg {
   static constexpr int OFF_AUG = OFF_STG + STG_BYTES;
   static constexpr int OFF_ONES = OFF_AUG + 2 * AUG_BYTES;
   // barriers: kv, q_full[2], q_empty[2], do_full[2], do_empty[2], s_full, p_full, dp_full,
-  //           ds_full, dv_done, dk_done, dq_full, dq_empty, ds_free, drain
-  static constexpr int NBAR = 19;
+  //           ds_full, dv_done, dk_done, dq_full, dq_empty, ds_free, drain, kv_empty
+  static constexpr int NBAR = 20;
   static constexpr int OFF_BAR = OFF_ONES + 3 * AUG_LBO;
   static constexpr int OFF_MISC = OFF_BAR + 160;
   static constexpr int SMEM_NEED = OFF_MISC + 16;             // from a 1024-aligned base
@@ -134,6 +134,14 @@ struct BwdQ128Cfg {
 __device__ __forceinline__ uint64_t sdesc_interleave(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
          (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// The k-th unit of CTA c among G CTAs: rounds of G units, every other round in reverse CTA order,
+// so that the heaviest units (the first of each band) are spread over the CTAs; -1 when none is
+// left.
+__device__ __forceinline__ int bwdq_unit_of(int k, int c, int G, int units) {
+  const int u = k * G + ((k & 1) ? (G - 1 - c) : c);
+  return u < units ? u : -1;
 }
 
 template <int D, bool CAUSAL>
@@ -162,14 +170,14 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
   FA_TRACE_DECL;
   FA_TRACE_EV(90, 0);  // CTA start
 
-  // ---- work unit: (key block j, key/value head) in the order of BwdUnit; for each query head
-  // of the group (see BwdGroup), query blocks i from j (causal) or 0 to the last
-  const BwdUnit unit(blockIdx.x, p, 1);
-  const int j = unit.j, kvh = unit.kvh;
-  const int k0 = j * C::BC;
+  // ---- work units: (key block j, key/value head [, share of a group's query heads]) in the
+  // order of BwdUnit; for each query head of the group (see BwdGroup), query blocks i from j
+  // (causal) or 0 to the last.  With a grid of G < (unit count) CTAs each CTA takes units in
+  // zig-zag rounds of G (see bwdq_unit_of) and every barrier's phases run on across them (global
+  // step index T); with one CTA per unit the loops below run once.
+  const int units = p.BHkv * p.nkb * p.gsplit;
   const int nqb = (p.N + C::BR - 1) / C::BR;
-  const BwdGroup grp(p, kvh, unit.gs, CAUSAL ? j : 0, nqb);
-  const int nit = grp.nheads * grp.nit_h;  // >= 1
+  const int G = int(gridDim.x), cta = int(blockIdx.x);
 
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
   const uint32_t BAR_KV = bar(0);
@@ -179,7 +187,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
   auto BAR_DOE = [&](int s) { return bar(7 + s); };
   const uint32_t BAR_SF = bar(9), BAR_PF = bar(10), BAR_DPF = bar(11), BAR_DSF = bar(12),
                  BAR_DVD = bar(13), BAR_DKD = bar(14), BAR_DQF = bar(15), BAR_DQE = bar(16),
-                 BAR_DSFREE = bar(17), BAR_DRAIN = bar(18);
+                 BAR_DSFREE = bar(17), BAR_DRAIN = bar(18), BAR_KVE = bar(19);
   constexpr int DS_ = C::DO_STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
@@ -204,6 +212,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
     mbar_init(BAR_DQE, 4);
     mbar_init(BAR_DSFREE, 1);
     mbar_init(BAR_DRAIN, 1);
+    mbar_init(BAR_KVE, 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -235,40 +244,61 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
-      mbar_arrive_expect_tx(BAR_KV, 2 * C::TILE);
-      for (int kb = 0; kb < C::KB; ++kb) {
-        tma_load_3d(sbase + C::OFF_K + kb * C::BLK, &tmK, BAR_KV, kb * 64, k0, kvh);
-        tma_load_3d(sbase + C::OFF_V + kb * C::BLK, &tmV, BAR_KV, kb * 64, k0, kvh);
-      }
-      int tq = 0, td = 0;  // Q / dO tiles issued
-      BwdCursor cur(grp);
-      for (int t = 0; t < nit; ++t) {
-        const int i = cur.i, head = cur.head;
-        cur.next();
-        const int s = t & 1;
-        // Q_i and its row-statistics operand into stage s once dK of step t-2 has released it
-        if (!W.wait(BAR_QE(s), ((t >> 1) & 1) ^ 1, 31)) break;
-        mbar_arrive_expect_tx(BAR_QF(s), C::TILE + C::AUG_BYTES);
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(sbase + C::OFF_Q + s * C::TILE + kb * C::BLK, &tmQ, BAR_QF(s), kb * 64,
-                      i * C::BR, head);
-        const size_t aoff = (size_t(head) * (p.Npad / C::BR) + size_t(i)) * C::AUG_BYTES;
-        bulk_load(sbase + C::OFF_AUG + s * C::AUG_BYTES,
-                  reinterpret_cast<const uint8_t*>(p.aug) + aoff, C::AUG_BYTES, BAR_QF(s));
-        ++tq;
-        FA_TRACE_EV(20, t);
-        // dO_i into its buffer once dP^T and dV of the step that used it last have read it
-        const int sd = t % DS_;
-        if (!W.wait(BAR_DOE(sd), ((t / DS_) & 1) ^ 1, 32)) break;
-        mbar_arrive_expect_tx(BAR_DOF(sd), C::TILE);
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(sbase + C::OFF_DO + sd * C::TILE + kb * C::BLK, &tmdO, BAR_DOF(sd), kb * 64,
-                      i * C::BR, head);
-        ++td;
+      int tq = 0, td = 0, tkv = 0;  // Q, dO, K/V tiles issued
+      bool ok = true;
+      int T = 0;  // global index of the unit's first step
+      for (int kc = 0; ok; ++kc) {
+        const int u = bwdq_unit_of(kc, cta, G, units);
+        if (u < 0) break;
+        const BwdUnit unit(u, p, 1);
+        const int j = unit.j, kvh = unit.kvh, k0 = j * C::BC;
+        const BwdGroup grp(p, kvh, unit.gs, CAUSAL ? j : 0, nqb);
+        const int nit = grp.nheads * grp.nit_h;  // >= 1
+        // Q_i / dO_i of the unit's steps in order; K_j, V_j once every MMA of the previous unit
+        // has completed, issued after the first step's tiles so that these load while the
+        // previous unit finishes
+        auto load_kv = [&]() -> bool {
+          if (!W.wait(BAR_KVE, (kc & 1) ^ 1, 30)) return false;
+          mbar_arrive_expect_tx(BAR_KV, 2 * C::TILE);
+          for (int kb = 0; kb < C::KB; ++kb) {
+            tma_load_3d(sbase + C::OFF_K + kb * C::BLK, &tmK, BAR_KV, kb * 64, k0, kvh);
+            tma_load_3d(sbase + C::OFF_V + kb * C::BLK, &tmV, BAR_KV, kb * 64, k0, kvh);
+          }
+          ++tkv;
+          return true;
+        };
+        BwdCursor cur(grp);
+        for (int tl = 0; tl < nit; ++tl) {
+          const int t = T + tl;
+          const int i = cur.i, head = cur.head;
+          cur.next();
+          const int s = t & 1;
+          // Q_i and its row-statistics operand into stage s once dK of step t-2 has released it
+          if (!(ok = W.wait(BAR_QE(s), ((t >> 1) & 1) ^ 1, 31))) break;
+          mbar_arrive_expect_tx(BAR_QF(s), C::TILE + C::AUG_BYTES);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_3d(sbase + C::OFF_Q + s * C::TILE + kb * C::BLK, &tmQ, BAR_QF(s), kb * 64,
+                        i * C::BR, head);
+          const size_t aoff = (size_t(head) * (p.Npad / C::BR) + size_t(i)) * C::AUG_BYTES;
+          bulk_load(sbase + C::OFF_AUG + s * C::AUG_BYTES,
+                    reinterpret_cast<const uint8_t*>(p.aug) + aoff, C::AUG_BYTES, BAR_QF(s));
+          ++tq;
+          FA_TRACE_EV(20, t);
+          // dO_i into its buffer once dP^T and dV of the step that used it last have read it
+          const int sd = t % DS_;
+          if (!(ok = W.wait(BAR_DOE(sd), ((t / DS_) & 1) ^ 1, 32))) break;
+          mbar_arrive_expect_tx(BAR_DOF(sd), C::TILE);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_3d(sbase + C::OFF_DO + sd * C::TILE + kb * C::BLK, &tmdO, BAR_DOF(sd),
+                        kb * 64, i * C::BR, head);
+          ++td;
+          if (tl == 0 && !(ok = load_kv())) break;
+        }
+        T += nit;
       }
       if (W.aborted()) {
         // let the copies already issued land before the CTA's shared memory goes away
-        W.drain(BAR_KV, 0);
+        if (tkv > 0) W.drain(BAR_KV, (tkv - 1) & 1);
         for (int jj = tq > 2 ? tq - 2 : 0; jj < tq; ++jj) W.drain(BAR_QF(jj & 1), (jj >> 1) & 1);
         for (int jj = td > DS_ ? td - DS_ : 0; jj < td; ++jj)
           W.drain(BAR_DOF(jj % DS_), (jj / DS_) & 1);
@@ -328,72 +358,87 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
         tc_commit(BAR_SF);
         return true;
       };
-      bool ok = W.wait(BAR_KV, 0, 40);
-      FA_TRACE_EV(92, 0);  // K_j, V_j landed
-      if (ok) ok = W.wait(BAR_QF(0), 0, 41);
-      FA_TRACE_EV(93, 0);  // first Q_i landed
-      if (ok) {
+      bool ok = true;
+      int T = 0;  // global index of the unit's first step
+      for (int kc = 0; ok; ++kc) {
+        const int u = bwdq_unit_of(kc, cta, G, units);
+        if (u < 0) break;
+        const BwdUnit unit(u, p, 1);
+        const int j = unit.j;
+        const BwdGroup grp(p, unit.kvh, unit.gs, CAUSAL ? j : 0, nqb);
+        const int nit = grp.nheads * grp.nit_h;  // >= 1
+        (void)j;
+        if (!(ok = W.wait(BAR_KV, kc & 1, 40))) break;
+        FA_TRACE_EV(92, T);  // K_j, V_j landed
+        // the unit's first S^T into R1 once dV of the previous step has read P^T there, its dP^T
+        // into R2 once the previous dQ^T has been drained from it
+        if (T > 0 && !(ok = W.wait(BAR_DVD, (T - 1) & 1, 38))) break;
+        if (T > 0 && !(ok = W.wait(BAR_DQE, (T - 1) & 1, 39))) break;
+        if (!(ok = W.wait(BAR_QF(T & 1), (T >> 1) & 1, 41))) break;
+        FA_TRACE_EV(93, T);  // first Q_i landed
         tc_fence_after();
-        issue_st(C::T_S, k_addr, q_addr(0), ones_s, aug_addr(0));
+        issue_st(C::T_S, k_addr, q_addr(T & 1), ones_s, aug_addr(T));
         tc_commit(BAR_SF);
-        ok = W.wait(BAR_DOF(0), 0, 42);
-      }
-      if (ok) {
+        if (!(ok = W.wait(BAR_DOF(T % DS_), (T / DS_) & 1, 42))) break;
         tc_fence_after();
-        issue_st(C::T_DP, v_addr, do_addr(0), ones_dp, aug_addr(0));
+        issue_st(C::T_DP, v_addr, do_addr(T), ones_dp, aug_addr(T));
         tc_commit(BAR_DPF);
-      }
-      for (int t = 0; ok && t < nit; ++t) {
-        const int s = t & 1;
-        const bool more = t + 1 < nit;
-        // dV += P^T dO_i
-        FA_TRACE_EV(1, t);
-        if (!(ok = W.wait(BAR_PF, t & 1, 43))) break;
-        FA_TRACE_EV(2, t);
-        tc_fence_after();
-        issue_kv(C::T_DV, C::T_S, do_addr(t), t > 0);
-        tc_commit(BAR_DVD);
-        tc_commit(BAR_DOE(t % DS_));
-        if (FA_BWDQ_EARLY_S && more && !(ok = next_s(t))) break;
-        FA_TRACE_EV(4, t);
-        if (!(ok = W.wait(BAR_DSF, t & 1, 46))) break;
-        FA_TRACE_EV(5, t);
-        tc_fence_after();
-        if (FA_BWDQ_DK_SS) {
-          // dQ_i^T = K_j^T dS^T into R2 (the dP^T columns, read by now), then dK += dS^T Q_i;
-          // both take dS^T from the shared tile
-          issue_dq();
-          tc_commit(BAR_DQF);
-          issue_dk_ss(q_addr(s), t > 0);
-          tc_commit(BAR_DKD);
-          tc_commit(BAR_QE(s));
-          FA_TRACE_EV(6, t);
-          if (!FA_BWDQ_EARLY_S && more && !(ok = next_s(t))) break;
-        } else {
-          // dK += dS^T Q_i (dS^T from tensor memory)
-          issue_kv(C::T_DK, C::T_DP, q_addr(s), t > 0);
-          tc_commit(BAR_DKD);
-          tc_commit(BAR_QE(s));
-          if (!FA_BWDQ_EARLY_S && more && !(ok = next_s(t))) break;
-          // dQ_i^T = K_j^T dS^T into R2 once dK has read dS^T
-          if (!(ok = W.wait(BAR_DKD, t & 1, 47))) break;
-          FA_TRACE_EV(6, t);
+        for (int tl = 0; ok && tl < nit; ++tl) {
+          const int t = T + tl;
+          const int s = t & 1;
+          const bool more = tl + 1 < nit;
+          // dV += P^T dO_i
+          FA_TRACE_EV(1, t);
+          if (!(ok = W.wait(BAR_PF, t & 1, 43))) break;
+          FA_TRACE_EV(2, t);
           tc_fence_after();
-          issue_dq();
-          tc_commit(BAR_DQF);
-        }
-        if (more) {
-          // dP^T(t+1) into R2 once dQ^T(t) has been read out (its statistics operand came with
-          // Q_{t+1}, which S^T(t+1) has already waited for)
-          if (!(ok = W.wait(BAR_DQE, t & 1, 48))) break;
-          if (!(ok = W.wait(BAR_DOF((t + 1) % DS_), ((t + 1) / DS_) & 1, 49))) break;
-          if (!FA_BWDQ_EARLY_S && !(ok = W.wait(BAR_QF((t + 1) & 1), ((t + 1) >> 1) & 1, 45)))
-            break;
-          FA_TRACE_EV(7, t);
+          issue_kv(C::T_DV, C::T_S, do_addr(t), tl > 0);
+          tc_commit(BAR_DVD);
+          tc_commit(BAR_DOE(t % DS_));
+          if (FA_BWDQ_EARLY_S && more && !(ok = next_s(t))) break;
+          FA_TRACE_EV(4, t);
+          if (!(ok = W.wait(BAR_DSF, t & 1, 46))) break;
+          FA_TRACE_EV(5, t);
           tc_fence_after();
-          issue_st(C::T_DP, v_addr, do_addr(t + 1), ones_dp, aug_addr(t + 1));
-          tc_commit(BAR_DPF);
+          if (FA_BWDQ_DK_SS) {
+            // dQ_i^T = K_j^T dS^T into R2 (the dP^T columns, read by now), then dK += dS^T Q_i;
+            // both take dS^T from the shared tile
+            issue_dq();
+            tc_commit(BAR_DQF);
+            issue_dk_ss(q_addr(s), tl > 0);
+            tc_commit(BAR_DKD);
+            tc_commit(BAR_QE(s));
+            FA_TRACE_EV(6, t);
+            if (!FA_BWDQ_EARLY_S && more && !(ok = next_s(t))) break;
+          } else {
+            // dK += dS^T Q_i (dS^T from tensor memory)
+            issue_kv(C::T_DK, C::T_DP, q_addr(s), tl > 0);
+            tc_commit(BAR_DKD);
+            tc_commit(BAR_QE(s));
+            if (!FA_BWDQ_EARLY_S && more && !(ok = next_s(t))) break;
+            // dQ_i^T = K_j^T dS^T into R2 once dK has read dS^T
+            if (!(ok = W.wait(BAR_DKD, t & 1, 47))) break;
+            FA_TRACE_EV(6, t);
+            tc_fence_after();
+            issue_dq();
+            tc_commit(BAR_DQF);
+          }
+          if (more) {
+            // dP^T(t+1) into R2 once dQ^T(t) has been read out (its statistics operand came with
+            // Q_{t+1}, which S^T(t+1) has already waited for)
+            if (!(ok = W.wait(BAR_DQE, t & 1, 48))) break;
+            if (!(ok = W.wait(BAR_DOF((t + 1) % DS_), ((t + 1) / DS_) & 1, 49))) break;
+            if (!FA_BWDQ_EARLY_S && !(ok = W.wait(BAR_QF((t + 1) & 1), ((t + 1) >> 1) & 1, 45)))
+              break;
+            FA_TRACE_EV(7, t);
+            tc_fence_after();
+            issue_st(C::T_DP, v_addr, do_addr(t + 1), ones_dp, aug_addr(t + 1));
+            tc_commit(BAR_DPF);
+          }
         }
+        // K_j, V_j are read by nothing once this unit's MMAs have completed
+        tc_commit(BAR_KVE);
+        T += nit;
       }
       // every MMA issued above has completed before the tensor memory is released
       tc_commit(BAR_DRAIN);
@@ -405,13 +450,22 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
     const int h = warp >> 2;                // query half
     const int c0 = 64 * h;                  // first query column of this thread
     const int r = (warp & 3) * 32 + lane;   // key row within the block == TMEM lane
-    const int key = k0 + r;
-    const bool key_ok = key < p.N;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     uint8_t* ds_row = smem + C::OFF_DS + h * C::BLK + r * 128;
     bool ok = true;
+    int T = 0;  // global index of the unit's first step
+    for (int kc = 0; ok; ++kc) {
+    const int u = bwdq_unit_of(kc, cta, G, units);
+    if (u < 0) break;
+    const BwdUnit unit(u, p, 1);
+    const int j = unit.j, kvh = unit.kvh, k0 = j * C::BC;
+    const BwdGroup grp(p, kvh, unit.gs, CAUSAL ? j : 0, nqb);
+    const int nit = grp.nheads * grp.nit_h;  // >= 1
+    const int key = k0 + r;
+    const bool key_ok = key < p.N;
     BwdCursor cur(grp);
-    for (int t = 0; t < nit; ++t) {
+    for (int tl = 0; tl < nit; ++tl) {
+      const int t = T + tl;
       const int i = cur.i;
       cur.next();
       if (!(ok = W.wait_warp(BAR_SF, t & 1, 50))) break;
@@ -505,12 +559,14 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
     }
     if (ok) {
       // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale), bf16
-      ok = W.wait_warp(BAR_DKD, (nit - 1) & 1, 55);
+      ok = W.wait_warp(BAR_DKD, (T + nit - 1) & 1, 55);
       FA_TRACE_EV(94, 0);  // epilogue start
       if (ok) {
         tc_fence_after();
         const uint32_t col = h == 0 ? C::T_DV : C::T_DK;
         const float mul = h == 0 ? 1.f : p.scale;
+        const CUtensorMap* tmo = h == 0 ? &tmdV : &tmdK;
+        const bool issuer = (warp & 3) == 0 && lane == 0;
         if (p.gsplit > 1) {
           // a group's query heads split over CTAs: fp32 reduce-adds into the accumulators
           const size_t base = (size_t(kvh) * p.N + key) * C::D;
@@ -522,9 +578,10 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
             tmem_wait_ld(v);
             bwd_store_chunk(v, mul, key_ok, nullptr, acc + 32 * c);
           }
-        } else {
-          // staged as a swizzled tile in Q stage h (no longer read: every MMA has completed),
-          // then written by TMA tensor stores in whole rows (rows past N are clipped)
+        } else if (bwdq_unit_of(kc + 1, cta, G, units) < 0) {
+          // the CTA's last unit: staged as a swizzled tile in Q stage h (no longer read: every
+          // MMA has completed and nothing is loaded after it), then written by TMA tensor stores
+          // in whole rows (rows past N are clipped)
           uint8_t* tile = smem + C::OFF_Q + h * C::TILE;
 #pragma unroll
           for (int c = 0; c < C::D / 32; ++c) {
@@ -535,17 +592,41 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
           }
           fence_async_smem();
           named_bar_sync(1 + h, 128);
-          if ((warp & 3) == 0 && lane == 0) {
+          if (issuer) {
 #pragma unroll
             for (int kb = 0; kb < C::KB; ++kb)
-              tma_store_3d(h == 0 ? &tmdV : &tmdK, sbase + C::OFF_Q + h * C::TILE + kb * C::BLK,
-                           kb * 64, k0, kvh);
+              tma_store_3d(tmo, sbase + C::OFF_Q + h * C::TILE + kb * C::BLK, kb * 64, k0, kvh);
             bulk_commit_group();
             bulk_wait_group_read<0>();  // the tile is read before the CTA's memory goes away
+          }
+        } else {
+          // another unit follows (the Q stages already hold its tiles): staged one 64-column
+          // block at a time in this warpgroup's half of the dS^T tile, free until this
+          // warpgroup writes the next unit's dS^T
+          uint8_t* blk = smem + C::OFF_DS + h * C::BLK;
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb) {
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+              uint32_t v[32];
+              tmem_ld32(tmem + lane_base + col + 32 * (2 * kb + c2), v);
+              tmem_wait_ld(v);
+              stage_chunk_sw128(v, mul, blk, r, c2);
+            }
+            fence_async_smem();
+            named_bar_sync(1 + h, 128);
+            if (issuer) {
+              tma_store_3d(tmo, sbase + C::OFF_DS + h * C::BLK, kb * 64, k0, kvh);
+              bulk_commit_group();
+              bulk_wait_group_read<0>();  // read before the block is written again
+            }
+            named_bar_sync(1 + h, 128);
           }
         }
       }
     }
+    T += nit;
+    }  // units
     tc_fence_before();
   } else {
     // ================================================================ dQ drain warpgroup
@@ -562,11 +643,20 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     float* wslot = reinterpret_cast<float*>(smem + C::OFF_STG) + wq * (32 * C::DW);
     if (issuer) tma_prefetch_desc(&tmdQ);
+    bool ok = true;
+    int T = 0;  // global index of the unit's first step
+    for (int kc = 0; ok; ++kc) {
+    const int u = bwdq_unit_of(kc, cta, G, units);
+    if (u < 0) break;
+    const BwdUnit unit(u, p, 1);
+    const BwdGroup grp(p, unit.kvh, unit.gs, CAUSAL ? unit.j : 0, nqb);
+    const int nit = grp.nheads * grp.nit_h;  // >= 1
     BwdCursor cur(grp);
-    for (int t = 0; t < nit; ++t) {
+    for (int tl = 0; tl < nit; ++tl) {
+      const int t = T + tl;
       const int i = cur.i, head = cur.head;
       cur.next();
-      if (!(W.wait_warp(BAR_DQF, t & 1, 60))) break;
+      if (!(ok = W.wait_warp(BAR_DQF, t & 1, 60))) break;
       FA_TRACE_EV(60, t);
       tc_fence_after();
       uint32_t v[4][32];
@@ -598,6 +688,8 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
         }
       }
     }
+    T += nit;
+    }  // units
     if (issuer) bulk_wait_group_all();
     tc_fence_before();
   }

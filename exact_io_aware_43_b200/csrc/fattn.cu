@@ -300,6 +300,14 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 #ifndef FA_BWD_Q128
 #define FA_BWD_Q128 1
 #endif
+// 128-query backward: 0 launches one CTA per unit (key block, K/V head [, share of a group]);
+// 1 launches one CTA per SM that loops over the units; 2 (default) picks the persistent grid
+// when units are short (at most kBwdqPersistSteps query-block steps each), where a CTA's set-up,
+// K/V load and dK/dV epilogue are a large part of a unit, and one CTA per unit otherwise.
+#ifndef FA_BWDQ_PERSIST
+#define FA_BWDQ_PERSIST 2
+#endif
+constexpr int kBwdqPersistSteps = 16;
 // d = 256 backward: CTA pairs exchanging P and dS through distributed shared memory
 // (fa_bwd_kernel_pair); 0 selects the kernel whose two CTAs per key block each recompute S^T, dP^T.
 #ifndef FA_BWD_PAIR
@@ -351,7 +359,12 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
     CUtensorMap mdk, mdv;
     if ((rc = make_map(&mdk, p.dk, p.BHkv, p.N, D, CQ::BC))) return rc;
     if ((rc = make_map(&mdv, p.dv, p.BHkv, p.N, D, CQ::BC))) return rc;
-    dim3 grid(unsigned(p.BHkv) * unsigned(p.nkb) * unsigned(p.gsplit));
+    // one CTA per unit, or (FA_BWDQ_PERSIST) one per SM looping over the units
+    const int units = p.BHkv * p.nkb * p.gsplit;
+    const int steps_max = p.gq * ((p.N + CQ::BR - 1) / CQ::BR);  // longest unit (non-causal)
+    const bool persist =
+        FA_BWDQ_PERSIST == 1 || (FA_BWDQ_PERSIST == 2 && steps_max <= kBwdqPersistSteps);
+    dim3 grid(unsigned(persist && units > sm_count() ? sm_count() : units));
     {
       TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
       kq<<<grid, CQ::THREADS, CQ::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p);
