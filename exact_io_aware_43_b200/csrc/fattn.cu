@@ -217,6 +217,11 @@ int sm_count() {
   return n;
 }
 
+// FA_FWD_TAIL_SPLIT: 1 cuts the units of a short last round in two (plain non-causal forward).
+#ifndef FA_FWD_TAIL_SPLIT
+#define FA_FWD_TAIL_SPLIT 1
+#endif
+
 template <int D, bool CAUSAL, int NQT>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mo, fattn::FwdParams p, int BH, cudaStream_t st) {
@@ -251,6 +256,18 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   } else {
     p.nqb = (p.Nq + NQT * C::BM - 1) / (NQT * C::BM);
     p.units = BH * p.nqb * p.splits;
+  }
+  p.tail_base = p.units;
+  if (FA_FWD_TAIL_SPLIT && !CAUSAL && !general && NQT == 2 && p.units > sm_count()) {
+    // the last round of the persistent grid holds `last` units: when that is at most half a
+    // round, cut each in two one-tile work items, so the round takes about half as long
+    const int g = sm_count();
+    const int rounds = (p.units + g - 1) / g;
+    const int last = p.units - (rounds - 1) * g;
+    if (2 * last <= g) {
+      p.tail_base = (rounds - 1) * g;
+      p.units = p.tail_base + 2 * last;
+    }
   }
   // persistent: one CTA per SM (at most one unit each when there are fewer units than SMs)
   const int G = FA_FWD_PERSISTENT ? (p.units < sm_count() ? p.units : sm_count()) : p.units;

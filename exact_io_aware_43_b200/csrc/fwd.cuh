@@ -74,7 +74,10 @@ struct FwdParams {
                      // (rows g * Nq + i; needs G * Nq <= 128), one unit per (K/V head, range)
   int Hkv;           // key/value heads per batch
   int kv_chunk;      // KV tiles of 128 keys per split
-  int units;         // BH * nqb * splits
+  int units;         // BH * nqb * splits, or more with a split tail (below)
+  int tail_base;     // work items from here on are single query tiles: the units of the last
+                     // (partial) round, each cut in two so that the round is shorter (plain
+                     // non-causal forward with two query tiles); = units when not used
   float scale_log2;  // scale * log2(e)
   uint64_t limit_ns;
 };
@@ -175,6 +178,13 @@ struct FwdUnit {
       J = nkv[0];
       return;
     }
+    // a split tail: work item u >= tail_base is query tile (u - tail_base) & 1 of unit
+    // tail_base + (u - tail_base) / 2, run as a one-tile unit
+    int half = -1;
+    if (!CAUSAL && !GENERAL && NQT == 2 && u >= p.tail_base) {
+      half = (u - p.tail_base) & 1;
+      u = p.tail_base + ((u - p.tail_base) >> 1);
+    }
     const int per_qb = p.BH * p.splits;
     const int qi = u / per_qb;
     const int rem = u - qi * per_qb;
@@ -197,6 +207,14 @@ struct FwdUnit {
       }
       nkv[t] = n;
       J = max(J, n);
+    }
+    if (half >= 0) {
+      // tile `half` of the unit, moved into tile slot 0; slot 1 stays empty
+      q0 += half * 128;
+      nkv[0] = nkv[half];
+#pragma unroll
+      for (int t = 1; t < NQT; ++t) nkv[t] = 0;
+      J = nkv[0];
     }
   }
 };

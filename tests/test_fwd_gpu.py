@@ -82,3 +82,12 @@ def test_deterministic():
     o2, l2 = fa.forward(dev["q"], dev["k"], dev["v"], True)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_split_tail_noncausal(d):
+    """B=7 H=8 N=700 non-causal: 168 units of two query tiles on 148 SMs; the 20 units of the
+    short last round run as 40 one-tile items, the last query block (rows 512..699) among them,
+    its second tile ragged."""
+    o, lse, O, L = run_fwd(7, 8, 700, d, False, seed=11)
+    assert_fwd(o, O, lse, L, f"split tail d={d}")
