@@ -45,6 +45,12 @@
 #ifndef FA_BWDQ_DK_SS
 #define FA_BWDQ_DK_SS 1
 #endif
+// FA_BWDQ_INORDER: 1 issues S^T(i+1) into R1 right behind dV(i), which reads P^T(i) there,
+// without waiting for dV(i) to complete: the MMAs of one issuing thread run through the tensor
+// core in issue order, so dV(i) has read its operand before S^T(i+1) writes.
+#ifndef FA_BWDQ_INORDER
+#define FA_BWDQ_INORDER 1
+#endif
 
 // FA_BWDQ_PIPE_LD: 1 loads the second 32 columns of S^T / dP^T while the first 32 are worked on
 // (one tcgen05.wait::ld covers all of a thread's loads, so the second load is issued after the
@@ -350,7 +356,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
                  sdesc_sw128(ds_addr + kk * 2048, C::BLK, 1024), C::IDESC_DQ, kk > 0 ? 1u : 0u);
       };
       auto next_s = [&](int t) -> bool {  // S^T(t+1) into R1 once dV(t) has read P^T(t)
-        if (!W.wait(BAR_DVD, t & 1, 44)) return false;
+        if (!FA_BWDQ_INORDER && !W.wait(BAR_DVD, t & 1, 44)) return false;
         if (!W.wait(BAR_QF((t + 1) & 1), ((t + 1) >> 1) & 1, 45)) return false;
         FA_TRACE_EV(3, t);
         tc_fence_after();
@@ -372,7 +378,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
         FA_TRACE_EV(92, T);  // K_j, V_j landed
         // the unit's first S^T into R1 once dV of the previous step has read P^T there, its dP^T
         // into R2 once the previous dQ^T has been drained from it
-        if (T > 0 && !(ok = W.wait(BAR_DVD, (T - 1) & 1, 38))) break;
+        if (!FA_BWDQ_INORDER && T > 0 && !(ok = W.wait(BAR_DVD, (T - 1) & 1, 38))) break;
         if (T > 0 && !(ok = W.wait(BAR_DQE, (T - 1) & 1, 39))) break;
         if (!(ok = W.wait(BAR_QF(T & 1), (T >> 1) & 1, 41))) break;
         FA_TRACE_EV(93, T);  // first Q_i landed
@@ -393,7 +399,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
           FA_TRACE_EV(2, t);
           tc_fence_after();
           issue_kv(C::T_DV, C::T_S, do_addr(t), tl > 0);
-          tc_commit(BAR_DVD);
+          if (!FA_BWDQ_INORDER) tc_commit(BAR_DVD);
           tc_commit(BAR_DOE(t % DS_));
           if (FA_BWDQ_EARLY_S && more && !(ok = next_s(t))) break;
           FA_TRACE_EV(4, t);

@@ -303,6 +303,7 @@ int launch_fwd_fp8(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   p.BH = BH;
   p.nqb = (p.Nq + NQT * C::BM - 1) / (NQT * C::BM);
   p.units = BH * p.nqb;
+  p.tail_base = p.units;  // no split tail: every unit keeps its two query tiles
   const int G = p.units < sm_count() ? p.units : sm_count();
   TimedLaunch tl(FA_KERNEL_FWD, st);
   kern<<<dim3(unsigned(G)), C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, p, v_scale);

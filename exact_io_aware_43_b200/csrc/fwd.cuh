@@ -54,6 +54,23 @@
 #ifndef FA_FWD_ONES_SUM
 #define FA_FWD_ONES_SUM 1
 #endif
+// FA_FWD_VST: V ring depth at d = 128 with two query tiles (the K ring keeps 2 stages).
+#ifndef FA_FWD_VST
+#define FA_FWD_VST 2
+#endif
+// FA_FWD_MMA_POLL: the two-tile MMA warp waits on its barriers with plain try_wait polling
+// instead of try_wait with a suspend hint (-1: at d = 128 only).
+#ifndef FA_FWD_MMA_POLL
+#define FA_FWD_MMA_POLL -1
+#endif
+// FA_FWD_INORDER: 1 issues S_t(j+1) right behind PV_t(j) without waiting for PV_t(j) to
+// complete.  S_t(j+1) overwrites the tensor memory that PV_t(j) reads P_t(j) from; the MMAs of
+// one issuing thread run through the tensor core in issue order, so PV_t(j) has read its
+// operands before S_t(j+1) writes (the same reliance as the sm100 attention collectives of
+// CUTLASS, which issue Q K^T of the next tile straight after P V of the previous one).
+#ifndef FA_FWD_INORDER
+#define FA_FWD_INORDER 1
+#endif
 
 namespace fattn {
 
@@ -93,6 +110,8 @@ struct FwdCfg {
   // a second tile would stay empty) the freed query buffer holds more stages.
   static constexpr int STAGES = NQT == 1 ? (D == 64 ? 6 : (D == 128 ? 3 : 1))
                                          : (D == 64 ? 4 : (D == 128 ? 2 : 1));
+  static constexpr int KST = STAGES;                                        // K ring
+  static constexpr int VST = (NQT == 2 && D == 128) ? FA_FWD_VST : STAGES;  // V ring
   static constexpr int SOFTMAX_WARPS = 4 * NQT;
   static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;  // control warpgroup: producer, MMA, 2 idle
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
@@ -124,8 +143,8 @@ struct FwdCfg {
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQT * QTILE_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KVTILE_BYTES;
-  static constexpr int OFF_ONES = OFF_V + STAGES * KVTILE_BYTES;  // [BN keys][64] bf16 ones
+  static constexpr int OFF_V = OFF_K + KST * KVTILE_BYTES;
+  static constexpr int OFF_ONES = OFF_V + VST * KVTILE_BYTES;  // [BN keys][64] bf16 ones
   // O written by TMA tensor stores from swizzled shared blocks of [128 rows][64 columns] (16 KB):
   // one per query tile at d = 64 (two tiles), two alternating at d = 256.  d = 128 stores its
   // rows directly: there the staging's warpgroup barriers cost more than the stores save (long
@@ -135,10 +154,10 @@ struct FwdCfg {
   static constexpr int STG_BLK = BM * 128;
   static constexpr int OFF_STG = OFF_ONES + (EXTRA ? BN * 128 : 0);
   static constexpr int OFF_BAR = OFF_STG + (TMA_EPI ? 2 * STG_BLK : 0);
-  // barriers: q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NB],
-  //           p_full[NB], o_done[NB], o_free[NQT], drain (slot = query tile, or with one query
-  //           tile the S buffer)
-  static constexpr int NBAR = 2 + 4 * STAGES + 3 * NB + NQT + 1;
+  // barriers: q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST],
+  //           s_full[NB], p_full[NB], o_done[NB], o_free[NQT], drain (slot = query tile, or
+  //           with one query tile the S buffer)
+  static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 3 * NB + NQT + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem address + abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);   // Q, K both K-major
@@ -243,27 +262,30 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
   const uint32_t BAR_Q = bar(0);
   const uint32_t BAR_QE = bar(1);
   auto BAR_KF = [&](int s) { return bar(2 + s); };
-  auto BAR_KE = [&](int s) { return bar(2 + C::STAGES + s); };
-  auto BAR_VF = [&](int s) { return bar(2 + 2 * C::STAGES + s); };
-  auto BAR_VE = [&](int s) { return bar(2 + 3 * C::STAGES + s); };
-  auto BAR_SF = [&](int b) { return bar(2 + 4 * C::STAGES + b); };
-  auto BAR_PF = [&](int b) { return bar(2 + 4 * C::STAGES + C::NB + b); };
-  auto BAR_OD = [&](int b) { return bar(2 + 4 * C::STAGES + 2 * C::NB + b); };
-  auto BAR_OF = [&](int t) { return bar(2 + 4 * C::STAGES + 3 * C::NB + t); };
+  constexpr int KV_BARS = 2 * C::KST + 2 * C::VST;
+  auto BAR_KE = [&](int s) { return bar(2 + C::KST + s); };
+  auto BAR_VF = [&](int s) { return bar(2 + 2 * C::KST + s); };
+  auto BAR_VE = [&](int s) { return bar(2 + 2 * C::KST + C::VST + s); };
+  auto BAR_SF = [&](int b) { return bar(2 + KV_BARS + b); };
+  auto BAR_PF = [&](int b) { return bar(2 + KV_BARS + C::NB + b); };
+  auto BAR_OD = [&](int b) { return bar(2 + KV_BARS + 2 * C::NB + b); };
+  auto BAR_OF = [&](int t) { return bar(2 + KV_BARS + 3 * C::NB + t); };
   // With the double score buffer (one query tile), key tile g (counted over the CTA's whole run)
   // uses S buffer / barrier slot g & 1, and is the (g >> 1)-th use of that slot.
   auto sbuf_col = [&](int g) -> uint32_t { return (g & 1) ? C::TMEM_S1 : C::TMEM_S; };
   const uint32_t BAR_DRAIN = bar(C::NBAR - 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
-  const Waiter W{abort_flag, p.limit_ns};
+  Waiter W{abort_flag, p.limit_ns};
 
   if (threadIdx.x == 0) {
     mbar_init(BAR_Q, 1);
     mbar_init(BAR_QE, 1);
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < C::KST; ++s) {
       mbar_init(BAR_KF(s), 1);
       mbar_init(BAR_KE(s), 1);
+    }
+    for (int s = 0; s < C::VST; ++s) {
       mbar_init(BAR_VF(s), 1);
       mbar_init(BAR_VE(s), 1);
     }
@@ -305,9 +327,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
         int kv_it = 0;   // KV tiles loaded so far (ring position)
         int kq = 0;      // units with work so far (the Q barriers' phase)
         int q_n = 0;     // Q loads issued, and K / V loads issued per ring stage: each issued load
-        int k_n[C::STAGES], v_n[C::STAGES];  // is one phase of its full barrier (drain below)
+        int k_n[C::KST], v_n[C::VST];  // is one phase of its full barrier (drain below)
 #pragma unroll
-        for (int s = 0; s < C::STAGES; ++s) k_n[s] = v_n[s] = 0;
+        for (int s = 0; s < C::KST; ++s) k_n[s] = 0;
+#pragma unroll
+        for (int s = 0; s < C::VST; ++s) v_n[s] = 0;
         bool ok = true;
         for (int k = 0;; ++k) {
           const int u = fwd_unit_of(k, cta, G, p.units);
@@ -336,8 +360,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           }
           for (int j = 0; j < un.J; ++j) {
             const int g = kv_it + j;
-            const int s = g % C::STAGES;
-            const uint32_t ph = (g / C::STAGES) & 1;
+            const int s = g % C::KST;
+            const uint32_t ph = (g / C::KST) & 1;
+            const int sv = g % C::VST;
+            const uint32_t phv = (g / C::VST) & 1;
 #ifdef FA_TEST_STARVE
             // Test build only (libfattn_starve.so): CTA 0 never issues the second K/V tile of its
             // first unit, so the MMA warp's bounded wait for it runs out and the kernel must
@@ -355,13 +381,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
               tma_load_3d(sbase + C::OFF_K + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmK,
                           BAR_KF(s), kb * 64, (un.kt0 + j) * C::BN, un.kv_head);
             ++k_n[s];
-            if (!(ok = W.wait(BAR_VE(s), ph ^ 1, 2))) break;
+            if (!(ok = W.wait(BAR_VE(sv), phv ^ 1, 2))) break;
             FA_TRACE_EV(21, j);
-            mbar_arrive_expect_tx(BAR_VF(s), C::KVTILE_BYTES);
+            mbar_arrive_expect_tx(BAR_VF(sv), C::KVTILE_BYTES);
             for (int kb = 0; kb < C::KB; ++kb)
-              tma_load_3d(sbase + C::OFF_V + s * C::KVTILE_BYTES + kb * (C::BN * 128), &tmV,
-                          BAR_VF(s), kb * 64, (un.kt0 + j) * C::BN, un.kv_head);
-            ++v_n[s];
+              tma_load_3d(sbase + C::OFF_V + sv * C::KVTILE_BYTES + kb * (C::BN * 128), &tmV,
+                          BAR_VF(sv), kb * 64, (un.kt0 + j) * C::BN, un.kv_head);
+            ++v_n[sv];
           }
           if (!ok) break;
           kv_it += un.J;
@@ -374,10 +400,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           // enough; a barrier with no load issued is skipped.
           if (q_n > 0) W.drain(BAR_Q, (q_n - 1) & 1);
 #pragma unroll
-          for (int s = 0; s < C::STAGES; ++s) {
+          for (int s = 0; s < C::KST; ++s)
             if (k_n[s] > 0) W.drain(BAR_KF(s), (k_n[s] - 1) & 1);
+#pragma unroll
+          for (int s = 0; s < C::VST; ++s)
             if (v_n[s] > 0) W.drain(BAR_VF(s), (v_n[s] - 1) & 1);
-          }
         }
       }
     } else if (warp == C::MMA_WARP && C::DBUF) {
@@ -398,8 +425,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           tc_commit(BAR_SF(g & 1));
         };
         // S buffer g & 1 is free once PV(g - 2) has completed (it read the P held there)
+        // (with FA_FWD_INORDER, S(g) simply follows PV(g - 2) in issue order; packed decoding
+        // keeps the wait, measured 1% faster there)
+        const bool inorder = FA_FWD_INORDER && !(SPLIT && p.pack > 1);
         auto sbuf_free = [&](int g, int site) -> bool {
-          return g < 2 || W.wait(BAR_OD(g & 1), ((g - 2) >> 1) & 1, site);
+          return inorder || g < 2 || W.wait(BAR_OD(g & 1), ((g - 2) >> 1) & 1, site);
         };
         int g = 0, kv_it = 0, kq = 0, nun = 0;
         bool ok = true;
@@ -409,9 +439,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           const Unit un(u, p);
           const int J = un.J;
           if (J == 0) continue;
-          const int s0 = kv_it % C::STAGES;
+          const int s0 = kv_it % C::KST;
           if (!(ok = W.wait(BAR_Q, kq & 1, 10))) break;
-          if (!(ok = W.wait(BAR_KF(s0), (kv_it / C::STAGES) & 1, 11))) break;
+          if (!(ok = W.wait(BAR_KF(s0), (kv_it / C::KST) & 1, 11))) break;
           if (!(ok = sbuf_free(g, 12))) break;
           tc_fence_after();
           issue_s(g, sbase + C::OFF_K + s0 * C::KVTILE_BYTES);
@@ -419,19 +449,20 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           if (J == 1) tc_commit(BAR_QE);
           for (int j = 0; ok && j < J; ++j) {
             const int gg = g + j;
-            const int s = (kv_it + j) % C::STAGES;
-            const int s1 = (kv_it + j + 1) % C::STAGES;
-            const uint32_t kph1 = ((kv_it + j + 1) / C::STAGES) & 1;
+            const int s = (kv_it + j) % C::VST;  // V stage of key tile j
+            const int s1 = (kv_it + j + 1) % C::KST;
+            const uint32_t kph1 = ((kv_it + j + 1) / C::KST) & 1;
             bool s_next = j + 1 < J;
             if (s_next && mbar_test_wait(BAR_KF(s1), kph1) &&
-                (gg + 1 < 2 || mbar_test_wait(BAR_OD((gg + 1) & 1), ((gg - 1) >> 1) & 1))) {
+                (inorder || gg + 1 < 2 ||
+                 mbar_test_wait(BAR_OD((gg + 1) & 1), ((gg - 1) >> 1) & 1))) {
               tc_fence_after();
               issue_s(gg + 1, sbase + C::OFF_K + s1 * C::KVTILE_BYTES);
               tc_commit(BAR_KE(s1));
               if (j + 2 == J) tc_commit(BAR_QE);  // every S of this unit is issued
               s_next = false;
             }
-            if (!(ok = W.wait(BAR_VF(s), ((kv_it + j) / C::STAGES) & 1, 13))) break;
+            if (!(ok = W.wait(BAR_VF(s), ((kv_it + j) / C::VST) & 1, 13))) break;
             if (!(ok = W.wait(BAR_PF(gg & 1), (gg >> 1) & 1, 14))) break;
             // the first PV of a unit overwrites O: the previous epilogue must have read it
             if (j == 0 && nun > 0 && !(ok = W.wait(BAR_OF(0), (nun - 1) & 1, 15))) break;
@@ -468,9 +499,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
       }
     } else if (warp == C::MMA_WARP) {
       // -------------------------------------------------------------- MMA issuer
+      W.sleep = !(FA_FWD_MMA_POLL == 1 || (FA_FWD_MMA_POLL < 0 && D == 128));
       // Order per KV tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  S_t(j+1) overwrites the
-      // tensor memory that holds P_t(j), so it waits for PV_t(j) to complete; issuing it right
-      // behind PV_t(j) lets softmax t start on tile j+1 while the other query tile's PV runs.
+      // tensor memory that holds P_t(j); it follows PV_t(j) in issue order (FA_FWD_INORDER, else
+      // it waits for PV_t(j) to complete), so softmax t starts on tile j+1 while the other query
+      // tile's PV runs.
       if (lane == 0) {
         auto issue_s = [&](int t, uint32_t k_addr) {
           const uint32_t q_addr = sbase + C::OFF_Q + t * C::QTILE_BYTES;
@@ -494,13 +527,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           const Unit un(u, p);
           const int J = un.J;
           if (J == 0) continue;  // skipped by the producer too
-          const int s0 = kv_it % C::STAGES;
+          const int s0 = kv_it % C::KST;
           if (!(ok = W.wait(BAR_Q, kq & 1, 10))) break;
-          if (!(ok = W.wait(BAR_KF(s0), (kv_it / C::STAGES) & 1, 11))) break;
+          if (!(ok = W.wait(BAR_KF(s0), (kv_it / C::KST) & 1, 11))) break;
           for (int t = 0; t < NQT && ok; ++t) {
             if (un.nkv[t] == 0) continue;
             // S_t's columns hold P_t of the previous unit's last tile until its PV completed
-            if (tit[t] > 0 && !(ok = W.wait(BAR_OD(t), (tit[t] - 1) & 1, 12))) break;
+            if (!FA_FWD_INORDER && tit[t] > 0 && !(ok = W.wait(BAR_OD(t), (tit[t] - 1) & 1, 12)))
+              break;
             tc_fence_after();
             issue_s(t, sbase + C::OFF_K + s0 * C::KVTILE_BYTES);
           }
@@ -509,11 +543,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
           if (J == 1) tc_commit(BAR_QE);  // every S of this unit is issued: Q may be replaced
           for (int j = 0; ok && j < J; ++j) {
             const int g = kv_it + j;
-            const int s = g % C::STAGES;
-            const int s1 = (g + 1) % C::STAGES;
+            const int s = g % C::VST;         // V stage of key tile j
+            const int s1 = (g + 1) % C::KST;  // K stage of key tile j + 1
             const uint32_t v_addr = sbase + C::OFF_V + s * C::KVTILE_BYTES;
             const uint32_t k1_addr = sbase + C::OFF_K + s1 * C::KVTILE_BYTES;
-            if (!(ok = W.wait(BAR_VF(s), (g / C::STAGES) & 1, 13))) break;
+            FA_TRACE_EV(8, j);
+            if (!(ok = W.wait(BAR_VF(s), (g / C::VST) & 1, 13))) break;
+            FA_TRACE_EV(9, j);
             bool k_ready = false;
             for (int t = 0; t < NQT && ok; ++t) {
               if (j >= un.nkv[t]) continue;
@@ -537,15 +573,18 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
                        (j > 0 || kk > 0) ? 1u : 0u);
               }
               tc_commit(BAR_OD(t));
+              FA_TRACE_EV(4 + 16 * t, j);
               if (j + 1 < un.nkv[t]) {
                 if (!k_ready &&
-                    !(ok = W.wait(BAR_KF(s1), ((g + 1) / C::STAGES) & 1, 16)))
+                    !(ok = W.wait(BAR_KF(s1), ((g + 1) / C::KST) & 1, 16)))
                   break;
                 k_ready = true;
-                if (!(ok = W.wait(BAR_OD(t), tit[t] & 1, 17))) break;  // P_t(j) consumed
+                if (!FA_FWD_INORDER && !(ok = W.wait(BAR_OD(t), tit[t] & 1, 17)))
+                  break;  // P_t(j) consumed
                 FA_TRACE_EV(3 + 16 * t, j);
                 tc_fence_after();
                 issue_s(t, k1_addr);
+                FA_TRACE_EV(5 + 16 * t, j);
               }
               ++tit[t];
             }
