@@ -38,9 +38,10 @@
 #define FA_FWD_RSUM 2
 #endif
 // FA_FWD_POLY_MASK: bit g set computes the exponentials of scores [4g, 4g+4) of every 32 on the
-// FMA pipe (exp2_fma2) instead of the MUFU unit.
+// FMA pipe (exp2_fma2) instead of the MUFU unit; -1: a quarter (groups 0 and 4) at d = 64, where
+// an exponential comes with half the MMA work of d = 128 and MUFU binds, none otherwise.
 #ifndef FA_FWD_POLY_MASK
-#define FA_FWD_POLY_MASK 0x00
+#define FA_FWD_POLY_MASK -1
 #endif
 #ifndef FA_FWD_RESCALE
 #define FA_FWD_RESCALE 8.0f
@@ -832,7 +833,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT>::THREADS, 1)
             f2unpack(ffma2(f2pack(__uint_as_float(s[c][2 * e]), __uint_as_float(s[c][2 * e + 1])),
                            sc2, nm2),
                      x0, x1);
-            if ((FA_FWD_POLY_MASK >> (e >> 1)) & 1) {
+            constexpr int kPoly =
+                FA_FWD_POLY_MASK >= 0 ? FA_FWD_POLY_MASK : (D == 64 ? 0x11 : 0x00);
+            if ((kPoly >> (e >> 1)) & 1) {
               exp2_fma2(x0, x1, p0, p1);
             } else {
               p0 = ex2(x0);
