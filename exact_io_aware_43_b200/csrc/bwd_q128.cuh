@@ -21,8 +21,10 @@
 // dS^T = P^T (dP^T - D) need no per-query value from shared memory (the broadcast loads of L and
 // D cost as many shared-memory wavefronts as the MMA operands of a GEMM).
 // dS^T (bf16) goes to a shared tile, from which both dQ^T and dK (dS^T Q_i, both operands in
-// shared memory) read it.  Reuse is ordered by completion barriers, never by issue order:
-// S^T(i+1) is issued once dV(i) has completed, dP^T(i+1) once dQ^T(i) has been read out.
+// shared memory) read it.  Tensor memory that other warps read is reused only after their
+// completion barrier: dP^T(i+1) is issued once dQ^T(i) has been read out.  S^T(i+1), which
+// overwrites the P^T(i) that this thread's own dV(i) reads, follows dV(i) in issue order
+// (FA_BWDQ_INORDER; else it waits for dV(i) to complete).
 // (Compile-time alternatives keep dS^T in tensor memory for dK -- dQ^T then waits for dK -- or
 // stage dQ in the dS^T tile's space.)
 //
