@@ -53,6 +53,13 @@
 #ifndef FA_BWDQ_INORDER
 #define FA_BWDQ_INORDER 1
 #endif
+// FA_BWDQ_DQ_OWN: 1 gives dQ^T its own tensor-memory columns where they are free (d = 64: dV and
+// dK take 64 columns each), so dP^T(i+1) need not wait for dQ^T(i) to be drained; dQ^T(i+1)
+// waits for it instead.  Needs FA_BWDQ_DK_SS (dK reading dS^T from shared memory).  d = 64
+// backward, TFLOP/s: 1x16x8192 causal 596 -> 630, 4x16x2048 causal 405 -> 426.
+#ifndef FA_BWDQ_DQ_OWN
+#define FA_BWDQ_DQ_OWN 1
+#endif
 
 // FA_BWDQ_PIPE_LD: 1 loads the second 32 columns of S^T / dP^T while the first 32 are worked on
 // (one tcgen05.wait::ld covers all of a thread's loads, so the second load is issued after the
@@ -101,7 +108,8 @@ struct BwdQ128Cfg {
   static_assert(2 * 128 * CMP_REGS + 128 * DQ_REGS + 128 * CTRL_REGS <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
   // tensor memory columns
-  static constexpr int T_S = 0, T_DP = 128, T_DQ = 128, T_DV = 256, T_DK = 256 + D;
+  static constexpr bool DQ_OWN = FA_BWDQ_DQ_OWN && FA_BWDQ_DK_SS && D == 64;
+  static constexpr int T_S = 0, T_DP = 128, T_DQ = DQ_OWN ? 384 : 128, T_DV = 256, T_DK = 256 + D;
   static constexpr int TMEM_COLS = 512;
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int OFF_K = 0;
@@ -381,7 +389,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
         // the unit's first S^T into R1 once dV of the previous step has read P^T there, its dP^T
         // into R2 once the previous dQ^T has been drained from it
         if (!FA_BWDQ_INORDER && T > 0 && !(ok = W.wait(BAR_DVD, (T - 1) & 1, 38))) break;
-        if (T > 0 && !(ok = W.wait(BAR_DQE, (T - 1) & 1, 39))) break;
+        if (!C::DQ_OWN && T > 0 && !(ok = W.wait(BAR_DQE, (T - 1) & 1, 39))) break;
         if (!(ok = W.wait(BAR_QF(T & 1), (T >> 1) & 1, 41))) break;
         FA_TRACE_EV(93, T);  // first Q_i landed
         tc_fence_after();
@@ -410,7 +418,10 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
           tc_fence_after();
           if (FA_BWDQ_DK_SS) {
             // dQ_i^T = K_j^T dS^T into R2 (the dP^T columns, read by now), then dK += dS^T Q_i;
-            // both take dS^T from the shared tile
+            // both take dS^T from the shared tile.  With its own columns, dQ^T(t) waits for the
+            // previous one to be drained instead.
+            if (C::DQ_OWN && t > 0 && !(ok = W.wait(BAR_DQE, (t - 1) & 1, 48))) break;
+            if (C::DQ_OWN) tc_fence_after();
             issue_dq();
             tc_commit(BAR_DQF);
             issue_dk_ss(q_addr(s), tl > 0);
@@ -434,7 +445,7 @@ __global__ void __launch_bounds__(BwdQ128Cfg<D>::THREADS, 1)
           if (more) {
             // dP^T(t+1) into R2 once dQ^T(t) has been read out (its statistics operand came with
             // Q_{t+1}, which S^T(t+1) has already waited for)
-            if (!(ok = W.wait(BAR_DQE, t & 1, 48))) break;
+            if (!C::DQ_OWN && !(ok = W.wait(BAR_DQE, t & 1, 48))) break;
             if (!(ok = W.wait(BAR_DOF((t + 1) % DS_), ((t + 1) / DS_) & 1, 49))) break;
             if (!FA_BWDQ_EARLY_S && !(ok = W.wait(BAR_QF((t + 1) & 1), ((t + 1) >> 1) & 1, 45)))
               break;
