@@ -72,6 +72,7 @@ struct BwdParams {
   int Hkv;         // key/value heads per batch (H is a multiple of Hkv)
   int G;           // query heads per key/value head, H / Hkv
   int BHkv;        // batch * key/value heads (CTAs of the main kernels: BHkv x key blocks)
+  int head_band;   // K/V heads per band of the CTA order (0: kBwdHeadBand)
   int gsplit;      // CTAs that share one (key block, key/value head), each taking gq query heads
   int gq;          //   of the group; with gsplit > 1 they add their dK, dV into dk_acc, dv_acc
   float* dk_acc;   // [BHkv, N, D] fp32 (scaled dK), used when gsplit > 1
@@ -131,10 +132,11 @@ struct BwdUnit {
   int j, kvh, gs, slice;
   __device__ __forceinline__ BwdUnit(int x, const BwdParams& p, int nsl) {
     const int per_head = nsl * p.gsplit;  // CTAs per (key block, K/V head)
-    const int band_ctas = kBwdHeadBand * p.nkb * per_head;
+    const int hb = p.head_band > 0 ? p.head_band : kBwdHeadBand;
+    const int band_ctas = hb * p.nkb * per_head;
     const int band = x / band_ctas;
-    const int h0 = band * kBwdHeadBand;
-    const int nh = min(kBwdHeadBand, p.BHkv - h0);
+    const int h0 = band * hb;
+    const int nh = min(hb, p.BHkv - h0);
     const int r = x - band * band_ctas;
     j = r / (nh * per_head);
     const int rem = r - j * (nh * per_head);

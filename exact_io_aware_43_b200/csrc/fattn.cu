@@ -326,6 +326,11 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 #define FA_BWDQ_PERSIST 2
 #endif
 constexpr int kBwdqPersistSteps = 16;
+// K/V heads per band of the unit order on the persistent grid (0: the default band).  Bands of 2
+// measured 4x16x2048 causal 663 -> 696 (d = 128), 418 -> 444 (d = 64), GPT-2 shape 283 -> 294.
+#ifndef FA_BWDQ_PERSIST_BAND
+#define FA_BWDQ_PERSIST_BAND 2
+#endif
 // d = 256 backward: CTA pairs exchanging P and dS through distributed shared memory
 // (fa_bwd_kernel_pair); 0 selects the kernel whose two CTAs per key block each recompute S^T, dP^T.
 #ifndef FA_BWD_PAIR
@@ -383,9 +388,11 @@ int launch_bwd(const void* q, const void* k, const void* v, fattn::BwdParams p, 
     const bool persist =
         FA_BWDQ_PERSIST == 1 || (FA_BWDQ_PERSIST == 2 && steps_max <= kBwdqPersistSteps);
     dim3 grid(unsigned(persist && units > sm_count() ? sm_count() : units));
+    fattn::BwdParams pq = p;
+    if (persist) pq.head_band = FA_BWDQ_PERSIST_BAND;
     {
       TimedLaunch tl(FA_KERNEL_BWD_MAIN, st);
-      kq<<<grid, CQ::THREADS, CQ::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p);
+      kq<<<grid, CQ::THREADS, CQ::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, pq);
     }
   } else if (D == 256 && FA_BWD_PAIR) {
     using CP = fattn::BwdPairCfg;
