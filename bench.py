@@ -67,6 +67,28 @@ def pass_bytes(B, H, Hkv, N, d, forward: bool) -> int:
     return 2 * q + 2 * kv + 2 * rows + q + 2 * kv
 
 
+def binding_roofline(work: float, nbytes: int, avg_ms: float, peaks: dict, peak_src: str) -> dict:
+    """Roofline of one attention kernel launch: `work` FLOP and `nbytes` compulsory HBM bytes in
+    `avg_ms`.  The binding roof is the one with the longer ideal time -- the FLOPs at the tensor
+    peak or the bytes at the copy bandwidth (short sequences are HBM bound, long ones tensor
+    bound); the other is reported beside it."""
+    t_tensor = work / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    tensor = {"bound": "tensor", "achieved": work / (avg_ms * 1e-3) / 1e12,
+              "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+              "peak_source": f"{peak_src} bf16_tflops (burst)"}
+    tensor["frac"] = tensor["achieved"] / tensor["peak"]
+    tensor["frac_of_sustained"] = tensor["achieved"] / peaks.get("bf16_tflops_sustained",
+                                                                 tensor["peak"])
+    hbm = {"bound": "hbm", "achieved": nbytes / (avg_ms * 1e-3) / 1e9,
+           "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs",
+           "algorithmic_bytes": nbytes}
+    hbm["frac"] = hbm["achieved"] / hbm["peak"]
+    roof, other = (hbm, tensor) if t_hbm > t_tensor else (tensor, hbm)
+    roof["other_roof"] = {k: other[k] for k in ("bound", "achieved", "unit", "frac")}
+    return roof
+
+
 def flops(B, H, N, d, causal):
     fwd = 4.0 * B * H * N * N * d * (0.5 if causal else 1.0)
     return fwd, 2.5 * fwd
@@ -435,20 +457,7 @@ def run_gpu(args):
         # the copy bandwidth; short sequences are HBM bound, long ones tensor bound
         work = ff if dom == fa.FA_KERNEL_FWD else fb
         nbytes = pass_bytes(B, H, W.get("H_kv", H), N, d, dom == fa.FA_KERNEL_FWD)
-        t_tensor = work / (peaks["bf16_tflops"] * 1e12)
-        t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-        tensor = {"bound": "tensor", "achieved": work / (avg_ms * 1e-3) / 1e12,
-                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                  "peak_source": f"{peak_src} bf16_tflops (burst)"}
-        tensor["frac"] = tensor["achieved"] / tensor["peak"]
-        tensor["frac_of_sustained"] = tensor["achieved"] / peaks.get("bf16_tflops_sustained",
-                                                                     tensor["peak"])
-        hbm = {"bound": "hbm", "achieved": nbytes / (avg_ms * 1e-3) / 1e9,
-               "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs",
-               "algorithmic_bytes": nbytes}
-        hbm["frac"] = hbm["achieved"] / hbm["peak"]
-        roof, other = (hbm, tensor) if t_hbm > t_tensor else (tensor, hbm)
-        roof["other_roof"] = {k: other[k] for k in ("bound", "achieved", "unit", "frac")}
+        roof = binding_roofline(work, nbytes, avg_ms, peaks, peak_src)
     else:
         nbytes = (B * H * N * d * 2 * 2 + B * H * N * 4 + B * H * N * d * 4 + 2 * B * H * N * 4
                   if dom == fa.FA_KERNEL_BWD_PRE else B * H * N * d * (4 + 2))

@@ -62,3 +62,21 @@ def test_compulsory_bytes_by_hand():
     # grouped heads: K, V (and dK, dV) have H_kv heads
     kv = B * 2 * N * d * 2
     assert bench.pass_bytes(B, H, 2, N, d, True) == 2 * t + 2 * kv + B * H * N * 4
+
+
+def test_binding_roof_is_the_longer_ideal_time():
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0}
+    # long causal backward: 1.374e12 FLOP against 0.6 GB -> tensor bound
+    r = bench.binding_roofline(1.374e12, 600_000_000, 1.4, peaks, "measured")
+    assert r["bound"] == "tensor" and r["other_roof"]["bound"] == "hbm"
+    assert abs(r["achieved"] - 1.374e12 / 1.4e-3 / 1e12) < 1e-9
+    assert abs(r["frac"] - r["achieved"] / 1600.0) < 1e-12
+    assert abs(r["frac_of_sustained"] - r["achieved"] / 1400.0) < 1e-12
+    # a short sequence: little work per byte -> HBM bound, with its algorithmic bytes
+    r = bench.binding_roofline(1.0e10, 200_000_000, 0.05, peaks, "measured")
+    assert r["bound"] == "hbm" and r["algorithmic_bytes"] == 200_000_000
+    assert abs(r["achieved"] - 200_000_000 / 0.05e-3 / 1e9) < 1e-6
+    assert r["other_roof"]["bound"] == "tensor"
+    # the crossover: equal ideal times pick the tensor roof
+    r = bench.binding_roofline(1600e12 * 1e-3, int(6500e9 * 1e-3), 2.0, peaks, "x")
+    assert r["bound"] == "tensor"
